@@ -1,0 +1,322 @@
+"""CPU oracle for the AWQ calibration / scale-search / pack path.
+
+TEST INFRASTRUCTURE. This module is the plain, slow, float64 statement of
+what the path computes; it exists to check the CUDA library. Only the tests,
+``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and reference
+legs may import it. The product path never calls it, and it shares no code
+with the CUDA library (it reads only the bf16 bit patterns the seeded input
+generator produces).
+
+Pages cited (by title and section):
+  [P1] "AWQ量化" tutorial (aiqz.cc): 量化基础 (uniform quantiser), 激活感知
+       (importance Omega_i), 缩放保护 (scale-quantise-restore), 误差分析,
+       GPTQ对比 (AWQ objective).
+  [P2] "AWQ量化技术解析：激活感知的权重量化革命" (kwkr.cn): §2.1 (INT4 clip to
+       [-8, 7], fp16 scale), §4.2 (two 4-bit values per byte).
+  [P3] "大模型的开发应用（十八）：大模型量化：GPTQ与AWQ" (ewbang.com): AWQ 二.2
+       (grid search of alpha on [0, 1]).
+  [P4] "AWQ 量化全流程拆解：将 70B 大模型塞进单张消费级 GPU" (lnrq.cn): §三
+       quant_config (zero_point, q_group_size = 128, w_bit = 4).
+  [P5] "AWQ" (scholia-log, inference-quantization/2_AWQ): §1.1 (Delta Y =
+       Delta W X), §1.2 (a_i = E|x_i|), §2.1 (W X = (W S)(S^-1 X)), §2.3
+       (Q(w) = Delta round(w / Delta)), §3.1-3.3 (worked examples, groups),
+       §4.1 (s_i = a_i^alpha and the boxed objective).
+
+Conventions. W is [d_out, d_in] (rows are output channels), X is [N, d_in]
+(tokens x input channels), so the layer output for token t is W x_t and the
+output error over the calibration set is Delta W X^T. Groups are g consecutive
+input channels within one row. Readings taken where the pages are silent are
+listed with each function.
+
+Every function here is pinned by tests/test_oracle_pins.py against values the
+pages print, closed forms, brute force or invariants; nothing is "parity
+unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+EPS_A = 1e-4       # floor on a_i before the power (dead channels; s_i > 0 required by [P5] §2.1)
+EPS_DELTA = 1e-8   # floor on a group's range (all-equal groups)
+
+_ROW_CHUNK = 1024
+_TOKEN_CHUNK = 8192
+
+
+# ---------------------------------------------------------------------------
+# inputs
+# ---------------------------------------------------------------------------
+def widen_bf16(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> exact float64 values."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# step a1: activation statistics
+# ---------------------------------------------------------------------------
+def act_stats(X_bits: np.ndarray) -> np.ndarray:
+    """a_i = (1/N) sum_t |X[t, i]|.
+
+    [P1] 激活感知: Omega_i is the mean absolute activation of channel i over
+    the N calibration samples; [P5] §1.2: a_i = E[|x_i|]. Summed in float64
+    over token chunks.
+    """
+    N, d_in = X_bits.shape
+    acc = np.zeros(d_in, dtype=np.float64)
+    for t0 in range(0, N, _TOKEN_CHUNK):
+        acc += np.abs(widen_bf16(X_bits[t0:t0 + _TOKEN_CHUNK])).sum(axis=0)
+    return acc / N
+
+
+# ---------------------------------------------------------------------------
+# step a2: candidate scales
+# ---------------------------------------------------------------------------
+def alpha_grid(n_alpha: int) -> np.ndarray:
+    """alpha_k = k / n_alpha, k = 0 .. n_alpha-1 (a grid on [0, 1), [P3] AWQ 二.2)."""
+    return np.arange(n_alpha, dtype=np.float64) / n_alpha
+
+
+def candidate_scales(a: np.ndarray, alpha: float, eps_a: float = EPS_A,
+                     normalise: bool = True) -> np.ndarray:
+    """s_i = max(a_i, eps_a)^alpha, divided by sqrt(max_j s_j * min_j s_j).
+
+    [P5] §4.1: s_i = a_i^alpha, alpha = 0 gives s = 1 (no activation-aware
+    scaling). The sqrt(max * min) normalisation is not on the pages; it is part
+    of the stated task and, since both quantisers are scale-equivariant, it
+    moves the loss only by rounding. Reading: a_i is floored at eps_a before the
+    power so that a dead channel still gets s_i > 0.
+    """
+    t = np.maximum(np.asarray(a, dtype=np.float64), eps_a) ** float(alpha)
+    if not normalise:
+        return t
+    return t / np.sqrt(t.max() * t.min())
+
+
+# ---------------------------------------------------------------------------
+# step a3: group-wise quantiser and fake quantisation
+# ---------------------------------------------------------------------------
+def quantize_groups(V: np.ndarray, bits: int, group: int, symmetric: bool,
+                    eps_delta: float = EPS_DELTA):
+    """Uniform group-wise quantisation of V[rows, d_in] along d_in.
+
+    Returns (V_hat, codes, delta, zero): V_hat the dequantised values, codes
+    the stored unsigned codes (one per element), delta[rows, groups] the step,
+    zero[rows, groups] the stored zero point.
+
+    Symmetric ([P1] 量化基础: q = round(W/s), s = max|W| / (2^(b-1) - 1);
+    [P2] §2.1: clip to [-8, 7] for INT4; [P5] §3.1: Delta = 1/7 for a group
+    maximum of 1 at INT4):
+        Delta = max(max_i |v_i|, eps) / (2^(b-1) - 1)
+        q_i   = clamp(rne(v_i / Delta), -2^(b-1), 2^(b-1) - 1)
+        v_hat = q_i * Delta;  stored code = q_i + 2^(b-1), stored zero = 2^(b-1).
+    Asymmetric with zero point ([P4] §三 zero_point = True; the pages give no
+    formula, this is the min/max affine reading):
+        Delta = max(max v - min v, eps) / (2^b - 1)
+        z     = clamp(rne(-min v / Delta), 0, 2^b - 1)
+        q_i   = clamp(rne(v_i / Delta) + z, 0, 2^b - 1)
+        v_hat = (q_i - z) * Delta.
+    rne = round half to even ([P5] §2.3 "round"; the demo's np.round is
+    half-to-even too).
+    """
+    V = np.asarray(V, dtype=np.float64)
+    rows, d_in = V.shape
+    if d_in % group:
+        raise ValueError("d_in must be a multiple of the group size")
+    G = V.reshape(rows, d_in // group, group)
+    if symmetric:
+        qmax = 2 ** (bits - 1) - 1
+        qmin = -(2 ** (bits - 1))
+        delta = np.maximum(np.abs(G).max(axis=-1), eps_delta) / qmax
+        q = np.clip(np.rint(G / delta[..., None]), qmin, qmax)
+        Vh = q * delta[..., None]
+        codes = (q - qmin).astype(np.int64)
+        zero = np.full(delta.shape, float(-qmin))
+    else:
+        levels = 2 ** bits - 1
+        mx = G.max(axis=-1)
+        mn = G.min(axis=-1)
+        delta = np.maximum(mx - mn, eps_delta) / levels
+        zero = np.clip(np.rint(-mn / delta), 0, levels)
+        q = np.clip(np.rint(G / delta[..., None]) + zero[..., None], 0, levels)
+        Vh = (q - zero[..., None]) * delta[..., None]
+        codes = q.astype(np.int64)
+    return Vh.reshape(rows, d_in), codes.reshape(rows, d_in), delta, zero
+
+
+def fake_quant(W: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool):
+    """W_hat = Q(W S) S^-1 for W[rows, d_in] (float64) and scales s[d_in].
+
+    [P1] 缩放保护: W~_i = s_i W_i, W^_i = Q(W~_i) / s_i; [P5] §2.2: Q(WS)S^-1.
+    Returns (W_hat, codes, delta, zero) with the quantiser of quantize_groups.
+    """
+    s = np.asarray(s, dtype=np.float64)
+    V = W * s[None, :]
+    Vh, codes, delta, zero = quantize_groups(V, bits, group, symmetric)
+    return Vh / s[None, :], codes, delta, zero
+
+
+def delta_weight(W: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool) -> np.ndarray:
+    """Delta W = Q(W S) S^-1 - W, formed before any contraction."""
+    What = fake_quant(W, s, bits, group, symmetric)[0]
+    return What - W
+
+
+# ---------------------------------------------------------------------------
+# steps a4/a5: output error and its squared Frobenius norm
+# ---------------------------------------------------------------------------
+def output_error(dW: np.ndarray, X: np.ndarray) -> np.ndarray:
+    """Delta Y = Delta W X^T ([P5] §1.1 boxed: Delta Y = Delta W X), [rows, N]."""
+    return dW @ X.T
+
+
+def loss_direct(dW: np.ndarray, X_bits: np.ndarray) -> float:
+    """||Delta W X^T||_F^2 = sum_r sum_t (sum_i dW[r,i] X[t,i])^2.
+
+    [P5] §4.1 boxed objective ||W X - Q(WS) S^-1 X||_F^2; [P1] GPTQ对比 writes
+    the same objective as an expectation over x (equal up to the constant 1/N).
+    """
+    return float(row_losses_direct(dW, X_bits).sum())
+
+
+def row_losses_direct(dW: np.ndarray, X_bits: np.ndarray) -> np.ndarray:
+    """Per-row losses l_r = sum_t (sum_i dW[r,i] X[t,i])^2, float64 [rows]."""
+    out = np.zeros(dW.shape[0], dtype=np.float64)
+    for t0 in range(0, X_bits.shape[0], _TOKEN_CHUNK):
+        Xc = widen_bf16(X_bits[t0:t0 + _TOKEN_CHUNK])
+        for r0 in range(0, dW.shape[0], _ROW_CHUNK):
+            D = output_error(dW[r0:r0 + _ROW_CHUNK], Xc)
+            out[r0:r0 + _ROW_CHUNK] += np.einsum("rt,rt->r", D, D)
+    return out
+
+
+def gram(X_bits: np.ndarray) -> np.ndarray:
+    """G = X^T X (float64, [d_in, d_in]); the loss is then sum_r dW_r G dW_r^T."""
+    d_in = X_bits.shape[1]
+    G = np.zeros((d_in, d_in), dtype=np.float64)
+    for t0 in range(0, X_bits.shape[0], _TOKEN_CHUNK):
+        Xc = widen_bf16(X_bits[t0:t0 + _TOKEN_CHUNK])
+        G += Xc.T @ Xc
+    return G
+
+
+def row_losses_gram(dW: np.ndarray, G: np.ndarray) -> np.ndarray:
+    """Per-row losses through the Gram matrix: l_r = dW_r G dW_r^T."""
+    out = np.empty(dW.shape[0], dtype=np.float64)
+    for r0 in range(0, dW.shape[0], _ROW_CHUNK):
+        blk = dW[r0:r0 + _ROW_CHUNK]
+        out[r0:r0 + _ROW_CHUNK] = np.einsum("ri,ri->r", blk @ G, blk)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# steps a2-a6 together: the search
+# ---------------------------------------------------------------------------
+def search(W_bits: np.ndarray, X_bits: np.ndarray, a: np.ndarray, bits: int, group: int,
+           symmetric: bool, n_alpha: int, form: str = "direct", G: np.ndarray | None = None,
+           rows=None):
+    """Loss of every alpha candidate and the chosen one.
+
+    For alpha_k in the grid: s = candidate_scales(a, alpha_k), dW = Q(WS)S^-1 - W,
+    L(alpha_k) = ||dW X^T||_F^2 ([P5] §4.1). k* = argmin_k L, the lowest k on
+    exact ties. ``form`` = "direct" contracts with X, "gram" with G = X^T X (the
+    same sum, reassociated). ``rows`` restricts to a subset of W's rows and then
+    also returns the per-row losses [n_alpha, len(rows)].
+
+    Returns dict(losses[n_alpha] float64, best k, s_best[d_in], alphas,
+    row_losses or None).
+    """
+    alphas = alpha_grid(n_alpha)
+    Wsel = W_bits if rows is None else W_bits[np.asarray(rows)]
+    W = widen_bf16(Wsel)
+    if form == "gram" and G is None:
+        G = gram(X_bits)
+    per_row = np.zeros((n_alpha, W.shape[0]), dtype=np.float64)
+    for k, al in enumerate(alphas):
+        s = candidate_scales(a, al)
+        dW = delta_weight(W, s, bits, group, symmetric)
+        if form == "gram":
+            per_row[k] = row_losses_gram(dW, G)
+        else:
+            per_row[k] = row_losses_direct(dW, X_bits)
+    losses = per_row.sum(axis=1)
+    best = choose(losses)
+    return dict(losses=losses, best=best, s_best=candidate_scales(a, alphas[best]),
+                alphas=alphas, row_losses=per_row if rows is not None else None)
+
+
+def choose(losses: np.ndarray) -> int:
+    """argmin over the grid; the lowest index among exact ties."""
+    losses = np.asarray(losses, dtype=np.float64)
+    return int(np.flatnonzero(losses == losses.min())[0])
+
+
+def acceptable_choices(losses: np.ndarray, rel: float = 0.005) -> list[int]:
+    """Indices whose loss is within ``rel`` (relative) of the minimum: any of
+    them is an acceptable choice when two candidates are that close."""
+    losses = np.asarray(losses, dtype=np.float64)
+    m = losses.min()
+    return [int(k) for k in np.flatnonzero(losses <= m * (1.0 + rel))]
+
+
+# ---------------------------------------------------------------------------
+# step a7: pack
+# ---------------------------------------------------------------------------
+def pack_codes(codes: np.ndarray) -> np.ndarray:
+    """uint32 word w of a row holds codes 8w .. 8w+7, code 8w+j in bits 4j..4j+3.
+
+    [P2] §4.2 stores two 4-bit values per byte; the 8-nibbles-per-uint32 order
+    (lowest input channel in the lowest nibble) is this library's stated
+    layout. 2- and 3-bit codes also take one nibble each.
+    """
+    codes = np.asarray(codes, dtype=np.uint64)
+    rows, d_in = codes.shape
+    if d_in % 8:
+        raise ValueError("d_in must be a multiple of 8")
+    c = codes.reshape(rows, d_in // 8, 8)
+    word = np.zeros((rows, d_in // 8), dtype=np.uint64)
+    for j in range(8):
+        word |= (c[:, :, j] & np.uint64(0xF)) << np.uint64(4 * j)
+    return word.astype(np.uint32)
+
+
+def to_fp16(x: np.ndarray) -> np.ndarray:
+    """float64 -> IEEE binary16, round to nearest even ([P2] §2.1 fp16 scale)."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16)
+
+
+def pack(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool):
+    """Codes of Q(W S) at the chosen scales, packed; fp16 step and zero point.
+
+    Returns (qweight uint32[rows, d_in/8], scales fp16[rows, d_in/g],
+    zeros fp16[rows, d_in/g], codes int64[rows, d_in], delta float64,
+    zero float64). The search uses the float64 step; only the stored copy is
+    rounded to fp16 (reading: the pages give an fp16 scale, [P2] §2.1).
+    """
+    W = widen_bf16(W_bits)
+    _, codes, delta, zero = fake_quant(W, s, bits, group, symmetric)
+    return pack_codes(codes), to_fp16(delta), to_fp16(zero), codes, delta, zero
+
+
+def boundary_mask(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool,
+                  band: float = 1e-4) -> np.ndarray:
+    """Elements whose code the float64 oracle decides within ``band`` of a
+    rounding boundary: v/Delta (or -min/Delta for the zero point of the
+    element's group) lies within ``band`` of a half-integer. A float32
+    computation may round those either way; everything else must match."""
+    W = widen_bf16(W_bits)
+    V = W * np.asarray(s, dtype=np.float64)[None, :]
+    rows, d_in = V.shape
+    G = V.reshape(rows, d_in // group, group)
+    if symmetric:
+        delta = np.maximum(np.abs(G).max(axis=-1), EPS_DELTA) / (2 ** (bits - 1) - 1)
+        r = G / delta[..., None]
+        near = np.abs(r - np.floor(r) - 0.5) < band
+    else:
+        mx, mn = G.max(axis=-1), G.min(axis=-1)
+        delta = np.maximum(mx - mn, EPS_DELTA) / (2 ** bits - 1)
+        r = G / delta[..., None]
+        near = np.abs(r - np.floor(r) - 0.5) < band
+        rz = -mn / delta
+        zn = np.abs(rz - np.floor(rz) - 0.5) < band
+        near |= zn[..., None]
+    return near.reshape(rows, d_in)

@@ -1,0 +1,444 @@
+"""Pins of the CPU oracle to facts fixed outside itself.
+
+Each test ties one oracle function to something the pages print (fixtures in
+tests/golden/ with their citation), a closed form, brute-force enumeration, a
+statistical law, or an invariant of the mathematics, chosen so that a dropped
+term, a wrong sign or index or a transposed operand in the oracle fails one of
+them. No GPU is used.
+"""
+import json
+import math
+import pathlib
+
+import numpy as np
+import pytest
+
+from oracle import awq_oracle as O
+from awq_inputs import WORKLOADS, make_inputs, custom, gen
+
+GOLD = json.loads((pathlib.Path(__file__).parent / "golden" / "p5_worked_examples.json").read_text())
+
+
+def _bits(x):
+    """float64 values that are exact in bf16 -> bf16 bit patterns."""
+    b = gen.f64_to_bf16_bits(np.asarray(x, dtype=np.float64))
+    assert np.array_equal(O.widen_bf16(b), np.asarray(x, dtype=np.float64))
+    return b
+
+
+# ---------------------------------------------------------------------------
+# the pages' worked examples
+# ---------------------------------------------------------------------------
+def test_quantiser_nonlinearity_step_one():
+    """Q(0.4)=0 but Q(0.8)/2=0.5 (AWQ, scholia-log §2.2). A symmetric INT4 group
+    whose largest magnitude is 7 has step exactly 1."""
+    f = GOLD["nonlinearity_step_one"]
+    for w, expect in ((f["w"], f["Q_w"]), (f["w"] * f["s"], f["Q_sw"])):
+        V = np.array([[7.0, w, 0, 0, 0, 0, 0, 0]])
+        Vh, codes, delta, zero = O.quantize_groups(V, 4, 8, True)
+        assert delta[0, 0] == f["step"]
+        assert Vh[0, 1] == expect
+    W = np.array([[7.0, f["w"], 0, 0, 0, 0, 0, 0]])
+    s = np.ones(8)
+    s[1] = f["s"]
+    assert O.fake_quant(W, s, 4, 8, True)[0][0, 1] == f["Q_sw_over_s"]
+    assert O.fake_quant(W, np.ones(8), 4, 8, True)[0][0, 1] == f["Q_w"]
+
+
+def test_int4_group_worked_example():
+    """w_max=1, Delta=1/7, w=0.05, x=10: output error -0.5 unscaled and
+    (1/28 - 0.05)*10 = -1/7 ~ -0.143 with s=4 (AWQ, scholia-log §3.1)."""
+    f = GOLD["int4_group_example"]
+    g, i = 128, 37
+    W = np.zeros((1, g))
+    W[0, 0] = f["w_max"]
+    W[0, i] = f["w_i"]
+    X = np.zeros((1, g))
+    X[0, i] = f["x_i"]
+    _, codes, delta, _ = O.quantize_groups(W, f["bits"], g, True)
+    assert delta[0, 0] == pytest.approx(f["delta"], rel=1e-15)
+    assert abs(delta[0, 0] - f["delta_printed"]) < 5e-4
+    assert codes[0, i] - 8 == f["unscaled_code"]
+    dy = O.output_error(O.delta_weight(W, np.ones(g), 4, g, True), X)[0, 0]
+    assert dy == pytest.approx(f["unscaled_dy"], abs=1e-15)
+
+    s = np.ones(g)
+    s[i] = f["s_i"]
+    V = W * s
+    assert V[0, i] == pytest.approx(f["scaled_w"])
+    assert f["x_i"] / f["s_i"] == f["scaled_x"]
+    Vh, codes, delta, _ = O.quantize_groups(V, 4, g, True)
+    assert delta[0, 0] == pytest.approx(f["delta"], rel=1e-15)   # group max unchanged
+    assert abs(V[0, i] / delta[0, 0] - f["scaled_ratio_printed"]) < 5e-3
+    assert codes[0, i] - 8 == f["scaled_code"]
+    assert abs((Vh[0, i] - V[0, i]) - f["scaled_weight_error_printed"]) < 5e-4
+    dy4 = O.output_error(O.delta_weight(W, s, 4, g, True), X)[0, 0]
+    assert dy4 == pytest.approx((1.0 / 28.0 - 0.05) * 10.0, rel=1e-12)
+    assert abs(dy4 - f["scaled_dy_printed"]) < 5e-4
+    assert abs(delta[0, 0] / s[i] - f["delta_eff_printed"]) < 5e-4
+
+
+def test_range_expansion_example():
+    """s=40 makes 0.05 -> 2 the group maximum; step 2/7 (AWQ, scholia-log §3.3)."""
+    f = GOLD["range_expansion"]
+    g, i = 128, 3
+    W = np.zeros((1, g))
+    W[0, 0] = f["w_max"]
+    W[0, i] = f["w_i"]
+    s = np.ones(g)
+    s[i] = f["s_i"]
+    _, _, delta, _ = O.quantize_groups(W * s, f["bits"], g, True)
+    assert (W * s)[0, i] == pytest.approx(f["scaled_w"])
+    assert delta[0, 0] == pytest.approx(f["delta"], rel=1e-15)
+    assert abs(delta[0, 0] - f["delta_printed"]) < 5e-4
+
+
+def test_output_error_products():
+    """Delta Y = Delta W X for single products (AWQ, scholia-log §1.1)."""
+    for dw, x, dy in GOLD["output_error_products"]["cases"]:
+        assert O.output_error(np.array([[dw]]), np.array([[x]]))[0, 0] == pytest.approx(dy, rel=1e-12)
+
+
+def test_output_error_orientation():
+    """Delta W [rows, d_in] times X [N, d_in] gives [rows, N], entry (r, t) =
+    sum_i dW[r,i] X[t,i]: checked on index-coded matrices (a transposed operand
+    or swapped index fails)."""
+    dW = np.arange(6, dtype=np.float64).reshape(2, 3)          # 2 rows, 3 channels
+    X = 10.0 ** np.arange(12, dtype=np.float64).reshape(4, 3)  # 4 tokens
+    D = O.output_error(dW, X)
+    assert D.shape == (2, 4)
+    for r in range(2):
+        for t in range(4):
+            assert D[r, t] == sum(dW[r, i] * X[t, i] for i in range(3))
+
+
+# ---------------------------------------------------------------------------
+# the quantiser: bounds, brute force, statistics
+# ---------------------------------------------------------------------------
+def _random_groups(rng, rows, g, mixed=True):
+    V = rng.standard_normal((rows, g))
+    if mixed:
+        V[:, 0] = -np.abs(V[:, 0]) - 0.01
+        V[:, 1] = np.abs(V[:, 1]) + 0.01
+    return V
+
+
+@pytest.mark.parametrize("bits,sym", [(4, False), (4, True), (3, True), (3, False), (2, False)])
+def test_rounding_error_bound(bits, sym):
+    """|v_hat - v| <= Delta/2 wherever no clipping applies ([P5] §2.3):
+    symmetric grids always cover [-max|v|, max|v|]; asymmetric grids cover the
+    group's range when it contains 0."""
+    rng = np.random.default_rng(1)
+    V = _random_groups(rng, 4000, 64)
+    Vh, codes, delta, zero = O.quantize_groups(V, bits, 64, sym)
+    err = np.abs(Vh - V)
+    assert np.all(err <= delta.repeat(64, axis=1) * (0.5 + 1e-12))
+
+
+def test_asymmetric_clips_one_signed_groups():
+    """A group with all values positive has zero point 0; values beyond 15*Delta
+    clip to code 15 (the range is not forced to include 0)."""
+    V = np.linspace(1.0, 2.0, 16)[None, :]
+    Vh, codes, delta, zero = O.quantize_groups(V, 4, 16, False)
+    assert zero[0, 0] == 0
+    assert delta[0, 0] == pytest.approx(1.0 / 15.0)
+    assert codes.max() == 15 and codes.min() == 15
+    assert Vh[0, -1] == pytest.approx(1.0)
+
+
+@pytest.mark.parametrize("bits,sym", [(4, False), (3, True), (4, True), (3, False)])
+def test_brute_force_codes(bits, sym):
+    """For each element, the code is the one of all 2^b codes whose
+    dequantised value is nearest to v (exact ties excluded), and the zero point
+    is the integer in range nearest to -min/Delta."""
+    rng = np.random.default_rng(2)
+    g = 16
+    V = _random_groups(rng, 300, g, mixed=False) * rng.uniform(0.1, 3.0, (300, 1))
+    Vh, codes, delta, zero = O.quantize_groups(V, bits, g, sym)
+    n = 2 ** bits
+    for r in range(V.shape[0]):
+        d, z = delta[r, 0], zero[r, 0]
+        offs = 2 ** (bits - 1) if sym else z
+        if not sym:
+            cand_z = np.arange(n)
+            dist = np.abs(-cand_z * d - V[r].min())
+            assert z == cand_z[np.argmin(dist)]
+        for i in range(g):
+            cands = (np.arange(n) - offs) * d
+            dist = np.abs(cands - V[r, i])
+            order = np.argsort(dist)
+            if dist[order[1]] - dist[order[0]] < 1e-12:
+                continue
+            assert codes[r, i] == order[0]
+            assert Vh[r, i] == pytest.approx(cands[order[0]], abs=1e-15)
+
+
+def test_symmetric_step_closed_form():
+    """Symmetric step = max|v| / (2^(b-1) - 1) ([P1] 量化基础); 1/7 for a group
+    maximum of 1 at INT4 and 1/3 at INT3; the -2^(b-1) code is never used."""
+    V = np.array([[1.0, -0.5, 0.25, 0.0, 0.3, -0.9, 0.1, 0.2]])
+    assert O.quantize_groups(V, 4, 8, True)[2][0, 0] == pytest.approx(1 / 7, rel=1e-15)
+    assert O.quantize_groups(-V, 3, 8, True)[2][0, 0] == pytest.approx(1 / 3, rel=1e-15)
+    rng = np.random.default_rng(3)
+    for bits in (3, 4):
+        codes = O.quantize_groups(rng.standard_normal((2000, 64)), bits, 64, True)[1]
+        assert codes.min() >= 1
+
+
+def test_asymmetric_zero_point_cases():
+    """A range symmetric about 0 at INT4 (min=-7.5, max=7.5): Delta=1, z=rne(7.5)=8;
+    a range starting at 0: z=0 and code = v/Delta."""
+    V = np.array([[-7.5, 7.5, 0.0, 1.0]])
+    _, codes, delta, zero = O.quantize_groups(V, 4, 4, False)
+    assert delta[0, 0] == 1.0 and zero[0, 0] == 8
+    assert list(codes[0]) == [0, 15, 8, 9]
+    V = np.array([[0.0, 1.5, 3.0, 0.2]])
+    _, codes, delta, zero = O.quantize_groups(V, 4, 4, False)
+    assert zero[0, 0] == 0 and delta[0, 0] == pytest.approx(0.2)
+    assert list(codes[0]) == [0, 8, 15, 1]
+
+
+def test_degenerate_groups():
+    """An all-zero group dequantises to exact zeros; an all-equal group too
+    (the range floor keeps Delta > 0)."""
+    V = np.zeros((2, 8))
+    V[1] = 0.0
+    for sym in (True, False):
+        Vh, codes, delta, zero = O.quantize_groups(V, 4, 8, sym)
+        assert np.all(Vh == 0.0) and np.all(delta > 0)
+
+
+def test_uniform_error_variance():
+    """Mean squared rounding error ~ Delta^2/12 ([P1] 误差分析) on 10^6 weights.
+    Each group's extremes fix its grid, so the law is checked on the other
+    elements, which fall uniformly within their cells."""
+    rng = np.random.default_rng(4)
+    V = rng.uniform(-1, 1, (8192, 128)) + rng.uniform(-0.5, 0.5, (8192, 1))
+    for sym in (False, True):
+        Vh, _, delta, _ = O.quantize_groups(V, 4, 128, sym)
+        e2 = (Vh - V) ** 2 / (delta.repeat(128, axis=1) ** 2 / 12.0)
+        order = np.argsort(V, axis=1)
+        inner = np.take_along_axis(e2, order[:, 1:-1], axis=1)
+        assert abs(inner.mean() - 1.0) < 0.01
+
+
+def test_protected_channel_error_shrinks_by_s_squared():
+    """Scaling one channel by s (without changing its group's range) divides
+    that channel's restored error variance by s^2 ([P1] 误差分析,
+    E_protected ~ (s_q/s_i)^2/12; [P5] §2.3 Delta_eff = Delta'/s)."""
+    rng = np.random.default_rng(5)
+    W = rng.uniform(-1, 1, (100000, 32))
+    W[:, 0] = 1.0
+    W[:, 1] = -1.0
+    W[:, 2] = rng.uniform(-0.2, 0.2, 100000)
+    base = O.fake_quant(W, np.ones(32), 4, 32, False)
+    s = np.ones(32)
+    s[2] = 3.0
+    prot = O.fake_quant(W, s, 4, 32, False)
+    d = base[2][:, 0]
+    e0 = np.mean((base[0][:, 2] - W[:, 2]) ** 2 / (d ** 2 / 12))
+    e1 = np.mean((prot[0][:, 2] - W[:, 2]) ** 2 / (d ** 2 / 12))
+    assert abs(e0 - 1.0) < 0.02
+    assert abs(e1 * 9.0 - 1.0) < 0.02
+
+
+# ---------------------------------------------------------------------------
+# statistics and scales
+# ---------------------------------------------------------------------------
+def test_act_stats_closed_form():
+    """a_i = mean_t |X[t,i]| ([P1] 激活感知, [P5] §1.2): alternating signs of a
+    per-channel magnitude give exactly that magnitude."""
+    c = np.array([0.5, 1.0, 3.0, 0.0, 40.0, 0.125, 2.0, 7.0])
+    X = np.array([(-1.0) ** t * c for t in range(6)])
+    a = O.act_stats(_bits(X))
+    assert np.array_equal(a, c)
+    X2 = np.array([[1.0, 2.0], [3.0, -6.0], [0.0, 1.0]])
+    assert np.allclose(O.act_stats(_bits(X2)), [4.0 / 3.0, 3.0], rtol=1e-15)
+
+
+def test_act_stats_half_normal_mean():
+    """For N(0,1) activations, E|x| = sqrt(2/pi)."""
+    W, X = make_inputs(WORKLOADS["C1"])
+    a = O.act_stats(X)
+    outl = gen.pick_channels(WORKLOADS["C1"].seed, 512, 5)
+    mask = np.ones(512, bool)
+    mask[outl] = False
+    assert abs(a[mask].mean() - math.sqrt(2 / math.pi)) < 0.01
+    assert abs(a[outl].mean() / math.sqrt(2 / math.pi) - 20.0) < 1.0
+
+
+def test_candidate_scales_closed_forms():
+    a = np.array([1.0, 4.0, 2.0])
+    assert np.array_equal(O.candidate_scales(a, 0.0), np.ones(3))   # alpha=0: no scaling ([P5] §4.1)
+    for al in (0.25, 0.5, 0.95):
+        s = O.candidate_scales(a, al)
+        # normalisation: max(s) * min(s) = 1, so s = a^alpha / sqrt(4^alpha)
+        assert s.max() * s.min() == pytest.approx(1.0, rel=1e-14)
+        assert np.allclose(s, a ** al / 2.0 ** al, rtol=1e-14)
+        assert np.allclose(O.candidate_scales(a, al, normalise=False), a ** al, rtol=1e-15)
+    # the floor keeps dead channels positive
+    s = O.candidate_scales(np.array([0.0, 1.0]), 0.5, normalise=False)
+    assert s[0] == pytest.approx(1e-2) and s[1] == 1.0
+    assert np.allclose(O.alpha_grid(20), [k / 20 for k in range(20)])
+
+
+def test_scale_equivariance_of_normalisation():
+    """Q(cV) = c Q(V) for c a power of two, so multiplying every s_i by c leaves
+    Q(WS)S^-1 bit-identical; the sqrt(max*min) normalisation therefore only
+    changes the loss by float64 rounding."""
+    W, X = make_inputs(WORKLOADS["C1"])
+    Wf = O.widen_bf16(W)
+    a = O.act_stats(X)
+    for sym, bits, g in ((False, 4, 128), (True, 3, 64)):
+        s = O.candidate_scales(a, 0.6)
+        ref = O.fake_quant(Wf, s, bits, g, sym)
+        for c in (0.25, 8.0):
+            got = O.fake_quant(Wf, c * s, bits, g, sym)
+            assert np.array_equal(got[0], ref[0]) and np.array_equal(got[1], ref[1])
+        l_norm = O.loss_direct(ref[0] - Wf, X)
+        su = O.candidate_scales(a, 0.6, normalise=False)
+        l_raw = O.loss_direct(O.fake_quant(Wf, su, bits, g, sym)[0] - Wf, X)
+        assert l_norm == pytest.approx(l_raw, rel=1e-9)
+
+
+def test_identity_without_quantisation():
+    """(W S)(S^-1 X^T) = W X^T for positive s, to float64 rounding ([P5] §2.1)."""
+    rng = np.random.default_rng(6)
+    W = rng.standard_normal((16, 64))
+    X = rng.standard_normal((32, 64))
+    s = O.candidate_scales(rng.uniform(0.01, 50, 64), 0.7)
+    lhs = O.output_error(W * s, X / s)
+    rhs = O.output_error(W, X)
+    assert np.allclose(lhs, rhs, rtol=1e-13, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# the search: special cases, brute force, reassociation
+# ---------------------------------------------------------------------------
+def _rtn_reference(W, bits, g):
+    """Plain asymmetric round-to-nearest per group, written with scalar loops."""
+    rows, d_in = W.shape
+    out = np.zeros_like(W)
+    levels = 2 ** bits - 1
+    for r in range(rows):
+        for g0 in range(0, d_in, g):
+            grp = [float(v) for v in W[r, g0:g0 + g]]
+            lo, hi = min(grp), max(grp)
+            step = max(hi - lo, 1e-8) / levels
+            zp = min(max(round(-lo / step), 0), levels)
+            for j, v in enumerate(grp):
+                q = min(max(round(v / step) + zp, 0), levels)
+                out[r, g0 + j] = (q - zp) * step
+    return out
+
+
+def test_alpha_zero_is_plain_rtn():
+    """alpha = 0 gives s = 1, so the candidate is plain group RTN of W
+    ([P5] §4.1)."""
+    wl = custom(8, 256, 16, seed=11)
+    W, X = make_inputs(wl)
+    a = O.act_stats(X)
+    Wf = O.widen_bf16(W)
+    s0 = O.candidate_scales(a, 0.0)
+    assert np.array_equal(s0, np.ones(256))
+    What = O.fake_quant(Wf, s0, 4, 128, False)[0]
+    assert np.array_equal(What, _rtn_reference(Wf, 4, 128))
+    res = O.search(W, X, a, 4, 128, False, 20)
+    dW = What - Wf
+    brute = sum(sum(sum(dW[r, i] * float(xv) for i, xv in enumerate(O.widen_bf16(X)[t])) ** 2
+                    for t in range(16)) for r in range(8))
+    assert res["losses"][0] == pytest.approx(brute, rel=1e-12)
+
+
+@pytest.mark.parametrize("sym,bits", [(False, 4), (True, 3)])
+def test_brute_force_loss_tiny(sym, bits):
+    """d_out=2, d_in=g=8, N=3: the loss for each alpha equals a triple loop over
+    (row, token, channel) with the dequantised weights found by enumerating
+    every code."""
+    rng = np.random.default_rng(7)
+    W = _bits(O.widen_bf16(gen.f64_to_bf16_bits(rng.standard_normal((2, 8)) * 0.05)))
+    X = _bits(O.widen_bf16(gen.f64_to_bf16_bits(rng.standard_normal((3, 8)) * np.array([1, 1, 9, 1, 1, 1, 2, 1]))))
+    Wf, Xf = O.widen_bf16(W), O.widen_bf16(X)
+    a = np.abs(Xf).mean(axis=0)
+    res = O.search(W, X, O.act_stats(X), bits, 8, sym, 5)
+    for k, al in enumerate(O.alpha_grid(5)):
+        s = O.candidate_scales(a, al)
+        total = 0.0
+        for r in range(2):
+            v = Wf[r] * s
+            if sym:
+                d = np.abs(v).max() / (2 ** (bits - 1) - 1)
+                grid = np.arange(-(2 ** (bits - 1)), 2 ** (bits - 1)) * d
+            else:
+                d = (v.max() - v.min()) / (2 ** bits - 1)
+                z = min(range(2 ** bits), key=lambda c: abs(c * d + v.min()))
+                grid = (np.arange(2 ** bits) - z) * d
+            vh = np.array([grid[np.argmin(np.abs(grid - x))] for x in v])
+            dw = vh / s - Wf[r]
+            for t in range(3):
+                total += sum(dw[i] * Xf[t, i] for i in range(8)) ** 2
+        assert res["losses"][k] == pytest.approx(total, rel=1e-12)
+
+
+def test_direct_and_gram_forms_agree():
+    """||dW X^T||_F^2 = sum_r dW_r (X^T X) dW_r^T, to float64 rounding."""
+    W, X = make_inputs(WORKLOADS["C1"])
+    a = O.act_stats(X)
+    d = O.search(W, X, a, 4, 128, False, 20, form="direct")
+    g = O.search(W, X, a, 4, 128, False, 20, form="gram")
+    assert np.allclose(d["losses"], g["losses"], rtol=1e-12)
+    assert d["best"] == g["best"]
+    rows = [0, 5, 255]
+    sub = O.search(W, X, a, 4, 128, False, 20, rows=rows)
+    full_rows = O.search(W[rows], X, a, 4, 128, False, 20)
+    assert np.allclose(sub["row_losses"].sum(axis=1), full_rows["losses"], rtol=1e-13)
+
+
+def test_choice_rules():
+    assert O.choose(np.array([3.0, 1.0, 1.0, 2.0])) == 1
+    assert O.acceptable_choices(np.array([3.0, 1.0, 1.004, 1.006])) == [1, 2]
+
+
+def test_search_prefers_scaling_on_outlier_layer():
+    """Expected direction (not a fixed value): with outlier channels the best
+    alpha beats plain RTN (alpha = 0) on C1."""
+    W, X = make_inputs(WORKLOADS["C1"])
+    res = O.search(W, X, O.act_stats(X), 4, 128, False, 20)
+    assert res["best"] > 0
+    assert res["losses"][res["best"]] < res["losses"][0]
+
+
+# ---------------------------------------------------------------------------
+# pack
+# ---------------------------------------------------------------------------
+def test_pack_nibble_order():
+    codes = np.array([[0, 1, 2, 3, 4, 5, 6, 7, 15, 15, 15, 15, 15, 15, 15, 15]])
+    words = O.pack_codes(codes)
+    assert words.dtype == np.uint32
+    assert list(words[0]) == [0x76543210, 0xFFFFFFFF]
+    for j in range(8):
+        c = np.zeros((1, 8), dtype=np.int64)
+        c[0, j] = 1
+        assert O.pack_codes(c)[0, 0] == 1 << (4 * j)
+
+
+def test_fp16_rounding_is_nearest_even():
+    assert O.to_fp16(1.0 + 2.0 ** -11) == 1.0
+    assert O.to_fp16(1.0 + 3 * 2.0 ** -11) == 1.0 + 2.0 ** -9
+    assert O.to_fp16(1.0 + 2.0 ** -11 + 2.0 ** -30) == 1.0 + 2.0 ** -10
+
+
+def test_pack_layer_consistency():
+    """Unpacking the words, and dequantising with the float64 step and zero,
+    reproduces Q(WS) for every element."""
+    W, X = make_inputs(WORKLOADS["C1"])
+    a = O.act_stats(X)
+    s = O.candidate_scales(a, 0.45)
+    qw, sc, zr, codes, delta, zero = O.pack(W, s, 4, 128, False)
+    assert qw.shape == (256, 64) and sc.shape == (256, 4) and sc.dtype == np.float16
+    unpacked = np.stack([(qw >> np.uint32(4 * j)) & np.uint32(0xF) for j in range(8)], axis=-1).reshape(256, 512)
+    assert np.array_equal(unpacked, codes)
+    Vh = (codes - zero.repeat(128, axis=1)) * delta.repeat(128, axis=1)
+    ref = O.fake_quant(O.widen_bf16(W), s, 4, 128, False)[0] * s
+    assert np.allclose(Vh, ref, rtol=1e-14, atol=1e-18)
+    assert np.array_equal(zr.astype(np.float64), zero)
