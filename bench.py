@@ -1,0 +1,423 @@
+"""Benchmark of the AWQ calibration / scale-search path on B200.
+
+One step = the whole hot path for one linear layer: activation statistics,
+candidate scales, the fake-quantised dW stack, (Gram product,) the tensor-core
+error contraction with its fused squared-sum epilogue, the fixed-order
+reduction with argmin, and the pack at the chosen scales.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C2] [--impl ours|reference]
+
+Prints one JSON line (rank 0). The metric is alpha-candidate layer
+evaluations per second (n_alpha / step time, summed over ranks); under
+torchrun every rank runs its own replica of the layer ("replicas only": the
+path has no exchange step). `--impl reference` times the CPU oracle on a
+bounded row sample of the same layer instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from awq_inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "AWQ search: alpha-candidate layer evals/s, TFLOP/s vs bf16 peak; stats GB/s"
+UNIT = "alpha-candidate layer evals/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("gemm_sm100.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "weight_only_int4_act_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config_key, form):
+    """Per-launch DRAM bytes of the contraction from the committed ncu summary,
+    if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"contract_{form}_{config_key}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm = [float(r[1]) for r in self.rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows if len(r) >= 9 for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sm)}
+
+
+def launches_per_step(form):
+    # stats 2 + scales 1 + fake-quant 1 + (transpose + Gram 2) + contraction 1 + reduce 2 + pack 1
+    return 8 + (2 if form == "gram" else 0)
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import weight_only_int4_act_b200 as awq
+    from weight_only_int4_act_b200 import binding as B
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.config]
+    Wb, Xb = make_inputs(wl)
+    d_out, d_in, N = wl.d_out, wl.d_in, wl.N
+    W = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).to(dev)
+    X = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).to(dev)
+    cfg = awq.make_cfg(wl.bits, wl.group, wl.symmetric, wl.n_alpha, form=args.form)
+    form = awq.search_form(d_out, d_in, N, cfg)
+    ws = awq.workspace(awq.search_workspace_size(d_out, d_in, N, cfg))
+    ws_stats = awq.workspace(awq.stats_workspace_size(N, d_in))
+    a = torch.empty(d_in, dtype=torch.float32, device=dev)
+    outs = dict(losses=torch.empty(wl.n_alpha, dtype=torch.float32, device=dev),
+                best=torch.empty(1, dtype=torch.int32, device=dev),
+                s_best=torch.empty(d_in, dtype=torch.float32, device=dev), row_losses=None)
+    ng = d_in // wl.group
+    packed = (torch.empty((d_out, d_in // 8), dtype=torch.int32, device=dev),
+              torch.empty((d_out, ng), dtype=torch.float16, device=dev),
+              torch.empty((d_out, ng), dtype=torch.float16, device=dev))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    L = B.lib()
+    import ctypes
+    cptr = ctypes.byref(cfg)
+    wsp, wsn = ctypes.c_void_p(ws.data_ptr()), ws.numel()
+
+    def step(ev=None):
+        st = B._stream()
+        if ev is not None:
+            ev[0].record()
+        awq.act_stats(X, ws_stats, out=a)
+        if ev is not None:
+            ev[1].record()
+        B._check(L.awq_step_scales(ctypes.c_void_p(a.data_ptr()), d_out, d_in, N, cptr, wsp, wsn, st), "scales")
+        B._check(L.awq_step_fake_quant(ctypes.c_void_p(W.data_ptr()), d_out, d_in, N, cptr, wsp, wsn, st), "fq")
+        if ev is not None:
+            ev[2].record()
+        B._check(L.awq_step_gram(ctypes.c_void_p(X.data_ptr()), d_out, d_in, N, cptr, wsp, wsn, st), "gram")
+        if ev is not None:
+            ev[3].record()
+        B._check(L.awq_step_contract(ctypes.c_void_p(X.data_ptr()), d_out, d_in, N, cptr, wsp, wsn, st), "contract")
+        if ev is not None:
+            ev[4].record()
+        B._check(L.awq_step_reduce(d_out, d_in, N, cptr, wsp, wsn, ctypes.c_void_p(outs["losses"].data_ptr()),
+                                   ctypes.c_void_p(outs["best"].data_ptr()),
+                                   ctypes.c_void_p(outs["s_best"].data_ptr()), None, st), "reduce")
+        if ev is not None:
+            ev[5].record()
+        awq.quantize_pack(W, outs["s_best"], cfg, outputs=packed)
+        if ev is not None:
+            ev[6].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    awq.workspace_error(ws)
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    t_wall0 = time.perf_counter()
+    for k in range(K):
+        flush.fill_(k & 0xFF)  # evict L2 between timed steps (outside the step's events)
+        step(evs[k])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_wall = time.perf_counter() - t_wall0
+    clk = clocks.stop()
+    awq.workspace_error(ws)
+
+    seg = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(6)] for k in range(K)])  # ms
+    step_ms = seg.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    mean = seg.mean(axis=0)
+    names = ["stats", "scales+fake_quant", "gram", "contraction", "reduce_argmin", "pack"]
+    breakdown = {n: round(float(v), 4) for n, v in zip(names, mean)}
+
+    # ---- end to end through the public API with host buffers
+    Wh = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Xh = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in
+                (outs["losses"], outs["best"], outs["s_best"], *packed)]
+    Wd = torch.empty_like(W)
+    Xd = torch.empty_like(X)
+
+    def e2e_step():
+        Wd.copy_(Wh, non_blocking=True)
+        Xd.copy_(Xh, non_blocking=True)
+        aa = awq.act_stats(Xd, ws_stats, out=a)
+        r = awq.search_scales(Wd, Xd, aa, cfg, ws=ws, outputs=outs)
+        p = awq.quantize_pack(Wd, r["s_best"], cfg, outputs=packed)
+        for h, d in zip(host_out, (r["losses"], r["best"], r["s_best"], *p)):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_ms = []
+    for k in range(K):
+        flush.fill_(k & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        e2e_step()
+        e1.record()
+        e1.synchronize()
+        e_ms.append(e0.elapsed_time(e1))
+    e2e_total = float(sum(e_ms))
+    if world > 1:
+        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    awq.workspace_error(ws)
+    h2d = Wb.nbytes + Xb.nbytes
+    d2h = sum(h.numel() * h.element_size() for h in host_out)
+
+    peaks = load_peaks()
+    n_a = wl.n_alpha
+    flops_direct = 2.0 * n_a * d_out * d_in * N
+    flops_search = flops_direct if form == "direct" else 2.0 * n_a * d_out * d_in * d_in
+    flops_gram = 0.0 if form == "direct" else 2.0 * N * d_in * d_in
+    c_ms = breakdown["contraction"]
+    achieved_tflops = flops_search / (c_ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    stats_bytes = N * d_in * 2 + d_in * 4
+    pack_bytes = d_out * d_in * 2 + d_out * d_in // 2 + 2 * 2 * d_out * (d_in // wl.group) + d_in * 4
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    stats_gbs = stats_bytes / (breakdown["stats"] * 1e-3) / 1e9
+    pack_gbs = pack_bytes / (breakdown["pack"] * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC,
+        "value": round(world * n_a / (ms_per_step * 1e-3), 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.key}: {wl.title}", "d_out": d_out, "d_in": d_in, "N": N, "bits": wl.bits,
+                   "group": wl.group, "symmetric": wl.symmetric, "n_alpha": n_a, "form": form,
+                   "l2": "flushed: 256 MiB write between timed steps, outside the step events",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"kernel": f"gemm_bf16_tcgen05 ({'sum of squares' if form == 'direct' else 'Gram dot'} epilogue)",
+                     "bound": "tensor", "achieved": round(achieved_tflops, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
+                     "peak_kind": f"bf16 sustained ({peaks.get('source')})",
+                     "traffic": profiled_traffic(wl.key, form),
+                     "algorithmic_flops_per_launch": flops_search},
+        "breakdown_ms": breakdown,
+        "stats_gbs": round(stats_gbs, 1), "stats_hbm_frac": round(stats_gbs / hbm, 4),
+        "pack_gbs": round(pack_gbs, 1), "pack_hbm_frac": round(pack_gbs / hbm, 4),
+        "gram_tflops": round(flops_gram / (breakdown["gram"] * 1e-3) / 1e12, 2) if flops_gram else None,
+        "candidate_weight_evals_per_s": round(world * n_a * d_out * d_in / (ms_per_step * 1e-3), 1),
+        "layers_per_s": round(world / (ms_per_step * 1e-3), 3),
+        "e2e": {"value": round(world * n_a * K / (e2e_total * 1e-3), 2), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": launches_per_step(form) * K,
+        "clocks": clk,
+        "wall_s_timed_region": round(t_wall, 3),
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, rows_total, block=256):
+    """Time the CPU oracle on a bounded sample of one layer: the full
+    statistics, the search on `rows_total` rows (the per-row cost is uniform)
+    and their pack; extrapolated to the whole layer."""
+    from oracle import awq_oracle as O
+    Wb, Xb = make_inputs(wl)
+    t0 = time.perf_counter()
+    a = O.act_stats(Xb)
+    t_stats = time.perf_counter() - t0
+    rows_total = min(rows_total, wl.d_out)
+    t_search = 0.0
+    t_pack = 0.0
+    for r0 in range(0, rows_total, block):
+        rows = np.arange(r0, min(rows_total, r0 + block))
+        t0 = time.perf_counter()
+        res = O.search(Wb, Xb, a, wl.bits, wl.group, wl.symmetric, wl.n_alpha, rows=rows)
+        t_search += time.perf_counter() - t0
+        t0 = time.perf_counter()
+        O.pack(Wb[rows], res["s_best"], wl.bits, wl.group, wl.symmetric)
+        t_pack += time.perf_counter() - t0
+    scale = wl.d_out / rows_total
+    t_layer = t_stats + (t_search + t_pack) * scale
+    return t_layer, rows_total, t_stats + t_search + t_pack
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("internal_api") == "openblas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline_entry(wl, rows):
+    t_layer, r, spent = oracle_sample(wl, rows)
+    return {"value": round(wl.n_alpha / t_layer, 4), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{wl.key}: full statistics + search and pack of {r} of {wl.d_out} rows x {wl.n_alpha} alphas "
+                      f"(float64 numpy, BLAS matmul), extrapolated by rows; {spent:.1f} s of CPU work"}
+
+
+def run_reference(args, wl):
+    K = args.steps
+    times = []
+    rows = args.ref_rows
+    for k in range(args.warmup + K):
+        t_layer, r, _ = oracle_sample(wl, rows)
+        if k >= args.warmup:
+            times.append(t_layer)
+    ms = 1e3 * sum(times) / K
+    value = wl.n_alpha / (ms * 1e-3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{wl.key}: {wl.title}", "d_out": wl.d_out, "d_in": wl.d_in, "N": wl.N},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"per step: full statistics + search and pack of {min(rows, wl.d_out)} of "
+                                   f"{wl.d_out} rows, extrapolated by rows"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="C2", choices=sorted(WORKLOADS))
+    ap.add_argument("--form", default="auto", choices=["auto", "direct", "gram"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = WORKLOADS[args.config]
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, wl)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline_entry(wl, args.cpu_rows)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

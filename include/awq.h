@@ -1,0 +1,164 @@
+/*
+ * awq.h - C ABI of the B200 (sm_100a) library for the AWQ calibration and
+ * scale-search path of one linear layer.
+ *
+ * The operations follow these pages (cited by title and section):
+ *   [P1] "AWQ量化" tutorial (aiqz.cc): 量化基础, 激活感知, 缩放保护, GPTQ对比.
+ *   [P2] "AWQ量化技术解析：激活感知的权重量化革命" (kwkr.cn): §2.1, §4.2.
+ *   [P3] "大模型的开发应用（十八）：大模型量化：GPTQ与AWQ" (ewbang.com): AWQ 二.2.
+ *   [P4] "AWQ 量化全流程拆解：将 70B 大模型塞进单张消费级 GPU" (lnrq.cn): §三.
+ *   [P5] "AWQ" (scholia-log, inference-quantization/2_AWQ): §1.1, §1.2, §2.1-2.3,
+ *        §3.1-3.3, §4.1.
+ *
+ * Conventions for every entry point:
+ *   - W is bf16 [d_out, d_in], row-major (rows are output channels).
+ *   - X is bf16 [N, d_in], row-major (N calibration tokens x input channels).
+ *   - Groups are g consecutive input channels within one row of W.
+ *   - Every pointer argument is DEVICE memory owned by the caller, unless the
+ *     comment says "host". The library allocates nothing and keeps no global
+ *     state; scratch memory is the caller's workspace.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream). A returned AWQ_OK means the work was
+ *     validated and enqueued. Errors the device finds (a wait that timed out,
+ *     non-finite losses) are written to a word in the workspace and read back
+ *     by awq_workspace_error().
+ *   - Argument and shape errors are returned before anything is enqueued; no
+ *     entry point aborts the process.
+ *   - Device pointers must be 16-byte aligned; workspaces 256-byte aligned.
+ */
+#ifndef AWQ_B200_H
+#define AWQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* awq_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  AWQ_OK = 0,
+  AWQ_ERR_INVALID_ARG = 1, /* null pointer, misaligned pointer, bad config value */
+  AWQ_ERR_SHAPE = 2,       /* d_in % g, d_in % 8, empty or oversized dimensions */
+  AWQ_ERR_WORKSPACE = 3,   /* workspace smaller than the matching *_workspace_size() */
+  AWQ_ERR_NONFINITE = 4,   /* a candidate loss was NaN or infinite (device-side) */
+  AWQ_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+  AWQ_ERR_DEVICE = 6,      /* a kernel gave up a bounded wait (device-side) */
+  AWQ_ERR_UNSUPPORTED = 7  /* no sm_100 device, or a configuration not built */
+} awq_status;
+
+typedef enum { AWQ_FORM_AUTO = 0, AWQ_FORM_DIRECT = 1, AWQ_FORM_GRAM = 2 } awq_form;
+
+/* Quantiser and search settings ([P4] §三 quant_config: w_bit, q_group_size,
+ * zero_point). */
+typedef struct {
+  int32_t bits;         /* 2, 3 or 4; codes are stored one per 4-bit nibble */
+  int32_t group;        /* g in {8, 16, 32, 64, 128, 256}; d_in % g == 0 */
+  int32_t symmetric;    /* 0: min/max affine with zero point; 1: symmetric */
+  int32_t n_alpha;      /* grid size, 1..64 */
+  int32_t form;         /* awq_form: how the loss contraction is evaluated */
+  float eps_a;          /* floor on a_i before the power; <= 0 selects 1e-4 */
+  const float* alphas;  /* HOST array [n_alpha] of grid points in [0, 1], or
+                           NULL for alpha_k = k / n_alpha ([P3] AWQ 二.2) */
+} awq_qcfg;
+
+/* Human-readable name of a status; never NULL. */
+const char* awq_status_str(awq_status s);
+
+/* ---------------------------------------------------------------------------
+ * Step a1: activation statistics.
+ * a[i] = (1/N) sum_t |X[t, i]|  ([P1] 激活感知, importance Omega_i; [P5] §1.2,
+ * a_i = E|x_i|). X: bf16 [N, d_in]; a: float [d_in]. Partial sums are kept in
+ * float64 and combined in a fixed order (bitwise repeatable).
+ * ws: scratch of awq_stats_workspace_size(N, d_in) bytes.
+ * Errors: AWQ_ERR_INVALID_ARG (null/misaligned), AWQ_ERR_SHAPE (N < 1,
+ * d_in < 8 or d_in % 8), AWQ_ERR_WORKSPACE, AWQ_ERR_CUDA.
+ * ------------------------------------------------------------------------- */
+size_t awq_stats_workspace_size(int64_t N, int64_t d_in);
+awq_status awq_act_stats(const void* X_bf16, int64_t N, int64_t d_in, float* a, void* ws,
+                         size_t ws_bytes, awq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Steps a2-a6: the scale search.
+ * For each alpha_k of the grid:
+ *   s_i = max(a_i, eps_a)^alpha_k / sqrt(max_j s_j * min_j s_j)      ([P5] §4.1)
+ *   dW  = Q(W S) S^-1 - W, group-wise along d_in                       ([P1] 缩放保护)
+ *         symmetric: Delta = max|v| / (2^(b-1)-1), q = clamp(rne(v/Delta), -2^(b-1), 2^(b-1)-1)
+ *         asymmetric: Delta = (max v - min v) / (2^b-1), z = clamp(rne(-min v/Delta), 0, 2^b-1),
+ *                     q = clamp(rne(v/Delta) + z, 0, 2^b-1), v_hat = (q - z) Delta
+ *   L_k = ||dW X^T||_F^2                                               ([P5] §1.1, §4.1)
+ * then best = argmin_k L_k (lowest k on ties) and s_best = s(alpha_best).
+ * The contraction runs on tcgen05 tensor cores with bf16 operands and fp32
+ * accumulation, either directly (dW X^T) or through G = X^T X.
+ * Outputs (device): losses float [n_alpha]; best int32 [1]; s_best float
+ * [d_in]; row_losses float [n_alpha, d_out] (per-row losses) or NULL.
+ * On non-finite losses the device sets best = -1, fills s_best with NaN and
+ * records AWQ_ERR_NONFINITE in the workspace.
+ * ws: scratch of awq_search_workspace_size(...) bytes (dominated by the
+ * n_alpha x d_out x d_in bf16 stack of candidate dW).
+ * ------------------------------------------------------------------------- */
+size_t awq_search_workspace_size(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg);
+awq_status awq_search_scales(const void* W_bf16, const void* X_bf16, const float* a, int64_t d_out,
+                             int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws, size_t ws_bytes,
+                             float* losses, int32_t* best, float* s_best, float* row_losses,
+                             awq_stream_t stream);
+
+/* The contraction form awq_search_scales will use for these sizes (1 direct,
+ * 2 Gram): AUTO picks the one with fewer multiply-adds,
+ * n_alpha*d_out*d_in*N versus N*d_in^2 + n_alpha*d_out*d_in^2. */
+int32_t awq_search_form(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg);
+
+/* Read back (synchronising `stream`) the device error word of a search or
+ * stats workspace and clear it: AWQ_OK, AWQ_ERR_NONFINITE or AWQ_ERR_DEVICE. */
+awq_status awq_workspace_error(void* ws, awq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Step a7: quantise at the chosen scales and pack.
+ * codes of Q(W S) with the quantiser above ([P2] §2.1 INT4 clip and fp16
+ * scale; [P4] §三 zero point), stored one per nibble, eight per uint32 word:
+ *   qweight uint32 [d_out, d_in/8], code of channel 8w+j in bits 4j..4j+3;
+ *   scales  fp16   [d_out, d_in/g] = Delta (rounded to nearest even);
+ *   zeros   fp16   [d_out, d_in/g] = z (asymmetric) or 2^(b-1) (symmetric,
+ *                                    whose codes are stored as q + 2^(b-1)).
+ * s: float [d_in] (typically s_best).
+ * ------------------------------------------------------------------------- */
+awq_status awq_quantize_pack(const void* W_bf16, const float* s, int64_t d_out, int64_t d_in,
+                             const awq_qcfg* cfg, uint32_t* qweight, void* scales_f16, void* zeros_f16,
+                             awq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * The search, one step at a time (awq_search_scales is exactly these calls
+ * in this order). They share the search workspace; offsets are internal.
+ * ------------------------------------------------------------------------- */
+/* a2: candidate scales s and 1/s of every alpha into the workspace. */
+awq_status awq_step_scales(const float* a, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg,
+                           void* ws, size_t ws_bytes, awq_stream_t stream);
+/* a3: the bf16 stack dW[k] = Q(W S_k) S_k^-1 - W for every alpha into the
+ * workspace (rows padded to a multiple of 128 with zeros). */
+awq_status awq_step_fake_quant(const void* W_bf16, int64_t d_out, int64_t d_in, int64_t N,
+                               const awq_qcfg* cfg, void* ws, size_t ws_bytes, awq_stream_t stream);
+/* a4 (Gram form only): X^T into the workspace, then G = X^T X (bf16). */
+awq_status awq_step_gram(const void* X_bf16, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg,
+                         void* ws, size_t ws_bytes, awq_stream_t stream);
+/* a5: the tensor-core contraction with the fused squared-sum epilogue, per
+ * (row, column-tile) partials into the workspace. X_bf16 is read by the
+ * direct form only. */
+awq_status awq_step_contract(const void* X_bf16, int64_t d_out, int64_t d_in, int64_t N,
+                             const awq_qcfg* cfg, void* ws, size_t ws_bytes, awq_stream_t stream);
+/* a6: fixed-order float64 reduction, argmin, s_best (outputs as in
+ * awq_search_scales). */
+awq_status awq_step_reduce(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                           size_t ws_bytes, float* losses, int32_t* best, float* s_best, float* row_losses,
+                           awq_stream_t stream);
+
+/* Copy of the candidate dW stack for inspection: dW for grid index k, rows
+ * [0, d_out), as bf16 [d_out, d_in] into dst (device). */
+awq_status awq_debug_copy_dw(const void* ws, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg,
+                             int32_t k, void* dst_bf16, awq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* AWQ_B200_H */

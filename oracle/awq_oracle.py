@@ -231,13 +231,18 @@ def search(W_bits: np.ndarray, X_bits: np.ndarray, a: np.ndarray, bits: int, gro
     if form == "gram" and G is None:
         G = gram(X_bits)
     per_row = np.zeros((n_alpha, W.shape[0]), dtype=np.float64)
-    for k, al in enumerate(alphas):
-        s = candidate_scales(a, al)
-        dW = delta_weight(W, s, bits, group, symmetric)
-        if form == "gram":
-            per_row[k] = row_losses_gram(dW, G)
-        else:
-            per_row[k] = row_losses_direct(dW, X_bits)
+    if form == "gram":
+        for k, al in enumerate(alphas):
+            per_row[k] = row_losses_gram(delta_weight(W, candidate_scales(a, al), bits, group, symmetric), G)
+    elif rows is not None:
+        # few rows: stack every candidate's dW and pass over X once
+        dWs = np.concatenate([delta_weight(W, candidate_scales(a, al), bits, group, symmetric)
+                              for al in alphas])
+        per_row = row_losses_direct(dWs, X_bits).reshape(n_alpha, W.shape[0])
+    else:
+        for k, al in enumerate(alphas):
+            per_row[k] = row_losses_direct(delta_weight(W, candidate_scales(a, al), bits, group, symmetric),
+                                           X_bits)
     losses = per_row.sum(axis=1)
     best = choose(losses)
     return dict(losses=losses, best=best, s_best=candidate_scales(a, alphas[best]),

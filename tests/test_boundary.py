@@ -1,0 +1,117 @@
+"""The C ABI without a GPU: the library loads, exports what include/awq.h
+declares, sizes its workspaces on the host, and rejects bad arguments before
+touching the device. No test here enqueues GPU work."""
+import ctypes
+import pathlib
+import re
+
+import pytest
+
+import weight_only_int4_act_b200 as awq
+from weight_only_int4_act_b200 import binding
+
+HEADER = pathlib.Path(__file__).resolve().parents[1] / "include" / "awq.h"
+FAKE = ctypes.c_void_p(0x10000)  # aligned, never dereferenced: every call below fails validation first
+
+
+def declared_symbols():
+    text = HEADER.read_text()
+    return sorted(set(re.findall(r"\b(awq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declarations_match_exports():
+    lib = awq.lib()
+    names = declared_symbols()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in awq.h but not exported"
+    assert sorted(binding.EXPORTED) == names
+
+
+def test_status_strings():
+    for s in range(8):
+        txt = awq.status_str(s)
+        assert txt.startswith(binding.STATUS_NAMES[s])
+    assert awq.status_str(99) == "AWQ_ERR_UNKNOWN"
+
+
+def test_workspace_sizes_and_form():
+    cfg = awq.make_cfg(4, 128, False, 20)
+    # C2 shape: direct form; stack of 20 x 4096 x 4096 bf16 dominates
+    n = awq.search_workspace_size(4096, 4096, 4096, cfg)
+    assert n >= 20 * 4096 * 4096 * 2
+    assert awq.search_form(4096, 4096, 4096, cfg) == "direct"
+    assert awq.search_form(11008, 4096, 16384, cfg) == "gram"
+    assert awq.search_form(28672, 8192, 65536, cfg) == "gram"
+    assert awq.search_form(4096, 11008, 16384, awq.make_cfg(3, 64, True, 20)) == "gram"
+    assert awq.search_form(256, 512, 256, cfg) == "direct"
+    forced = awq.make_cfg(4, 128, False, 20, form="gram")
+    assert awq.search_form(256, 512, 256, forced) == "gram"
+    assert awq.search_workspace_size(256, 512, 256, forced) > awq.search_workspace_size(256, 512, 256, cfg)
+    # ragged rows pad to 128
+    assert awq.search_workspace_size(200, 512, 256, cfg) == awq.search_workspace_size(256, 512, 256, cfg)
+    assert awq.stats_workspace_size(65536, 8192) > 0
+    # invalid configurations size to 0
+    assert awq.search_workspace_size(256, 500, 256, cfg) == 0
+    assert awq.search_workspace_size(256, 512, 0, cfg) == 0
+    assert awq.stats_workspace_size(0, 512) == 0
+
+
+@pytest.mark.parametrize("field,value", [
+    ("bits", 1), ("bits", 5), ("group", 96), ("group", 4), ("group", 512), ("symmetric", 2),
+    ("n_alpha", 0), ("n_alpha", 65), ("form", 3),
+])
+def test_bad_config_rejected(field, value):
+    cfg = awq.make_cfg(4, 128, False, 20)
+    setattr(cfg, field, value)
+    lib = awq.lib()
+    st = lib.awq_search_scales(FAKE, FAKE, FAKE, 256, 512, 256, ctypes.byref(cfg), FAKE, 1 << 40,
+                               FAKE, FAKE, FAKE, None, None)
+    assert st == 1  # AWQ_ERR_INVALID_ARG
+    assert awq.search_workspace_size(256, 512, 256, cfg) == 0
+
+
+def test_bad_alpha_grid_rejected():
+    cfg = awq.make_cfg(4, 128, False, 3, alphas=[0.0, 0.5, 1.5])
+    assert awq.search_workspace_size(256, 512, 256, cfg) == 0
+
+
+def test_shape_and_pointer_errors():
+    lib = awq.lib()
+    cfg = awq.make_cfg(4, 128, False, 20)
+    c = ctypes.byref(cfg)
+    big = 1 << 40
+    # d_in not a multiple of the group
+    assert lib.awq_search_scales(FAKE, FAKE, FAKE, 256, 500, 256, c, FAKE, big, FAKE, FAKE, FAKE, None, None) == 2
+    # no tokens / no rows
+    assert lib.awq_search_scales(FAKE, FAKE, FAKE, 256, 512, 0, c, FAKE, big, FAKE, FAKE, FAKE, None, None) == 2
+    assert lib.awq_search_scales(FAKE, FAKE, FAKE, 0, 512, 256, c, FAKE, big, FAKE, FAKE, FAKE, None, None) == 2
+    # null pointers
+    assert lib.awq_search_scales(None, FAKE, FAKE, 256, 512, 256, c, FAKE, big, FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.awq_search_scales(FAKE, FAKE, FAKE, 256, 512, 256, c, None, big, FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.awq_search_scales(FAKE, FAKE, FAKE, 256, 512, 256, c, FAKE, big, None, FAKE, FAKE, None, None) == 1
+    # misaligned pointers
+    odd = ctypes.c_void_p(0x10002)
+    assert lib.awq_search_scales(odd, FAKE, FAKE, 256, 512, 256, c, FAKE, big, FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.awq_search_scales(FAKE, FAKE, FAKE, 256, 512, 256, c, odd, big, FAKE, FAKE, FAKE, None, None) == 1
+    # workspace too small
+    need = awq.search_workspace_size(256, 512, 256, cfg)
+    assert lib.awq_search_scales(FAKE, FAKE, FAKE, 256, 512, 256, c, FAKE, need - 1, FAKE, FAKE, FAKE, None,
+                                 None) == 3
+    # stats
+    assert lib.awq_act_stats(None, 16, 512, FAKE, FAKE, big, None) == 1
+    assert lib.awq_act_stats(FAKE, 0, 512, FAKE, FAKE, big, None) == 2
+    assert lib.awq_act_stats(FAKE, 16, 500, FAKE, FAKE, big, None) == 2
+    assert lib.awq_act_stats(FAKE, 16, 512, FAKE, FAKE, 8, None) == 3
+    # pack
+    assert lib.awq_quantize_pack(FAKE, FAKE, 256, 500, c, FAKE, FAKE, FAKE, None) == 2
+    assert lib.awq_quantize_pack(FAKE, None, 256, 512, c, FAKE, FAKE, FAKE, None) == 1
+    # workspace error read-back needs a workspace
+    assert lib.awq_workspace_error(None, None) == 1
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    X = torch.zeros((4, 16), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        awq.act_stats(X)

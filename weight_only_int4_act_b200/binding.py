@@ -1,0 +1,227 @@
+"""Python binding of the C ABI in include/awq.h (ctypes; argument marshalling only).
+
+Every computation runs in the CUDA library; PyTorch only provides device
+memory and the current stream. If the library is missing the calls raise:
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_float, c_int32, c_int64, c_size_t, c_void_p
+
+from ._build import LIB_PATH
+
+AWQ_OK = 0
+STATUS_NAMES = {
+    0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_SHAPE", 3: "AWQ_ERR_WORKSPACE",
+    4: "AWQ_ERR_NONFINITE", 5: "AWQ_ERR_CUDA", 6: "AWQ_ERR_DEVICE", 7: "AWQ_ERR_UNSUPPORTED",
+}
+FORMS = {"auto": 0, "direct": 1, "gram": 2}
+
+# every symbol include/awq.h declares
+EXPORTED = (
+    "awq_status_str", "awq_stats_workspace_size", "awq_act_stats", "awq_search_workspace_size",
+    "awq_search_scales", "awq_search_form", "awq_workspace_error", "awq_quantize_pack",
+    "awq_step_scales", "awq_step_fake_quant", "awq_step_gram", "awq_step_contract", "awq_step_reduce",
+    "awq_debug_copy_dw",
+)
+
+
+class AwqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class QCfg(ctypes.Structure):
+    _fields_ = [
+        ("bits", c_int32), ("group", c_int32), ("symmetric", c_int32), ("n_alpha", c_int32),
+        ("form", c_int32), ("eps_a", c_float), ("alphas", POINTER(c_float)),
+    ]
+
+
+def make_cfg(bits=4, group=128, symmetric=False, n_alpha=20, form="auto", eps_a=1e-4, alphas=None) -> QCfg:
+    cfg = QCfg(int(bits), int(group), int(bool(symmetric)), int(n_alpha), FORMS[form], float(eps_a), None)
+    if alphas is not None:
+        arr = (c_float * len(alphas))(*[float(x) for x in alphas])
+        cfg.alphas = ctypes.cast(arr, POINTER(c_float))
+        cfg._keep = arr  # keep the host array alive with the struct
+    return cfg
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library {LIB_PATH} is missing; build it with __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        cfgp = POINTER(QCfg)
+        sig = {
+            "awq_status_str": (c_char_p, [c_int32]),
+            "awq_stats_workspace_size": (c_size_t, [c_int64, c_int64]),
+            "awq_act_stats": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_size_t, c_void_p]),
+            "awq_search_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, cfgp]),
+            "awq_search_form": (c_int32, [c_int64, c_int64, c_int64, cfgp]),
+            "awq_search_scales": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, cfgp,
+                                            c_void_p, c_size_t, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+            "awq_workspace_error": (c_int32, [c_void_p, c_void_p]),
+            "awq_quantize_pack": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_void_p, c_void_p,
+                                            c_void_p, c_void_p]),
+            "awq_step_scales": (c_int32, [c_void_p, c_int64, c_int64, c_int64, cfgp, c_void_p, c_size_t, c_void_p]),
+            "awq_step_fake_quant": (c_int32, [c_void_p, c_int64, c_int64, c_int64, cfgp, c_void_p, c_size_t,
+                                              c_void_p]),
+            "awq_step_gram": (c_int32, [c_void_p, c_int64, c_int64, c_int64, cfgp, c_void_p, c_size_t, c_void_p]),
+            "awq_step_contract": (c_int32, [c_void_p, c_int64, c_int64, c_int64, cfgp, c_void_p, c_size_t,
+                                            c_void_p]),
+            "awq_step_reduce": (c_int32, [c_int64, c_int64, c_int64, cfgp, c_void_p, c_size_t, c_void_p, c_void_p,
+                                          c_void_p, c_void_p, c_void_p]),
+            "awq_debug_copy_dw": (c_int32, [c_void_p, c_int64, c_int64, c_int64, cfgp, c_int32, c_void_p,
+                                            c_void_p]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().awq_status_str(status).decode()
+
+
+def _check(status: int, what: str):
+    if status != AWQ_OK:
+        raise AwqError(status, what)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream():
+    return c_void_p(_torch().cuda.current_stream().cuda_stream)
+
+
+def _req(t, dtype, shape, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _ptr(t):
+    return c_void_p(t.data_ptr()) if t is not None else None
+
+
+# --------------------------------------------------------------------------- sizes
+def stats_workspace_size(N: int, d_in: int) -> int:
+    return int(lib().awq_stats_workspace_size(N, d_in))
+
+
+def search_workspace_size(d_out: int, d_in: int, N: int, cfg: QCfg) -> int:
+    return int(lib().awq_search_workspace_size(d_out, d_in, N, ctypes.byref(cfg)))
+
+
+def search_form(d_out: int, d_in: int, N: int, cfg: QCfg) -> str:
+    f = int(lib().awq_search_form(d_out, d_in, N, ctypes.byref(cfg)))
+    return {1: "direct", 2: "gram"}.get(f, "invalid")
+
+
+def workspace(nbytes: int):
+    torch = _torch()
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device="cuda")
+
+
+# --------------------------------------------------------------------------- a1
+def act_stats(X, ws=None, out=None):
+    """a[i] = mean_t |X[t, i]| for bf16 X [N, d_in] (float32 [d_in])."""
+    torch = _torch()
+    _req(X, torch.bfloat16, None, "X")
+    N, d_in = X.shape
+    if ws is None:
+        ws = workspace(stats_workspace_size(N, d_in))
+    a = out if out is not None else torch.empty(d_in, dtype=torch.float32, device=X.device)
+    _check(lib().awq_act_stats(_ptr(X), N, d_in, _ptr(a), _ptr(ws), ws.numel(), _stream()), "awq_act_stats")
+    return a
+
+
+# --------------------------------------------------------------------------- a2-a6
+def search_scales(W, X, a, cfg: QCfg, ws=None, row_losses=False, outputs=None):
+    """Loss of every alpha, the chosen index and its scales (device tensors).
+
+    Returns dict(losses float32[n_alpha], best int32[1], s_best float32[d_in],
+    row_losses float32[n_alpha, d_out] or None, ws)."""
+    torch = _torch()
+    _req(W, torch.bfloat16, None, "W")
+    d_out, d_in = W.shape
+    _req(X, torch.bfloat16, None, "X")
+    N = X.shape[0]
+    if X.shape[1] != d_in:
+        raise ValueError("X must have d_in columns")
+    _req(a, torch.float32, (d_in,), "a")
+    if ws is None:
+        ws = workspace(search_workspace_size(d_out, d_in, N, cfg))
+    if outputs is None:
+        outputs = dict(
+            losses=torch.empty(cfg.n_alpha, dtype=torch.float32, device=W.device),
+            best=torch.empty(1, dtype=torch.int32, device=W.device),
+            s_best=torch.empty(d_in, dtype=torch.float32, device=W.device),
+            row_losses=torch.empty((cfg.n_alpha, d_out), dtype=torch.float32, device=W.device) if row_losses else None,
+        )
+    o = outputs
+    _check(lib().awq_search_scales(_ptr(W), _ptr(X), _ptr(a), d_out, d_in, N, ctypes.byref(cfg), _ptr(ws),
+                                   ws.numel(), _ptr(o["losses"]), _ptr(o["best"]), _ptr(o["s_best"]),
+                                   _ptr(o["row_losses"]), _stream()), "awq_search_scales")
+    return dict(o, ws=ws)
+
+
+def workspace_error(ws):
+    """Raise AwqError if a kernel recorded an error in the workspace (synchronises)."""
+    _check(lib().awq_workspace_error(_ptr(ws), _stream()), "device")
+
+
+def step(name: str, *args):
+    """Call one awq_step_* entry point with already-marshalled arguments."""
+    fn = getattr(lib(), "awq_step_" + name)
+    _check(fn(*args), "awq_step_" + name)
+
+
+def debug_dw(ws, d_out, d_in, N, cfg, k):
+    """bf16 [d_out, d_in] copy of the candidate dW for grid index k."""
+    torch = _torch()
+    dst = torch.empty((d_out, d_in), dtype=torch.bfloat16, device="cuda")
+    _check(lib().awq_debug_copy_dw(_ptr(ws), d_out, d_in, N, ctypes.byref(cfg), k, _ptr(dst), _stream()),
+           "awq_debug_copy_dw")
+    return dst
+
+
+# --------------------------------------------------------------------------- a7
+def quantize_pack(W, s, cfg: QCfg, outputs=None):
+    """(qweight int32 view of uint32 [d_out, d_in/8], scales fp16 [d_out, d_in/g], zeros fp16 [d_out, d_in/g])."""
+    torch = _torch()
+    _req(W, torch.bfloat16, None, "W")
+    d_out, d_in = W.shape
+    _req(s, torch.float32, (d_in,), "s")
+    if outputs is None:
+        ng = d_in // cfg.group if cfg.group > 0 else 0
+        outputs = (torch.empty((d_out, d_in // 8), dtype=torch.int32, device=W.device),
+                   torch.empty((d_out, ng), dtype=torch.float16, device=W.device),
+                   torch.empty((d_out, ng), dtype=torch.float16, device=W.device))
+    q, sc, zr = outputs
+    _check(lib().awq_quantize_pack(_ptr(W), _ptr(s), d_out, d_in, ctypes.byref(cfg), _ptr(q), _ptr(sc), _ptr(zr),
+                                   _stream()), "awq_quantize_pack")
+    return q, sc, zr

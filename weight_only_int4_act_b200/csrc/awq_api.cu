@@ -1,0 +1,419 @@
+// C ABI of the AWQ search library (declared in include/awq.h): argument
+// validation, workspace layout, TMA descriptor set-up and the launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/awq.h"
+#include "awq_kernels.cuh"
+#include "gemm_sm100.cuh"
+
+using namespace awq;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+constexpr int kStatsTargetBlocks = 148 * 8;
+constexpr int kGroupN = 8;
+
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline cudaStream_t as_stream(awq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ------------------------------------------------------------------ validation
+awq_status check_cfg(const awq_qcfg* cfg) {
+  if (!cfg) return AWQ_ERR_INVALID_ARG;
+  if (cfg->bits < 2 || cfg->bits > 4) return AWQ_ERR_INVALID_ARG;
+  const int g = cfg->group;
+  if (g < 8 || g > 256 || (g & (g - 1)) != 0) return AWQ_ERR_INVALID_ARG;
+  if (cfg->symmetric != 0 && cfg->symmetric != 1) return AWQ_ERR_INVALID_ARG;
+  if (cfg->n_alpha < 1 || cfg->n_alpha > MAX_ALPHA) return AWQ_ERR_INVALID_ARG;
+  if (cfg->form < AWQ_FORM_AUTO || cfg->form > AWQ_FORM_GRAM) return AWQ_ERR_INVALID_ARG;
+  if (!(cfg->eps_a <= 0.f || std::isfinite(cfg->eps_a))) return AWQ_ERR_INVALID_ARG;
+  if (cfg->alphas) {
+    for (int k = 0; k < cfg->n_alpha; ++k)
+      if (!(cfg->alphas[k] >= 0.f && cfg->alphas[k] <= 1.f)) return AWQ_ERR_INVALID_ARG;
+  }
+  return AWQ_OK;
+}
+
+// sizes valid for the search / pack: d_in a multiple of g (hence of 8); bounds
+// keep every index of the kernels and TMA coordinates inside int32.
+awq_status check_layer_shape(int64_t d_out, int64_t d_in, const awq_qcfg* cfg) {
+  if (d_out < 1 || d_in < 8 || d_in % 8 != 0) return AWQ_ERR_SHAPE;
+  if (d_in % cfg->group != 0) return AWQ_ERR_SHAPE;
+  if (d_in > (1 << 20) || d_out > (1 << 24)) return AWQ_ERR_SHAPE;
+  const long long M = (long long)cfg->n_alpha * cdiv(d_out, GEMM_BM) * GEMM_BM;
+  if (M > (long long)INT32_MAX / 2) return AWQ_ERR_SHAPE;
+  return AWQ_OK;
+}
+
+awq_status check_tokens(int64_t N) {
+  if (N < 1 || N > (int64_t)INT32_MAX / 2) return AWQ_ERR_SHAPE;
+  return AWQ_OK;
+}
+
+double alpha_value(const awq_qcfg* cfg, int k) {
+  return cfg->alphas ? (double)cfg->alphas[k] : (double)k / (double)cfg->n_alpha;
+}
+
+float eps_value(const awq_qcfg* cfg) { return cfg->eps_a > 0.f ? cfg->eps_a : 1e-4f; }
+
+// ------------------------------------------------------------------ device checks
+awq_status check_device(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (major != 10 || minor != 0) return AWQ_ERR_UNSUPPORTED;
+  if (num_sms && cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  return AWQ_OK;
+}
+
+awq_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? AWQ_OK : AWQ_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ stats layout
+struct StatsLayout {
+  int col_blocks, rows_per_chunk, n_chunks;
+  size_t off_part, total;
+};
+
+StatsLayout stats_layout(int64_t N, int64_t d_in) {
+  StatsLayout L{};
+  L.col_blocks = (int)cdiv(d_in, STATS_COLS);
+  long long rpc = cdiv((long long)N * L.col_blocks, kStatsTargetBlocks);
+  rpc = cdiv(rpc < 32 ? 32 : rpc, 32) * 32;
+  L.rows_per_chunk = (int)rpc;
+  L.n_chunks = (int)cdiv(N, rpc);
+  L.off_part = kAlign;  // [0, 1024): error word
+  L.total = L.off_part + align_up((size_t)L.n_chunks * d_in * sizeof(double));
+  return L;
+}
+
+// ------------------------------------------------------------------ search layout
+struct SearchLayout {
+  int form;         // 1 direct, 2 Gram
+  int n_alpha;
+  int d_out_pad;
+  long long M;      // rows of the dW stack
+  int n_blocks_n;   // column tiles of the contraction
+  int n_red_chunks; // blocks per alpha in the row reduction
+  long long ld_t;   // padded token count of X^T (Gram)
+  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_xt, off_g, total;
+};
+
+int choose_form(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg) {
+  if (cfg->form == AWQ_FORM_DIRECT || cfg->form == AWQ_FORM_GRAM) return cfg->form;
+  const double direct = (double)cfg->n_alpha * d_out * d_in * N;
+  const double gram = (double)N * d_in * d_in + (double)cfg->n_alpha * d_out * d_in * d_in;
+  return direct <= gram ? AWQ_FORM_DIRECT : AWQ_FORM_GRAM;
+}
+
+SearchLayout search_layout(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg) {
+  SearchLayout L{};
+  L.form = choose_form(d_out, d_in, N, cfg);
+  L.n_alpha = cfg->n_alpha;
+  L.d_out_pad = (int)(cdiv(d_out, GEMM_BM) * GEMM_BM);
+  L.M = (long long)L.n_alpha * L.d_out_pad;
+  L.n_blocks_n = (int)cdiv(L.form == AWQ_FORM_DIRECT ? N : d_in, GEMM_BN);
+  L.n_red_chunks = (int)cdiv(d_out, REDUCE_THREADS);
+  L.ld_t = cdiv(N, 64) * 64;
+  size_t off = kAlign;  // [0, 1024): error word
+  L.off_s = off;      off += align_up((size_t)L.n_alpha * d_in * sizeof(float));
+  L.off_inv = off;    off += align_up((size_t)L.n_alpha * d_in * sizeof(float));
+  L.off_dw = off;     off += align_up((size_t)L.M * d_in * 2);
+  L.off_part = off;   off += align_up((size_t)L.n_blocks_n * L.M * sizeof(float));
+  L.off_blk = off;    off += align_up((size_t)L.n_alpha * L.n_red_chunks * sizeof(double));
+  L.off_loss64 = off; off += align_up((size_t)L.n_alpha * sizeof(double));
+  if (L.form == AWQ_FORM_GRAM) {
+    L.off_xt = off;   off += align_up((size_t)d_in * L.ld_t * 2);
+    L.off_g = off;    off += align_up((size_t)d_in * d_in * 2);
+  }
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off); }
+
+awq_status check_search_common(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                               size_t ws_bytes, SearchLayout* L) {
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_layer_shape(d_out, d_in, cfg)) != AWQ_OK) return st;
+  if ((st = check_tokens(N)) != AWQ_OK) return st;
+  if (!ws || !aligned(ws, 256)) return AWQ_ERR_INVALID_ARG;
+  *L = search_layout(d_out, d_in, N, cfg);
+  if (ws_bytes < L->total) return AWQ_ERR_WORKSPACE;
+  return AWQ_OK;
+}
+
+// ------------------------------------------------------------------ TMA
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, cols] matrix with leading dimension ld
+// (elements), box = box_rows x 64 columns, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// D = A[M, K] * B[Nr, K]^T with the given epilogue.
+template <int MODE>
+awq_status run_gemm(const void* A, long long M, long long lda, const void* B, long long Nr, long long ldb, long long K,
+                    GemmArgs args, int num_sms, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, lda, GEMM_BM)) return AWQ_ERR_CUDA;
+  if (!make_map(&tb, B, Nr, K, ldb, GEMM_BN)) return AWQ_ERR_CUDA;
+  args.M = (int)M;
+  args.N = (int)Nr;
+  args.K = (int)K;
+  args.n_blocks_m = (int)cdiv(M, GEMM_BM);
+  args.n_blocks_n = (int)cdiv(Nr, GEMM_BN);
+  args.group_n = kGroupN < args.n_blocks_n ? kGroupN : args.n_blocks_n;
+  if (cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) !=
+      cudaSuccess)
+    return AWQ_ERR_CUDA;
+  const long long tiles = (long long)args.n_blocks_m * args.n_blocks_n;
+  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+  gemm_bf16_tcgen05<MODE><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(ta, tb, args);
+  return launch_status();
+}
+
+int elementwise_grid(long long threads_needed, int num_sms) {
+  long long blocks = cdiv(threads_needed, 256);
+  const long long cap = (long long)num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  return (int)(blocks < 1 ? 1 : blocks);
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* awq_status_str(awq_status s) {
+  switch (s) {
+    case AWQ_OK: return "AWQ_OK";
+    case AWQ_ERR_INVALID_ARG: return "AWQ_ERR_INVALID_ARG: null or misaligned pointer, or bad config value";
+    case AWQ_ERR_SHAPE: return "AWQ_ERR_SHAPE: unsupported or inconsistent sizes";
+    case AWQ_ERR_WORKSPACE: return "AWQ_ERR_WORKSPACE: workspace smaller than required";
+    case AWQ_ERR_NONFINITE: return "AWQ_ERR_NONFINITE: a candidate loss was NaN or infinite";
+    case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: CUDA runtime call or launch failed";
+    case AWQ_ERR_DEVICE: return "AWQ_ERR_DEVICE: a kernel gave up a bounded wait";
+    case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED: needs an sm_100 (B200) device";
+  }
+  return "AWQ_ERR_UNKNOWN";
+}
+
+size_t awq_stats_workspace_size(int64_t N, int64_t d_in) {
+  if (N < 1 || d_in < 8) return 0;
+  return stats_layout(N, d_in).total;
+}
+
+awq_status awq_act_stats(const void* X, int64_t N, int64_t d_in, float* a, void* ws, size_t ws_bytes,
+                         awq_stream_t stream) {
+  if (!X || !a || !ws) return AWQ_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(ws, 256)) return AWQ_ERR_INVALID_ARG;
+  if (check_tokens(N) != AWQ_OK || d_in < 8 || d_in % 8 != 0 || d_in > (1 << 20)) return AWQ_ERR_SHAPE;
+  const StatsLayout L = stats_layout(N, d_in);
+  if (ws_bytes < L.total) return AWQ_ERR_WORKSPACE;
+  awq_status st = check_device(nullptr);
+  if (st != AWQ_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  dim3 grid(L.col_blocks, L.n_chunks);
+  act_absmean_partial<<<grid, STATS_THREADS, 0, s>>>(static_cast<const __nv_bfloat16*>(X), N, (int)d_in,
+                                                     L.rows_per_chunk, at<double>(ws, L.off_part));
+  if ((st = launch_status()) != AWQ_OK) return st;
+  act_absmean_final<<<(unsigned)cdiv(d_in, 256), 256, 0, s>>>(at<double>(ws, L.off_part), L.n_chunks, N, (int)d_in, a);
+  return launch_status();
+}
+
+size_t awq_search_workspace_size(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg) {
+  if (check_cfg(cfg) != AWQ_OK || check_layer_shape(d_out, d_in, cfg) != AWQ_OK || check_tokens(N) != AWQ_OK)
+    return 0;
+  return search_layout(d_out, d_in, N, cfg).total;
+}
+
+int32_t awq_search_form(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg) {
+  if (check_cfg(cfg) != AWQ_OK || check_layer_shape(d_out, d_in, cfg) != AWQ_OK || check_tokens(N) != AWQ_OK)
+    return 0;
+  return choose_form(d_out, d_in, N, cfg);
+}
+
+awq_status awq_step_scales(const float* a, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                           size_t ws_bytes, awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  if (!a) return AWQ_ERR_INVALID_ARG;
+  if ((st = check_device(nullptr)) != AWQ_OK) return st;
+  AlphaGrid grid{};
+  for (int k = 0; k < cfg->n_alpha; ++k) grid.v[k] = alpha_value(cfg, k);
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return AWQ_ERR_CUDA;
+  candidate_scales<<<cfg->n_alpha, 512, 0, s>>>(a, (int)d_in, grid, eps_value(cfg), at<float>(ws, L.off_s),
+                                                at<float>(ws, L.off_inv));
+  return launch_status();
+}
+
+awq_status awq_step_fake_quant(const void* W, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                               size_t ws_bytes, awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  if (!W || !aligned(W, 16)) return AWQ_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((st = check_device(&sms)) != AWQ_OK) return st;
+  const long long units = (long long)L.d_out_pad * (d_in / 8);
+  fake_quant_delta<<<elementwise_grid(units, sms), 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in, L.d_out_pad, at<float>(ws, L.off_s),
+      at<float>(ws, L.off_inv), cfg->n_alpha, cfg->bits, cfg->symmetric, cfg->group / 8,
+      at<__nv_bfloat16>(ws, L.off_dw));
+  return launch_status();
+}
+
+awq_status awq_step_gram(const void* X, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                         size_t ws_bytes, awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  if (L.form != AWQ_FORM_GRAM) return AWQ_OK;
+  if (!X || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((st = check_device(&sms)) != AWQ_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  dim3 tgrid((unsigned)(L.ld_t / 64), (unsigned)cdiv(d_in, 64));
+  transpose_bf16<<<tgrid, dim3(64, 4), 0, s>>>(static_cast<const __nv_bfloat16*>(X), N, (int)d_in, L.ld_t,
+                                               at<__nv_bfloat16>(ws, L.off_xt));
+  if ((st = launch_status()) != AWQ_OK) return st;
+  GemmArgs ga{};
+  ga.C = at<__nv_bfloat16>(ws, L.off_g);
+  ga.ldC = d_in;
+  ga.err = at<int>(ws, 0);
+  const void* xt = at<void>(ws, L.off_xt);
+  return run_gemm<EPI_STORE>(xt, d_in, L.ld_t, xt, d_in, L.ld_t, L.ld_t, ga, sms, s);
+}
+
+awq_status awq_step_contract(const void* X, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                             size_t ws_bytes, awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  int sms = 0;
+  if ((st = check_device(&sms)) != AWQ_OK) return st;
+  GemmArgs ga{};
+  ga.part = at<float>(ws, L.off_part);
+  ga.err = at<int>(ws, 0);
+  const void* dw = at<void>(ws, L.off_dw);
+  if (L.form == AWQ_FORM_DIRECT) {
+    if (!X || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
+    return run_gemm<EPI_SUMSQ>(dw, L.M, d_in, X, N, d_in, d_in, ga, sms, as_stream(stream));
+  }
+  ga.E = at<__nv_bfloat16>(ws, L.off_dw);
+  ga.ldE = d_in;
+  return run_gemm<EPI_DOT>(dw, L.M, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, sms, as_stream(stream));
+}
+
+awq_status awq_step_reduce(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws, size_t ws_bytes,
+                           float* losses, int32_t* best, float* s_best, float* row_losses, awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  if (!losses || !best || !s_best) return AWQ_ERR_INVALID_ARG;
+  if ((st = check_device(nullptr)) != AWQ_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  dim3 rgrid(L.n_red_chunks, L.n_alpha);
+  row_loss_reduce<<<rgrid, REDUCE_THREADS, 0, s>>>(at<float>(ws, L.off_part), L.n_blocks_n, L.M, (int)d_out,
+                                                  L.d_out_pad, row_losses, at<double>(ws, L.off_blk));
+  if ((st = launch_status()) != AWQ_OK) return st;
+  loss_argmin<<<1, 256, 0, s>>>(at<double>(ws, L.off_blk), L.n_red_chunks, L.n_alpha, at<float>(ws, L.off_s),
+                                (int)d_in, losses, at<double>(ws, L.off_loss64), best, s_best, at<int>(ws, 0));
+  return launch_status();
+}
+
+awq_status awq_search_scales(const void* W, const void* X, const float* a, int64_t d_out, int64_t d_in, int64_t N,
+                             const awq_qcfg* cfg, void* ws, size_t ws_bytes, float* losses, int32_t* best,
+                             float* s_best, float* row_losses, awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  if (!W || !X || !a || !losses || !best || !s_best) return AWQ_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
+  if ((st = awq_step_scales(a, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  if ((st = awq_step_fake_quant(W, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  if ((st = awq_step_gram(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  if ((st = awq_step_contract(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  return awq_step_reduce(d_out, d_in, N, cfg, ws, ws_bytes, losses, best, s_best, row_losses, stream);
+}
+
+awq_status awq_workspace_error(void* ws, awq_stream_t stream) {
+  if (!ws) return AWQ_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  int word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (word == 0) return AWQ_OK;
+  if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return AWQ_ERR_CUDA;
+  return word == ERR_NONFINITE ? AWQ_ERR_NONFINITE : AWQ_ERR_DEVICE;
+}
+
+awq_status awq_quantize_pack(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
+                             uint32_t* qweight, void* scales, void* zeros, awq_stream_t stream) {
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_layer_shape(d_out, d_in, cfg)) != AWQ_OK) return st;
+  if (!W || !s || !qweight || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(s, 16) || !aligned(qweight, 4) || !aligned(scales, 2) || !aligned(zeros, 2))
+    return AWQ_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((st = check_device(&sms)) != AWQ_OK) return st;
+  const long long units = (long long)d_out * (d_in / 8);
+  quantize_pack<<<elementwise_grid(units, sms), 256, 0, as_stream(stream)>>>(
+      static_cast<const __nv_bfloat16*>(W), s, (int)d_out, (int)d_in, cfg->bits, cfg->symmetric, cfg->group / 8,
+      qweight, static_cast<__half*>(scales), static_cast<__half*>(zeros));
+  return launch_status();
+}
+
+awq_status awq_debug_copy_dw(const void* ws, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, int32_t k,
+                             void* dst, awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, const_cast<void*>(ws), SIZE_MAX, &L);
+  if (st != AWQ_OK) return st;
+  if (!dst || k < 0 || k >= cfg->n_alpha) return AWQ_ERR_INVALID_ARG;
+  const void* src = static_cast<const uint8_t*>(ws) + L.off_dw + (size_t)k * L.d_out_pad * d_in * 2;
+  if (cudaMemcpyAsync(dst, src, (size_t)d_out * d_in * 2, cudaMemcpyDeviceToDevice, as_stream(stream)) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  return AWQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,351 @@
+// SIMT kernels of the AWQ search path (everything except the tensor-core
+// contraction): activation statistics, candidate scales, the fake-quantised
+// dW stack, the transpose feeding the Gram product, the fixed-order loss
+// reduction with argmin, and the pack.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fq.cuh"
+
+namespace awq {
+
+constexpr int ERR_NONFINITE = 0x201;
+constexpr int MAX_ALPHA = 64;
+
+struct AlphaGrid {
+  double v[MAX_ALPHA];
+};
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4 u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    f[2 * h] = __uint_as_float(w[h] << 16);
+    f[2 * h + 1] = __uint_as_float(w[h] & 0xFFFF0000u);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a1: a[i] = (1/N) sum_t |X[t, i]|   ([P1] 激活感知 Omega_i, [P5] §1.2)
+// Block = 256 threads covering 256 columns (each lane 8 columns, 16-byte
+// loads; warps take interleaved rows) and `rows_per_chunk` rows. Each thread
+// sums 4 rows in fp32, then accumulates in fp64; the 8 warps are combined in a
+// fixed order and the chunk's fp64 column sums are written to `part`.
+// ---------------------------------------------------------------------------
+constexpr int STATS_THREADS = 256;
+constexpr int STATS_COLS = 256;
+
+__global__ void __launch_bounds__(STATS_THREADS) act_absmean_partial(const __nv_bfloat16* __restrict__ X, long long N,
+                                                                     int d_in, int rows_per_chunk,
+                                                                     double* __restrict__ part) {
+  __shared__ double red[STATS_THREADS / 32][STATS_COLS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int col = blockIdx.x * STATS_COLS + lane * 8;
+  const long long r0 = (long long)blockIdx.y * rows_per_chunk;
+  const long long r1 = min(N, r0 + rows_per_chunk);
+  double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (col < d_in) {
+    const __nv_bfloat16* base = X + col;
+    for (long long r = r0 + warp; r < r1; r += 4 * 8) {
+      uint4 u[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const long long rr = r + 8 * k;
+        u[k] = rr < r1 ? __ldcs(reinterpret_cast<const uint4*>(base + rr * d_in)) : make_uint4(0, 0, 0, 0);
+      }
+      float s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float f[8];
+        unpack_bf16x8(u[k], f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s[j] += fabsf(f[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] += (double)s[j];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[warp][lane * 8 + j] = acc[j];
+  __syncthreads();
+  const int c = blockIdx.x * STATS_COLS + threadIdx.x;
+  if (c < d_in) {
+    double t = 0.0;
+#pragma unroll
+    for (int w = 0; w < STATS_THREADS / 32; ++w) t += red[w][threadIdx.x];
+    part[(long long)blockIdx.y * d_in + c] = t;
+  }
+}
+
+__global__ void act_absmean_final(const double* __restrict__ part, int n_chunks, long long N, int d_in,
+                                  float* __restrict__ a) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= d_in) return;
+  double t = 0.0;
+  for (int k = 0; k < n_chunks; ++k) t += part[(long long)k * d_in + c];
+  a[c] = (float)(t / (double)N);
+}
+
+// ---------------------------------------------------------------------------
+// a2: s_k,i = max(a_i, eps)^alpha_k / sqrt(max_j t_j * min_j t_j), and 1/s.
+// ([P5] §4.1 s_i = a_i^alpha.) One block per alpha; the power and the
+// normalisation are taken in fp64 and rounded once to fp32.
+// ---------------------------------------------------------------------------
+__global__ void candidate_scales(const float* __restrict__ a, int d_in, AlphaGrid grid, float eps_a,
+                                 float* __restrict__ s_all, float* __restrict__ inv_all) {
+  __shared__ double smax[32], smin[32];
+  const double alpha = grid.v[blockIdx.x];
+  double mx = 0.0, mn = 1e300;
+  for (int i = threadIdx.x; i < d_in; i += blockDim.x) {
+    const double t = pow(fmax((double)a[i], (double)eps_a), alpha);
+    mx = fmax(mx, t);
+    mn = fmin(mn, t);
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (lane == 0) {
+    smax[warp] = mx;
+    smin[warp] = mn;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    mx = lane < nw ? smax[lane] : 0.0;
+    mn = lane < nw ? smin[lane] : 1e300;
+    for (int off = 16; off > 0; off >>= 1) {
+      mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    }
+    if (lane == 0) {
+      smax[0] = mx;
+      smin[0] = mn;
+    }
+  }
+  __syncthreads();
+  const double norm = sqrt(smax[0] * smin[0]);
+  for (int i = threadIdx.x; i < d_in; i += blockDim.x) {
+    const double s = pow(fmax((double)a[i], (double)eps_a), alpha) / norm;
+    s_all[(long long)blockIdx.x * d_in + i] = (float)s;
+    inv_all[(long long)blockIdx.x * d_in + i] = (float)(1.0 / s);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a3: dW[k][r][:] = Q(W_r S_k) S_k^-1 - W_r as bf16, for every alpha k.
+// ([P1] 缩放保护 W~ = sW, W^ = Q(W~)/s; [P5] §2.2 Q(WS)S^-1.)
+// One thread = 8 consecutive channels of one row; W is read once and reused
+// for every alpha; rows d_out..d_out_pad-1 of each slice are written as zeros.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) fake_quant_delta(const __nv_bfloat16* __restrict__ W, int d_out, int d_in,
+                                                        int d_out_pad, const float* __restrict__ s_all,
+                                                        const float* __restrict__ inv_all, int n_alpha, int bits,
+                                                        int symmetric, int gl, __nv_bfloat16* __restrict__ dW) {
+  const int chunks = d_in >> 3;
+  const long long total = (long long)d_out_pad * chunks;
+  const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool sym = symmetric != 0;
+  const long long slice = (long long)d_out_pad * d_in;
+  for (long long base = warp_global * 32; base < total; base += n_warps * 32) {
+    const long long u = base + lane;
+    const bool active = u < total;
+    const int row = active ? (int)(u / chunks) : 0;
+    const int c0 = active ? (int)(u - (long long)row * chunks) * 8 : 0;
+    const bool real = active && row < d_out;
+    float w[8];
+    if (real) {
+      unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(W + (long long)row * d_in + c0)), w);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w[j] = 0.f;
+    }
+    for (int k = 0; k < n_alpha; ++k) {
+      float s[8], is[8], v[8];
+      const float4* sp = reinterpret_cast<const float4*>(s_all + (long long)k * d_in + c0);
+      const float4* ip = reinterpret_cast<const float4*>(inv_all + (long long)k * d_in + c0);
+      const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1), i0 = __ldg(ip), i1 = __ldg(ip + 1);
+      s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w; s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
+      is[0] = i0.x; is[1] = i0.y; is[2] = i0.z; is[3] = i0.w; is[4] = i1.x; is[5] = i1.y; is[6] = i1.z; is[7] = i1.w;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = w[j] * s[j];
+      FqResult fr;
+      fq_group8(v, bits, sym, gl, fr);
+      uint32_t out[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float d0 = real ? fq_dequant(fr, 2 * h, sym) * is[2 * h] - w[2 * h] : 0.f;
+        const float d1 = real ? fq_dequant(fr, 2 * h + 1, sym) * is[2 * h + 1] - w[2 * h + 1] : 0.f;
+        __nv_bfloat162 p = __floats2bfloat162_rn(d0, d1);
+        out[h] = *reinterpret_cast<uint32_t*>(&p);
+      }
+      if (active)
+        __stcs(reinterpret_cast<uint4*>(dW + k * slice + (long long)row * d_in + c0),
+               make_uint4(out[0], out[1], out[2], out[3]));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a4 feed: XT[i][t] = X[t][i] (tokens padded with zeros to ld_t columns), so
+// that G = X^T X is a K-major product of XT with itself.
+// ---------------------------------------------------------------------------
+__global__ void transpose_bf16(const __nv_bfloat16* __restrict__ X, long long N, int d_in, long long ld_t,
+                               __nv_bfloat16* __restrict__ XT) {
+  __shared__ __nv_bfloat16 tile[64][65];
+  const long long t0 = (long long)blockIdx.x * 64;
+  const int i0 = blockIdx.y * 64;
+  for (int k = threadIdx.y; k < 64; k += blockDim.y) {
+    const long long t = t0 + k;
+    const int i = i0 + threadIdx.x;
+    __nv_bfloat16 v = __float2bfloat16(0.f);
+    if (t < N && i < d_in) v = X[t * d_in + i];
+    tile[k][threadIdx.x] = v;
+  }
+  __syncthreads();
+  for (int k = threadIdx.y; k < 64; k += blockDim.y) {
+    const int i = i0 + k;
+    const long long t = t0 + threadIdx.x;
+    if (i < d_in && t < ld_t) XT[(long long)i * ld_t + t] = tile[threadIdx.x][k];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a6, first half: per-row losses l[k][r] = sum over column tiles of the
+// contraction's partials (fp64, column tiles in order), optional fp32 copy,
+// and per-block fp64 sums (fixed tree) per alpha.
+// part layout: [n_blocks_n][M] with M = n_alpha * d_out_pad, row = k*d_out_pad + r.
+// ---------------------------------------------------------------------------
+constexpr int REDUCE_THREADS = 256;
+
+__global__ void __launch_bounds__(REDUCE_THREADS) row_loss_reduce(const float* __restrict__ part, int n_blocks_n,
+                                                                  long long M, int d_out, int d_out_pad,
+                                                                  float* __restrict__ row_losses,
+                                                                  double* __restrict__ block_sums) {
+  __shared__ double red[REDUCE_THREADS];
+  const int k = blockIdx.y;
+  const int r = blockIdx.x * REDUCE_THREADS + threadIdx.x;
+  double s = 0.0;
+  if (r < d_out) {
+    const long long m = (long long)k * d_out_pad + r;
+    for (int nb = 0; nb < n_blocks_n; ++nb) s += (double)part[(long long)nb * M + m];
+    if (row_losses) row_losses[(long long)k * d_out + r] = (float)s;
+  }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = REDUCE_THREADS / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) block_sums[(long long)k * gridDim.x + blockIdx.x] = red[0];
+}
+
+// a6, second half: losses, argmin (lowest index on ties), s_best. One block.
+__global__ void loss_argmin(const double* __restrict__ block_sums, int n_chunks, int n_alpha,
+                            const float* __restrict__ s_all, int d_in, float* __restrict__ losses,
+                            double* __restrict__ losses64, int* __restrict__ best_out, float* __restrict__ s_best,
+                            int* err) {
+  __shared__ double L[MAX_ALPHA];
+  __shared__ int best_sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int k = warp; k < n_alpha; k += nw) {
+    double s = 0.0;
+    for (int c = lane; c < n_chunks; c += 32) s += block_sums[(long long)k * n_chunks + c];
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) L[k] = s;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // warp-shuffle argmin over (loss, index); ties go to the lower index
+    double bv = INFINITY;
+    int bi = MAX_ALPHA;
+    bool finite = true;
+    for (int k = lane; k < n_alpha; k += 32) {
+      const double v = L[k];
+      if (!isfinite(v)) finite = false;
+      if (v < bv) {
+        bv = v;
+        bi = k;
+      }
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (ov < bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    finite = __all_sync(0xffffffffu, finite);
+    if (lane == 0) {
+      best_sh = finite ? bi : -1;
+      *best_out = best_sh;
+      if (!finite && err) atomicCAS(err, 0, ERR_NONFINITE);
+    }
+    for (int k = lane; k < n_alpha; k += 32) {
+      losses[k] = (float)L[k];
+      losses64[k] = L[k];
+    }
+  }
+  __syncthreads();
+  const int b = best_sh;
+  for (int i = threadIdx.x; i < d_in; i += blockDim.x)
+    s_best[i] = b >= 0 ? s_all[(long long)b * d_in + i] : __int_as_float(0x7fc00000);
+}
+
+// ---------------------------------------------------------------------------
+// a7: pack. Codes of Q(W S) (same quantiser as the search), 8 nibbles per
+// uint32 (channel 8w+j in bits 4j..4j+3), fp16 step and zero per group.
+// ([P2] §2.1 INT4 with fp16 scale, §4.2 packed 4-bit storage; [P4] §三.)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __restrict__ W, const float* __restrict__ s,
+                                                     int d_out, int d_in, int bits, int symmetric, int gl,
+                                                     uint32_t* __restrict__ qweight, __half* __restrict__ scales,
+                                                     __half* __restrict__ zeros) {
+  const int chunks = d_in >> 3;
+  const long long total = (long long)d_out * chunks;
+  const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool sym = symmetric != 0;
+  const int groups = d_in / (gl * 8);
+  for (long long base = warp_global * 32; base < total; base += n_warps * 32) {
+    const long long u = base + lane;
+    const bool active = u < total;
+    const int row = active ? (int)(u / chunks) : 0;
+    const int chunk = active ? (int)(u - (long long)row * chunks) : 0;
+    const int c0 = chunk * 8;
+    float v[8];
+    if (active) {
+      float w[8];
+      unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(W + (long long)row * d_in + c0)), w);
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + c0));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + c0 + 4));
+      v[0] = w[0] * s0.x; v[1] = w[1] * s0.y; v[2] = w[2] * s0.z; v[3] = w[3] * s0.w;
+      v[4] = w[4] * s1.x; v[5] = w[5] * s1.y; v[6] = w[6] * s1.z; v[7] = w[7] * s1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = 0.f;
+    }
+    FqResult fr;
+    fq_group8(v, bits, sym, gl, fr);
+    if (active) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) word |= (fq_code(fr, j, sym) & 0xFu) << (4 * j);
+      qweight[(long long)row * chunks + chunk] = word;
+      if ((chunk & (gl - 1)) == 0) {
+        const long long gidx = (long long)row * groups + chunk / gl;
+        scales[gidx] = __float2half_rn(fr.delta);
+        zeros[gidx] = __float2half_rn(fr.zero);
+      }
+    }
+  }
+}
+
+}  // namespace awq

@@ -1,0 +1,278 @@
+// Persistent tcgen05 GEMM for sm_100a with the AWQ loss epilogues.
+//
+// D[m, n] = sum_k A[m, k] * B[n, k]   (A [M, K], B [N, K], both bf16 row-major,
+// i.e. K-major operands), fp32 accumulation in tensor memory. Tiles are
+// 128 x 256 (one CTA per SM, cta_group::1, M=128 N=256 K=16 instructions),
+// K is staged 64 at a time through a 4-deep shared-memory ring filled by TMA
+// (128-byte swizzle, no multicast).
+//
+// Warp roles (192 threads):
+//   warp 0      one thread issues the TMA loads of A and B;
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
+//               one thread issues tcgen05.mma, committing each stage back to
+//               the loader and each finished tile to the epilogue;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32*(w%4)..+31, i.e. tile rows), then one of
+//     EPI_SUMSQ  part[n_blk][m] = sum_{n in tile} D[m,n]^2         (||dW X^T||^2)
+//     EPI_DOT    part[n_blk][m] = sum_{n in tile} D[m,n] E[m,n]    (trace(dW G dW^T))
+//     EPI_STORE  C[m, n] = bf16(D[m, n])                            (G = X^T X)
+// The accumulator is released before the partials are written, so the next
+// tile's MMAs overlap this tile's epilogue.
+//
+// Tiles are visited in groups of `group_n` N-blocks (M-major inside a group)
+// so that the CTAs running at one time share A panels and a B slice in L2.
+// Every wait is bounded (ptx.cuh); on a timeout the CTA records an error in
+// *err, drains its in-flight TMA loads and MMAs, frees TMEM and returns.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+
+namespace awq {
+
+enum EpiMode { EPI_SUMSQ = 0, EPI_DOT = 1, EPI_STORE = 2 };
+
+constexpr int GEMM_BM = 128;
+constexpr int GEMM_BN = 256;
+constexpr int GEMM_BK = 64;
+constexpr int GEMM_STAGES = 4;
+constexpr int GEMM_THREADS = 192;
+constexpr int GEMM_A_STAGE = GEMM_BM * GEMM_BK * 2;  // 16 KB
+constexpr int GEMM_B_STAGE = GEMM_BN * GEMM_BK * 2;  // 32 KB
+constexpr int GEMM_TMEM_COLS = 512;
+constexpr int GEMM_SMEM_BYTES = 1024 /* alignment slack */ + GEMM_STAGES * (GEMM_A_STAGE + GEMM_B_STAGE) + 256;
+
+// error codes written to *err by the GEMM (distinct per wait site)
+constexpr int ERR_WAIT_EMPTY = 0x101, ERR_WAIT_FULL = 0x102, ERR_WAIT_TEMPTY = 0x103, ERR_WAIT_TFULL = 0x104;
+
+struct GemmArgs {
+  int M, N, K;                 // problem size (rows of A, rows of B, contraction length)
+  int n_blocks_m, n_blocks_n;  // ceil(M/128), ceil(N/256)
+  int group_n;                 // raster group width in N-blocks
+  float* part;                 // SUMSQ / DOT: [n_blocks_n][M] per-row partial sums
+  const __nv_bfloat16* E;      // DOT: E[M, ldE]; element (m, n) multiplies D[m, n]
+  long long ldE;
+  __nv_bfloat16* C;            // STORE: C[M, ldC]
+  long long ldC;
+  int* err;                    // device error word
+};
+
+__device__ __forceinline__ void gemm_tile_coords(int t, const GemmArgs& a, int& mb, int& nb) {
+  const int gn = a.group_n;
+  const int per_group = a.n_blocks_m * gn;
+  const int g = t / per_group;
+  const int first = g * gn;
+  const int width = min(gn, a.n_blocks_n - first);
+  const int r = t - g * per_group;
+  mb = r / width;
+  nb = first + (r - mb * width);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <int MODE>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + GEMM_STAGES * GEMM_A_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + GEMM_STAGES * GEMM_B_STAGE);
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * GEMM_STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + GEMM_STAGES + s); };
+  auto tfull_bar = [&](int a) { return smem_u32(bars + 2 * GEMM_STAGES + a); };
+  auto tempty_bar = [&](int a) { return smem_u32(bars + 2 * GEMM_STAGES + 2 + a); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * GEMM_STAGES + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GEMM_STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), GEMM_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = args.n_blocks_m * args.n_blocks_n;
+  const int num_kb = (args.K + GEMM_BK - 1) / GEMM_BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, last_parity = 0;  // bit s: stage s has been loaded; parity of its last load
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+        int mb, nb;
+        gemm_tile_coords(t, args, mb, nb);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.err, ERR_WAIT_EMPTY)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), GEMM_A_STAGE + GEMM_B_STAGE);
+          tma_load_2d(smem_u32(sA + stage * GEMM_A_STAGE), &tmA, full_bar(stage), kb * GEMM_BK, mb * GEMM_BM);
+          tma_load_2d(smem_u32(sB + stage * GEMM_B_STAGE), &tmB, full_bar(stage), kb * GEMM_BK, nb * GEMM_BN);
+          issued |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == GEMM_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // every issued load must have landed before the CTA may exit
+      for (int s = 0; s < GEMM_STAGES; ++s)
+        if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (last_parity >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, GEMM_BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.err, ERR_WAIT_TEMPTY)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * GEMM_BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, args.err, ERR_WAIT_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * GEMM_A_STAGE);
+          const uint32_t b_base = smem_u32(sB + stage * GEMM_B_STAGE);
+#pragma unroll
+          for (int k = 0; k < GEMM_BK / 16; ++k) {
+            mma_bf16(d_tmem, desc_kmajor_sw128(a_base + k * 32), desc_kmajor_sw128(b_base + k * 32), IDESC,
+                     (kb | k) != 0);
+          }
+          mma_commit(empty_bar(stage));
+          if (++stage == GEMM_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) mma_commit(tfull_bar(acc));
+      }
+      // all MMAs of this thread must complete before TMEM is freed
+      mma_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5)
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    int local = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+      int mb, nb;
+      gemm_tile_coords(t, args, mb, nb);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      // warp-uniform decision: the tcgen05.ld below is .sync.aligned
+      const bool ready = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, args.err, ERR_WAIT_TFULL);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * GEMM_BN;
+      const int m = mb * GEMM_BM + row_in_tile;
+      const int n0 = nb * GEMM_BN;
+      float sum = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < GEMM_BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, r);
+        tmem_ld_wait();
+        if constexpr (MODE == EPI_SUMSQ) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float d = __uint_as_float(r[j]);
+            sum = fmaf(d, d, sum);
+          }
+        } else if constexpr (MODE == EPI_DOT) {
+          const int col = n0 + c * 32;
+          if (m < args.M) {
+            const __nv_bfloat16* erow = args.E + (long long)m * args.ldE + col;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col + v * 8 < args.N) {
+                const uint4 e = __ldg(reinterpret_cast<const uint4*>(erow + v * 8));
+                const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  sum = fmaf(__uint_as_float(r[v * 8 + 2 * h]), bf16lo(ew[h]), sum);
+                  sum = fmaf(__uint_as_float(r[v * 8 + 2 * h + 1]), bf16hi(ew[h]), sum);
+                }
+              }
+            }
+          }
+        } else {
+          const int col = n0 + c * 32;
+          if (m < args.M) {
+            __nv_bfloat16* crow = args.C + (long long)m * args.ldC + col;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col + v * 8 < args.N) {
+                uint32_t w[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  __nv_bfloat162 p = __floats2bfloat162_rn(__uint_as_float(r[v * 8 + 2 * h]),
+                                                           __uint_as_float(r[v * 8 + 2 * h + 1]));
+                  w[h] = *reinterpret_cast<uint32_t*>(&p);
+                }
+                *reinterpret_cast<uint4*>(crow + v * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if constexpr (MODE != EPI_STORE) {
+        if (m < args.M) args.part[(long long)nb * args.M + m] = sum;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, GEMM_TMEM_COLS);
+  }
+}
+
+}  // namespace awq
