@@ -55,6 +55,24 @@ def check_pack(Wb, s_ref, q, sc, zr, bits, g, sym):
     return int((codes != codes_ref).sum()), int(near.sum())
 
 
+def check_row_losses(Wb, Xb, a_ref, wl, rows, rl_gpu):
+    """Per-row losses of the given rows against the oracle. A row holding an
+    element whose code the oracle decides within 1e-4 of a rounding boundary
+    may legitimately differ by more (one flipped code moves its row's loss by
+    up to a few percent); such rows are counted and left to the total-loss
+    check."""
+    sub = O.search(Wb, Xb, a_ref, wl.bits, wl.group, wl.symmetric, wl.n_alpha, rows=rows)
+    ref = sub["row_losses"]
+    got = rl_gpu[:, rows]
+    tol = LOSS_RTOL * ref + 1e-3 * ref.mean()
+    ok = np.abs(got - ref) <= tol
+    near = np.stack([O.boundary_mask(Wb[rows], O.candidate_scales(a_ref, al), wl.bits, wl.group,
+                                     wl.symmetric).any(axis=1) for al in O.alpha_grid(wl.n_alpha)])
+    bad = ~ok & ~near
+    assert not bad.any(), f"{bad.sum()} (alpha, row) losses differ away from rounding boundaries"
+    return int((~ok).sum()), int(near.sum())
+
+
 def run_case(wl, form="auto", check_rows=True):
     Wb, Xb = make_inputs(wl)
     W, X = to_device(Wb), to_device(Xb)
@@ -74,9 +92,7 @@ def run_case(wl, form="auto", check_rows=True):
     rl = res["row_losses"].cpu().numpy().astype(np.float64)
     assert np.allclose(rl.sum(axis=1), losses, rtol=1e-5)
     if check_rows:
-        sub = O.search(Wb, Xb, a_ref, wl.bits, wl.group, wl.symmetric, wl.n_alpha, rows=np.arange(wl.d_out))
-        tol = LOSS_RTOL * sub["row_losses"] + 1e-3 * sub["row_losses"].mean()
-        assert np.all(np.abs(rl - sub["row_losses"]) <= tol)
+        check_row_losses(Wb, Xb, a_ref, wl, np.arange(wl.d_out), rl)
     best = int(res["best"].item())
     assert best in O.acceptable_choices(ref["losses"], TIE_REL), (best, ref["best"], ref["losses"])
     s_ref = O.candidate_scales(a_ref, O.alpha_grid(wl.n_alpha)[best])
