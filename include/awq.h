@@ -81,6 +81,26 @@ awq_status awq_act_stats(const void* X_bf16, int64_t N, int64_t d_in, float* a, 
                          size_t ws_bytes, awq_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Step a1 for callers that cannot allocate device memory (no counterpart on
+ * the pages; it exists for the library's users). Same result as
+ * awq_act_stats, but the fp64 partial sums go to a fixed scratch array of
+ * 4 MiB (524288 doubles) compiled into the library, which every GPU that
+ * loads the library holds until the process exits. No cudaMalloc, cudaFree or
+ * other allocating call is made.
+ *   - Limits: N >= 1, d_in a multiple of 8 and at most 524288; larger d_in
+ *     returns AWQ_ERR_SHAPE (tall inputs use fewer, taller row chunks).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls in the process share the one array: calls whose work overlaps
+ *     on the GPU (different streams or threads) race and give wrong results.
+ *     Calls ordered on one stream are safe; nothing needs clearing between
+ *     them because every partial read is first written by the same call.
+ * Other errors as awq_act_stats.
+ * ------------------------------------------------------------------------- */
+awq_status awq_act_stats_noalloc(const void* X_bf16, int64_t N, int64_t d_in, float* a, awq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Steps a2-a6: the scale search.
  * For each alpha_k of the grid:
  *   s_i = max(a_i, eps_a)^alpha_k / sqrt(max_j s_j * min_j s_j)      ([P5] §4.1)

@@ -24,7 +24,7 @@ EXPORTED = (
     "awq_status_str", "awq_stats_workspace_size", "awq_act_stats", "awq_search_workspace_size",
     "awq_search_scales", "awq_search_form", "awq_workspace_error", "awq_quantize_pack",
     "awq_step_scales", "awq_step_fake_quant", "awq_step_gram", "awq_step_contract", "awq_step_reduce",
-    "awq_debug_copy_dw",
+    "awq_debug_copy_dw", "awq_act_stats_noalloc",
 )
 
 
@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
             "awq_status_str": (c_char_p, [c_int32]),
             "awq_stats_workspace_size": (c_size_t, [c_int64, c_int64]),
             "awq_act_stats": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_size_t, c_void_p]),
+            "awq_act_stats_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
             "awq_search_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, cfgp]),
             "awq_search_form": (c_int32, [c_int64, c_int64, c_int64, cfgp]),
             "awq_search_scales": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, cfgp,

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/awq.h"
 #include "awq_kernels.cuh"
@@ -417,3 +418,70 @@ awq_status awq_debug_copy_dw(const void* ws, int64_t d_out, int64_t d_in, int64_
 }
 
 }  // extern "C"
+
+// =================================================================== statistics without allocation
+// Some callers cannot allocate device memory at the point where they need the
+// activation statistics: code that runs inside a memory pool or arena they do
+// not own, a plugin host that hands out only its own tensors, or a region where
+// a cudaMalloc would synchronise the device. For them awq_act_stats_noalloc
+// takes its scratch from a fixed array that lives in this library's device
+// image instead of from a caller workspace.
+namespace {
+
+constexpr long long kNoallocScratchDoubles = 1ll << 19;  // 4 MiB of fp64 partial sums
+constexpr int kNoallocMaxDevices = 64;
+
+// Loaded on every device that loads the library and held until the process exits.
+static __device__ __align__(256) double g_noalloc_stats_scratch[kNoallocScratchDoubles];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Device address of the scratch array on the current device. In host code the
+// array's name is only a host-side stand-in, so its address is looked up once
+// per device (with that device current) and cached.
+awq_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return AWQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_stats_scratch) != cudaSuccess || !p) return AWQ_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return AWQ_OK;
+}
+
+}  // namespace
+
+extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t d_in, float* a, awq_stream_t stream) {
+  if (!X || !a) return AWQ_ERR_INVALID_ARG;
+  if (!aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
+  if (check_tokens(N) != AWQ_OK || d_in < 8 || d_in % 8 != 0 || d_in > kNoallocScratchDoubles) return AWQ_ERR_SHAPE;
+  // same chunking as awq_act_stats, with fewer, taller row chunks when the
+  // partial sums (one fp64 per chunk and channel) would not fit the array
+  StatsLayout L = stats_layout(N, d_in);
+  const long long max_chunks = kNoallocScratchDoubles / d_in;
+  if ((long long)L.n_chunks > max_chunks) {
+    long long rpc = cdiv(N, max_chunks);
+    rpc = cdiv(rpc, 32) * 32;
+    L.rows_per_chunk = (int)rpc;
+    L.n_chunks = (int)cdiv(N, rpc);
+  }
+  if ((long long)L.n_chunks * d_in > kNoallocScratchDoubles) return AWQ_ERR_SHAPE;
+  awq_status st = check_device(nullptr);
+  if (st != AWQ_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != AWQ_OK) return st;
+  double* part = static_cast<double*>(scratch);
+  cudaStream_t s = as_stream(stream);
+  // every partial the second kernel reads is written by the first one in this
+  // call, so nothing needs clearing between calls
+  act_absmean_partial<<<dim3(L.col_blocks, L.n_chunks), STATS_THREADS, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(X), N, (int)d_in, L.rows_per_chunk, part);
+  if ((st = launch_status()) != AWQ_OK) return st;
+  act_absmean_final<<<(unsigned)cdiv(d_in, 256), 256, 0, s>>>(part, L.n_chunks, N, (int)d_in, a);
+  return launch_status();
+}
