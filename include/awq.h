@@ -126,8 +126,11 @@ awq_status awq_search_scales(const void* W_bf16, const void* X_bf16, const float
                              awq_stream_t stream);
 
 /* The contraction form awq_search_scales will use for these sizes (1 direct,
- * 2 Gram): AUTO picks the one with fewer multiply-adds,
- * n_alpha*d_out*d_in*N versus N*d_in^2 + n_alpha*d_out*d_in^2. */
+ * 2 Gram): AUTO picks the one with fewer multiply-adds, n_alpha*d_out*d_in*N
+ * versus (N + n_alpha*d_out) * T(d_in), where T(d_in) ~ d_in^2/2 counts the
+ * lower block triangle of the symmetric G = X^T X (256-wide blocks) that the
+ * Gram form evaluates: sum_{i,j} dW_i G_ij dW_j over j's block <= i's block,
+ * off-diagonal blocks doubled. */
 int32_t awq_search_form(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg);
 
 /* Read back (synchronising `stream`) the device error word of a search or

@@ -37,10 +37,12 @@ def test_status_strings():
 
 def test_workspace_sizes_and_form():
     cfg = awq.make_cfg(4, 128, False, 20)
-    # C2 shape: direct form; stack of 20 x 4096 x 4096 bf16 dominates
+    # C2 shape: the stack of 20 x 4096 x 4096 bf16 dominates; N = d_in, so the
+    # block-triangular Gram form needs about half the multiply-adds of the direct one
     n = awq.search_workspace_size(4096, 4096, 4096, cfg)
     assert n >= 20 * 4096 * 4096 * 2
-    assert awq.search_form(4096, 4096, 4096, cfg) == "direct"
+    assert awq.search_form(4096, 4096, 4096, cfg) == "gram"
+    assert awq.search_form(4096, 4096, 1024, cfg) == "direct"
     assert awq.search_form(11008, 4096, 16384, cfg) == "gram"
     assert awq.search_form(28672, 8192, 65536, cfg) == "gram"
     assert awq.search_form(4096, 11008, 16384, awq.make_cfg(3, 64, True, 20)) == "gram"

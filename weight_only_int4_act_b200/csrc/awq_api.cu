@@ -113,10 +113,23 @@ struct SearchLayout {
   size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_xt, off_g, total;
 };
 
+// sum over 256-wide column blocks J of width(J) * min(d_in, 256 (J + 1)): the
+// multiply-adds per row of the block-triangular Gram contraction
+double tri_macs_per_row(int64_t d_in) {
+  double t = 0.0;
+  for (int64_t j0 = 0; j0 < d_in; j0 += GEMM_BN) {
+    const int64_t w = d_in - j0 < GEMM_BN ? d_in - j0 : GEMM_BN;
+    const int64_t k = j0 + GEMM_BN < d_in ? j0 + GEMM_BN : d_in;
+    t += (double)w * (double)k;
+  }
+  return t;
+}
+
 int choose_form(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg) {
   if (cfg->form == AWQ_FORM_DIRECT || cfg->form == AWQ_FORM_GRAM) return cfg->form;
   const double direct = (double)cfg->n_alpha * d_out * d_in * N;
-  const double gram = (double)N * d_in * d_in + (double)cfg->n_alpha * d_out * d_in * d_in;
+  const double tri = tri_macs_per_row(d_in);
+  const double gram = (double)N * tri + (double)cfg->n_alpha * d_out * tri;
   return direct <= gram ? AWQ_FORM_DIRECT : AWQ_FORM_GRAM;
 }
 
@@ -190,7 +203,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 // D = A[M, K] * B[Nr, K]^T with the given epilogue.
 template <int MODE>
 awq_status run_gemm(const void* A, long long M, long long lda, const void* B, long long Nr, long long ldb, long long K,
-                    GemmArgs args, int num_sms, cudaStream_t st) {
+                    GemmArgs args, int tri, int num_sms, cudaStream_t st) {
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, M, K, lda, GEMM_BM)) return AWQ_ERR_CUDA;
   if (!make_map(&tb, B, Nr, K, ldb, GEMM_BN)) return AWQ_ERR_CUDA;
@@ -200,10 +213,14 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
   args.n_blocks_m = (int)cdiv(M, GEMM_BM);
   args.n_blocks_n = (int)cdiv(Nr, GEMM_BN);
   args.group_n = kGroupN < args.n_blocks_n ? kGroupN : args.n_blocks_n;
+  args.tri = tri;
+  const long long tiles = tri == TRI_LOWER_STORE ? tri_lower_tiles(args.n_blocks_m)
+                                                 : (long long)args.n_blocks_m * args.n_blocks_n;
+  if (tiles > INT32_MAX) return AWQ_ERR_SHAPE;
+  args.num_tiles = (int)tiles;
   if (cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) !=
       cudaSuccess)
     return AWQ_ERR_CUDA;
-  const long long tiles = (long long)args.n_blocks_m * args.n_blocks_n;
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
   gemm_bf16_tcgen05<MODE><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(ta, tb, args);
   return launch_status();
@@ -294,7 +311,7 @@ awq_status awq_step_fake_quant(const void* W, int64_t d_out, int64_t d_in, int64
   if (!W || !aligned(W, 16)) return AWQ_ERR_INVALID_ARG;
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;
-  const long long units = (long long)L.d_out_pad * (d_in / 8);
+  const long long units = (long long)(L.d_out_pad / FQ_ROWS) * (d_in / 8);
   fake_quant_delta<<<elementwise_grid(units, sms), 256, 0, as_stream(stream)>>>(
       static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in, L.d_out_pad, at<float>(ws, L.off_s),
       at<float>(ws, L.off_inv), cfg->n_alpha, cfg->bits, cfg->symmetric, cfg->group / 8,
@@ -321,7 +338,7 @@ awq_status awq_step_gram(const void* X, int64_t d_out, int64_t d_in, int64_t N, 
   ga.ldC = d_in;
   ga.err = at<int>(ws, 0);
   const void* xt = at<void>(ws, L.off_xt);
-  return run_gemm<EPI_STORE>(xt, d_in, L.ld_t, xt, d_in, L.ld_t, L.ld_t, ga, sms, s);
+  return run_gemm<EPI_STORE>(xt, d_in, L.ld_t, xt, d_in, L.ld_t, L.ld_t, ga, TRI_LOWER_STORE, sms, s);
 }
 
 awq_status awq_step_contract(const void* X, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
@@ -337,11 +354,12 @@ awq_status awq_step_contract(const void* X, int64_t d_out, int64_t d_in, int64_t
   const void* dw = at<void>(ws, L.off_dw);
   if (L.form == AWQ_FORM_DIRECT) {
     if (!X || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
-    return run_gemm<EPI_SUMSQ>(dw, L.M, d_in, X, N, d_in, d_in, ga, sms, as_stream(stream));
+    return run_gemm<EPI_SUMSQ>(dw, L.M, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, as_stream(stream));
   }
   ga.E = at<__nv_bfloat16>(ws, L.off_dw);
   ga.ldE = d_in;
-  return run_gemm<EPI_DOT>(dw, L.M, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, sms, as_stream(stream));
+  return run_gemm<EPI_DOT>(dw, L.M, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms,
+                           as_stream(stream));
 }
 
 awq_status awq_step_reduce(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws, size_t ws_bytes,

@@ -138,15 +138,18 @@ __global__ void candidate_scales(const float* __restrict__ a, int d_in, AlphaGri
 // ---------------------------------------------------------------------------
 // a3: dW[k][r][:] = Q(W_r S_k) S_k^-1 - W_r as bf16, for every alpha k.
 // ([P1] 缩放保护 W~ = sW, W^ = Q(W~)/s; [P5] §2.2 Q(WS)S^-1.)
-// One thread = 8 consecutive channels of one row; W is read once and reused
-// for every alpha; rows d_out..d_out_pad-1 of each slice are written as zeros.
+// One thread = 8 consecutive channels of FQ_ROWS consecutive rows: W is read
+// once and reused for every alpha, and each alpha's 8 scales are loaded once
+// for the FQ_ROWS rows. Rows d_out..d_out_pad-1 of each slice are zeros.
 // ---------------------------------------------------------------------------
+constexpr int FQ_ROWS = 4;
+
 __global__ void __launch_bounds__(256) fake_quant_delta(const __nv_bfloat16* __restrict__ W, int d_out, int d_in,
                                                         int d_out_pad, const float* __restrict__ s_all,
                                                         const float* __restrict__ inv_all, int n_alpha, int bits,
                                                         int symmetric, int gl, __nv_bfloat16* __restrict__ dW) {
   const int chunks = d_in >> 3;
-  const long long total = (long long)d_out_pad * chunks;
+  const long long total = (long long)(d_out_pad / FQ_ROWS) * chunks;
   const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -155,38 +158,48 @@ __global__ void __launch_bounds__(256) fake_quant_delta(const __nv_bfloat16* __r
   for (long long base = warp_global * 32; base < total; base += n_warps * 32) {
     const long long u = base + lane;
     const bool active = u < total;
-    const int row = active ? (int)(u / chunks) : 0;
-    const int c0 = active ? (int)(u - (long long)row * chunks) * 8 : 0;
-    const bool real = active && row < d_out;
-    float w[8];
-    if (real) {
-      unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(W + (long long)row * d_in + c0)), w);
-    } else {
+    const int quad = active ? (int)(u / chunks) : 0;
+    const int c0 = active ? (int)(u - (long long)quad * chunks) * 8 : 0;
+    const int row0 = quad * FQ_ROWS;
+    float w[FQ_ROWS][8];
+    bool real[FQ_ROWS];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) w[j] = 0.f;
+    for (int r = 0; r < FQ_ROWS; ++r) {
+      real[r] = active && row0 + r < d_out;
+      if (real[r]) {
+        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0)), w[r]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[r][j] = 0.f;
+      }
     }
+    __nv_bfloat16* out_base = dW + (long long)row0 * d_in + c0;
     for (int k = 0; k < n_alpha; ++k) {
-      float s[8], is[8], v[8];
+      float s[8], is[8];
       const float4* sp = reinterpret_cast<const float4*>(s_all + (long long)k * d_in + c0);
       const float4* ip = reinterpret_cast<const float4*>(inv_all + (long long)k * d_in + c0);
       const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1), i0 = __ldg(ip), i1 = __ldg(ip + 1);
       s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w; s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
       is[0] = i0.x; is[1] = i0.y; is[2] = i0.z; is[3] = i0.w; is[4] = i1.x; is[5] = i1.y; is[6] = i1.z; is[7] = i1.w;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = w[j] * s[j];
-      FqResult fr;
-      fq_group8(v, bits, sym, gl, fr);
-      uint32_t out[4];
+      for (int r = 0; r < FQ_ROWS; ++r) {
+        float v[8];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float d0 = real ? fq_dequant(fr, 2 * h, sym) * is[2 * h] - w[2 * h] : 0.f;
-        const float d1 = real ? fq_dequant(fr, 2 * h + 1, sym) * is[2 * h + 1] - w[2 * h + 1] : 0.f;
-        __nv_bfloat162 p = __floats2bfloat162_rn(d0, d1);
-        out[h] = *reinterpret_cast<uint32_t*>(&p);
+        for (int j = 0; j < 8; ++j) v[j] = w[r][j] * s[j];
+        FqResult fr;
+        fq_group8(v, bits, sym, gl, fr);
+        uint32_t out[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float d0 = real[r] ? fq_dequant(fr, 2 * h, sym) * is[2 * h] - w[r][2 * h] : 0.f;
+          const float d1 = real[r] ? fq_dequant(fr, 2 * h + 1, sym) * is[2 * h + 1] - w[r][2 * h + 1] : 0.f;
+          __nv_bfloat162 p = __floats2bfloat162_rn(d0, d1);
+          out[h] = *reinterpret_cast<uint32_t*>(&p);
+        }
+        if (active)
+          __stcs(reinterpret_cast<uint4*>(out_base + k * slice + (long long)r * d_in),
+                 make_uint4(out[0], out[1], out[2], out[3]));
       }
-      if (active)
-        __stcs(reinterpret_cast<uint4*>(dW + k * slice + (long long)row * d_in + c0),
-               make_uint4(out[0], out[1], out[2], out[3]));
     }
   }
 }

@@ -13,13 +13,19 @@
 //   asymmetric: Delta = max(max v - min v, eps) / (2^b - 1)
 //               z = clamp(rne(-min v / Delta), 0, 2^b - 1)
 //               q = clamp(rne(v / Delta) + z, 0, 2^b - 1),   v_hat = (q - z) Delta
-// Arithmetic is fp32; v / Delta is taken as v * (1 / Delta).
+// Arithmetic is fp32; Delta is the range times the fp32 constant 1/levels and
+// v / Delta is taken as v * (1 / Delta) (correctly rounded reciprocal).
 #pragma once
 #include <cuda_runtime.h>
 
 namespace awq {
 
 constexpr float kEpsDelta = 1e-8f;
+
+// 1 / (2^b - 1) rounded to fp32, for b = 1..4 (the step is range * this).
+__device__ __forceinline__ float inv_levels(int b) {
+  return b == 4 ? (1.0f / 15.0f) : b == 3 ? (1.0f / 7.0f) : b == 2 ? (1.0f / 3.0f) : 1.0f;
+}
 
 struct FqResult {
   float delta;  // quantisation step of the group
@@ -35,8 +41,8 @@ __device__ __forceinline__ void fq_group8(const float (&v)[8], int bits, bool sy
     for (int off = 1; off < gl; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
     const float qmax = (float)((1 << (bits - 1)) - 1);
     const float qmin = -(float)(1 << (bits - 1));
-    r.delta = fmaxf(amax, kEpsDelta) / qmax;
-    const float inv = 1.0f / r.delta;
+    r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
+    const float inv = __frcp_rn(r.delta);
     r.zero = -qmin;
 #pragma unroll
     for (int j = 0; j < 8; ++j) r.q[j] = fminf(fmaxf(rintf(v[j] * inv), qmin), qmax);
@@ -52,8 +58,8 @@ __device__ __forceinline__ void fq_group8(const float (&v)[8], int bits, bool sy
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     }
     const float levels = (float)((1 << bits) - 1);
-    r.delta = fmaxf(mx - mn, kEpsDelta) / levels;
-    const float inv = 1.0f / r.delta;
+    r.delta = fmaxf(mx - mn, kEpsDelta) * inv_levels(bits);
+    const float inv = __frcp_rn(r.delta);
     r.zero = fminf(fmaxf(rintf(-mn * inv), 0.f), levels);
 #pragma unroll
     for (int j = 0; j < 8; ++j) r.q[j] = fminf(fmaxf(rintf(v[j] * inv) + r.zero, 0.f), levels);

@@ -21,6 +21,13 @@
 //
 // Tiles are visited in groups of `group_n` N-blocks (M-major inside a group)
 // so that the CTAs running at one time share A panels and a B slice in L2.
+//
+// Block-triangular modes (the Gram form uses the symmetry of G = X^T X, with
+// 256-wide channel blocks J): TRI_LOWER_STORE computes only the tiles of G
+// whose column block is <= their row block and stores G' = 2G on strictly
+// lower blocks, G on diagonal blocks; TRI_K then stops the contraction of
+// column tile J at k < 256(J+1), so that sum over tiles of (dW G')[m, J] dW[m, J]
+// = dW G dW^T (each off-diagonal block pair counted once, doubled).
 // Every wait is bounded (ptx.cuh); on a timeout the CTA records an error in
 // *err, drains its in-flight TMA loads and MMAs, frees TMEM and returns.
 #pragma once
@@ -47,8 +54,12 @@ constexpr int GEMM_SMEM_BYTES = 1024 /* alignment slack */ + GEMM_STAGES * (GEMM
 // error codes written to *err by the GEMM (distinct per wait site)
 constexpr int ERR_WAIT_EMPTY = 0x101, ERR_WAIT_FULL = 0x102, ERR_WAIT_TEMPTY = 0x103, ERR_WAIT_TFULL = 0x104;
 
+enum TriMode { TRI_NONE = 0, TRI_LOWER_STORE = 1, TRI_K = 2 };
+
 struct GemmArgs {
   int M, N, K;                 // problem size (rows of A, rows of B, contraction length)
+  int tri;                     // TriMode
+  int num_tiles;               // tiles visited (all, or the lower block triangle)
   int n_blocks_m, n_blocks_n;  // ceil(M/128), ceil(N/256)
   int group_n;                 // raster group width in N-blocks
   float* part;                 // SUMSQ / DOT: [n_blocks_n][M] per-row partial sums
@@ -59,7 +70,29 @@ struct GemmArgs {
   int* err;                    // device error word
 };
 
+// Number of tiles of the lower block triangle with n_blocks_m row tiles of
+// 128: row tile mb holds column tiles 0..(mb>>1).
+__host__ __device__ inline long long tri_lower_tiles(long long n_blocks_m) {
+  const long long q = n_blocks_m >> 1;
+  return (n_blocks_m & 1) ? (q + 1) * (q + 1) : q * (q + 1);
+}
+
 __device__ __forceinline__ void gemm_tile_coords(int t, const GemmArgs& a, int& mb, int& nb) {
+  if (a.tri == TRI_LOWER_STORE) {
+    // rows 2q and 2q+1 each hold q+1 tiles; tiles before row 2q: q(q+1)
+    int q = (int)((sqrtf(4.0f * (float)t + 1.0f) - 1.0f) * 0.5f);
+    while ((long long)(q + 1) * (q + 2) <= t) ++q;
+    while ((long long)q * (q + 1) > t) --q;
+    const int r = t - q * (q + 1);
+    if (r <= q) {
+      mb = 2 * q;
+      nb = r;
+    } else {
+      mb = 2 * q + 1;
+      nb = r - (q + 1);
+    }
+    return;
+  }
   const int gn = a.group_n;
   const int per_group = a.n_blocks_m * gn;
   const int g = t / per_group;
@@ -68,6 +101,13 @@ __device__ __forceinline__ void gemm_tile_coords(int t, const GemmArgs& a, int& 
   const int r = t - g * per_group;
   mb = r / width;
   nb = first + (r - mb * width);
+  if (a.tri == TRI_K) nb = a.n_blocks_n - 1 - nb;  // longest contractions first
+}
+
+__device__ __forceinline__ int gemm_num_kb(const GemmArgs& a, int nb) {
+  int k = a.K;
+  if (a.tri == TRI_K) k = min(k, (nb + 1) * GEMM_BN);
+  return (k + GEMM_BK - 1) / GEMM_BK;
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -120,8 +160,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = args.n_blocks_m * args.n_blocks_n;
-  const int num_kb = (args.K + GEMM_BK - 1) / GEMM_BK;
+  const int num_tiles = args.num_tiles;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -133,6 +172,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
         int mb, nb;
         gemm_tile_coords(t, args, mb, nb);
+        const int num_kb = gemm_num_kb(args, nb);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.err, ERR_WAIT_EMPTY)) {
             ok = false;
@@ -167,6 +207,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.err, ERR_WAIT_TEMPTY)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * GEMM_BN;
+        int mb, nb;
+        gemm_tile_coords(t, args, mb, nb);
+        const int num_kb = gemm_num_kb(args, nb);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, args.err, ERR_WAIT_FULL)) {
             ok = false;
@@ -240,6 +283,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
         } else {
           const int col = n0 + c * 32;
+          const float scale = (args.tri == TRI_LOWER_STORE && nb < (mb >> 1)) ? 2.0f : 1.0f;
           if (m < args.M) {
             __nv_bfloat16* crow = args.C + (long long)m * args.ldC + col;
 #pragma unroll
@@ -248,8 +292,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 uint32_t w[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                  __nv_bfloat162 p = __floats2bfloat162_rn(__uint_as_float(r[v * 8 + 2 * h]),
-                                                           __uint_as_float(r[v * 8 + 2 * h + 1]));
+                  __nv_bfloat162 p = __floats2bfloat162_rn(scale * __uint_as_float(r[v * 8 + 2 * h]),
+                                                           scale * __uint_as_float(r[v * 8 + 2 * h + 1]));
                   w[h] = *reinterpret_cast<uint32_t*>(&p);
                 }
                 *reinterpret_cast<uint4*>(crow + v * 8) = make_uint4(w[0], w[1], w[2], w[3]);
