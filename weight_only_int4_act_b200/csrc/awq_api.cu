@@ -18,7 +18,7 @@ using namespace awq;
 namespace {
 
 constexpr size_t kAlign = 1024;
-constexpr int kStatsTargetBlocks = 148 * 8;
+constexpr int kStatsTargetBlocks = 148 * 4;  // one wave at 4 resident blocks per SM
 constexpr int kGroupN = 8;
 
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
@@ -93,7 +93,7 @@ StatsLayout stats_layout(int64_t N, int64_t d_in) {
   StatsLayout L{};
   L.col_blocks = (int)cdiv(d_in, STATS_COLS);
   long long rpc = cdiv((long long)N * L.col_blocks, kStatsTargetBlocks);
-  rpc = cdiv(rpc < 32 ? 32 : rpc, 32) * 32;
+  rpc = cdiv(rpc < 64 ? 64 : rpc, 64) * 64;
   L.rows_per_chunk = (int)rpc;
   L.n_chunks = (int)cdiv(N, rpc);
   L.off_part = kAlign;  // [0, 1024): error word
@@ -226,9 +226,14 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
   return launch_status();
 }
 
-int elementwise_grid(long long threads_needed, int num_sms) {
+// Grid of a grid-stride kernel with 256-thread blocks: enough blocks for the
+// work, at most one wave of resident blocks.
+template <typename K>
+int elementwise_grid(K kernel, long long threads_needed, int num_sms) {
   long long blocks = cdiv(threads_needed, 256);
-  const long long cap = (long long)num_sms * 8;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
+  const long long cap = (long long)num_sms * per_sm;
   if (blocks > cap) blocks = cap;
   return (int)(blocks < 1 ? 1 : blocks);
 }
@@ -312,10 +317,22 @@ awq_status awq_step_fake_quant(const void* W, int64_t d_out, int64_t d_in, int64
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;
   const long long units = (long long)(L.d_out_pad / FQ_ROWS) * (d_in / 8);
-  fake_quant_delta<<<elementwise_grid(units, sms), 256, 0, as_stream(stream)>>>(
-      static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in, L.d_out_pad, at<float>(ws, L.off_s),
-      at<float>(ws, L.off_inv), cfg->n_alpha, cfg->bits, cfg->symmetric, cfg->group / 8,
-      at<__nv_bfloat16>(ws, L.off_dw));
+  auto launch = [&](auto kernel) {
+    const int grid = elementwise_grid(kernel, units, sms);
+    kernel<<<grid, 256, 0, as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in,
+                                                L.d_out_pad, at<float>(ws, L.off_s), at<float>(ws, L.off_inv),
+                                                cfg->n_alpha, cfg->bits, cfg->symmetric,
+                                                at<__nv_bfloat16>(ws, L.off_dw));
+  };
+  switch (cfg->group / 8) {
+    case 1: launch(fake_quant_delta<1>); break;
+    case 2: launch(fake_quant_delta<2>); break;
+    case 4: launch(fake_quant_delta<4>); break;
+    case 8: launch(fake_quant_delta<8>); break;
+    case 16: launch(fake_quant_delta<16>); break;
+    case 32: launch(fake_quant_delta<32>); break;
+    default: return AWQ_ERR_INVALID_ARG;
+  }
   return launch_status();
 }
 
@@ -416,10 +433,22 @@ awq_status awq_quantize_pack(const void* W, const float* s, int64_t d_out, int64
     return AWQ_ERR_INVALID_ARG;
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;
-  const long long units = (long long)d_out * (d_in / 8);
-  quantize_pack<<<elementwise_grid(units, sms), 256, 0, as_stream(stream)>>>(
-      static_cast<const __nv_bfloat16*>(W), s, (int)d_out, (int)d_in, cfg->bits, cfg->symmetric, cfg->group / 8,
-      qweight, static_cast<__half*>(scales), static_cast<__half*>(zeros));
+  const long long units = cdiv(d_out, PACK_ROWS) * (d_in / 8);
+  auto launch = [&](auto kernel) {
+    const int grid = elementwise_grid(kernel, units, sms);
+    kernel<<<grid, 256, 0, as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(W), s, (int)d_out, (int)d_in,
+                                                cfg->bits, cfg->symmetric, qweight, static_cast<__half*>(scales),
+                                                static_cast<__half*>(zeros));
+  };
+  switch (cfg->group / 8) {
+    case 1: launch(quantize_pack<1>); break;
+    case 2: launch(quantize_pack<2>); break;
+    case 4: launch(quantize_pack<4>); break;
+    case 8: launch(quantize_pack<8>); break;
+    case 16: launch(quantize_pack<16>); break;
+    case 32: launch(quantize_pack<32>); break;
+    default: return AWQ_ERR_INVALID_ARG;
+  }
   return launch_status();
 }
 

@@ -32,11 +32,12 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4 u, float (&f)[8]) {
 // a1: a[i] = (1/N) sum_t |X[t, i]|   ([P1] 激活感知 Omega_i, [P5] §1.2)
 // Block = 256 threads covering 256 columns (each lane 8 columns, 16-byte
 // loads; warps take interleaved rows) and `rows_per_chunk` rows. Each thread
-// sums 4 rows in fp32, then accumulates in fp64; the 8 warps are combined in a
+// sums 8 rows in fp32, then accumulates in fp64; the 8 warps are combined in a
 // fixed order and the chunk's fp64 column sums are written to `part`.
 // ---------------------------------------------------------------------------
 constexpr int STATS_THREADS = 256;
 constexpr int STATS_COLS = 256;
+constexpr int STATS_UNROLL = 8;  // rows summed in fp32 (and loads in flight) per thread and step
 
 __global__ void __launch_bounds__(STATS_THREADS) act_absmean_partial(const __nv_bfloat16* __restrict__ X, long long N,
                                                                      int d_in, int rows_per_chunk,
@@ -49,16 +50,16 @@ __global__ void __launch_bounds__(STATS_THREADS) act_absmean_partial(const __nv_
   double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (col < d_in) {
     const __nv_bfloat16* base = X + col;
-    for (long long r = r0 + warp; r < r1; r += 4 * 8) {
-      uint4 u[4];
+    for (long long r = r0 + warp; r < r1; r += STATS_UNROLL * 8) {
+      uint4 u[STATS_UNROLL];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < STATS_UNROLL; ++k) {
         const long long rr = r + 8 * k;
         u[k] = rr < r1 ? __ldcs(reinterpret_cast<const uint4*>(base + rr * d_in)) : make_uint4(0, 0, 0, 0);
       }
       float s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < STATS_UNROLL; ++k) {
         float f[8];
         unpack_bf16x8(u[k], f);
 #pragma unroll
@@ -144,10 +145,11 @@ __global__ void candidate_scales(const float* __restrict__ a, int d_in, AlphaGri
 // ---------------------------------------------------------------------------
 constexpr int FQ_ROWS = 4;
 
-__global__ void __launch_bounds__(256) fake_quant_delta(const __nv_bfloat16* __restrict__ W, int d_out, int d_in,
+template <int GL>
+__global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* __restrict__ W, int d_out, int d_in,
                                                         int d_out_pad, const float* __restrict__ s_all,
                                                         const float* __restrict__ inv_all, int n_alpha, int bits,
-                                                        int symmetric, int gl, __nv_bfloat16* __restrict__ dW) {
+                                                        int symmetric, __nv_bfloat16* __restrict__ dW) {
   const int chunks = d_in >> 3;
   const long long total = (long long)(d_out_pad / FQ_ROWS) * chunks;
   const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(256) fake_quant_delta(const __nv_bfloat16* __r
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[j] = w[r][j] * s[j];
         FqResult fr;
-        fq_group8(v, bits, sym, gl, fr);
+        fq_group8<GL>(v, bits, sym, fr);
         uint32_t out[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
@@ -316,46 +318,63 @@ __global__ void loss_argmin(const double* __restrict__ block_sums, int n_chunks,
 // uint32 (channel 8w+j in bits 4j..4j+3), fp16 step and zero per group.
 // ([P2] §2.1 INT4 with fp16 scale, §4.2 packed 4-bit storage; [P4] §三.)
 // ---------------------------------------------------------------------------
+// One thread = 8 consecutive channels of PACK_ROWS consecutive rows (the 8
+// scales are loaded once for all of them; PACK_ROWS independent 16-byte loads
+// of W are in flight per thread).
+constexpr int PACK_ROWS = 4;
+
+template <int GL>
 __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __restrict__ W, const float* __restrict__ s,
-                                                     int d_out, int d_in, int bits, int symmetric, int gl,
+                                                     int d_out, int d_in, int bits, int symmetric,
                                                      uint32_t* __restrict__ qweight, __half* __restrict__ scales,
                                                      __half* __restrict__ zeros) {
   const int chunks = d_in >> 3;
-  const long long total = (long long)d_out * chunks;
+  const int row_groups = (d_out + PACK_ROWS - 1) / PACK_ROWS;
+  const long long total = (long long)row_groups * chunks;
   const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int lane = threadIdx.x & 31;
   const bool sym = symmetric != 0;
-  const int groups = d_in / (gl * 8);
+  const int groups = d_in / (GL * 8);
   for (long long base = warp_global * 32; base < total; base += n_warps * 32) {
     const long long u = base + lane;
     const bool active = u < total;
-    const int row = active ? (int)(u / chunks) : 0;
-    const int chunk = active ? (int)(u - (long long)row * chunks) : 0;
+    const int rg = active ? (int)(u / chunks) : 0;
+    const int chunk = active ? (int)(u - (long long)rg * chunks) : 0;
     const int c0 = chunk * 8;
-    float v[8];
-    if (active) {
-      float w[8];
-      unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(W + (long long)row * d_in + c0)), w);
+    const int row0 = rg * PACK_ROWS;
+    uint4 wraw[PACK_ROWS];
+#pragma unroll
+    for (int r = 0; r < PACK_ROWS; ++r)
+      wraw[r] = (active && row0 + r < d_out)
+                    ? __ldcs(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0))
+                    : make_uint4(0, 0, 0, 0);
+    float sc[8];
+    {
       const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + c0));
       const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + c0 + 4));
-      v[0] = w[0] * s0.x; v[1] = w[1] * s0.y; v[2] = w[2] * s0.z; v[3] = w[3] * s0.w;
-      v[4] = w[4] * s1.x; v[5] = w[5] * s1.y; v[6] = w[6] * s1.z; v[7] = w[7] * s1.w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = 0.f;
+      sc[0] = s0.x; sc[1] = s0.y; sc[2] = s0.z; sc[3] = s0.w; sc[4] = s1.x; sc[5] = s1.y; sc[6] = s1.z; sc[7] = s1.w;
     }
-    FqResult fr;
-    fq_group8(v, bits, sym, gl, fr);
-    if (active) {
-      uint32_t word = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) word |= (fq_code(fr, j, sym) & 0xFu) << (4 * j);
-      qweight[(long long)row * chunks + chunk] = word;
-      if ((chunk & (gl - 1)) == 0) {
-        const long long gidx = (long long)row * groups + chunk / gl;
-        scales[gidx] = __float2half_rn(fr.delta);
-        zeros[gidx] = __float2half_rn(fr.zero);
+    for (int r = 0; r < PACK_ROWS; ++r) {
+      const bool real = active && row0 + r < d_out;
+      float v[8];
+      unpack_bf16x8(wraw[r], v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] *= sc[j];
+      FqResult fr;
+      fq_group8<GL>(v, bits, sym, fr);
+      if (real) {
+        const int row = row0 + r;
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) word |= (fq_code(fr, j, sym) & 0xFu) << (4 * j);
+        __stcs(qweight + (long long)row * chunks + chunk, word);
+        if ((chunk & (GL - 1)) == 0) {
+          const long long gidx = (long long)row * groups + chunk / GL;
+          scales[gidx] = __float2half_rn(fr.delta);
+          zeros[gidx] = __float2half_rn(fr.zero);
+        }
       }
     }
   }

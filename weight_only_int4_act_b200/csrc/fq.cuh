@@ -13,8 +13,9 @@
 //   asymmetric: Delta = max(max v - min v, eps) / (2^b - 1)
 //               z = clamp(rne(-min v / Delta), 0, 2^b - 1)
 //               q = clamp(rne(v / Delta) + z, 0, 2^b - 1),   v_hat = (q - z) Delta
-// Arithmetic is fp32; Delta is the range times the fp32 constant 1/levels and
-// v / Delta is taken as v * (1 / Delta) (correctly rounded reciprocal).
+// Arithmetic is fp32; Delta is the range times the fp32 constant 1/levels,
+// 1/Delta is the correctly rounded reciprocal, and rne(v / Delta) is rounded
+// from the exact product v * (1/Delta). GL = g/8 lanes form one group.
 #pragma once
 #include <cuda_runtime.h>
 
@@ -33,19 +34,44 @@ struct FqResult {
   float q[8];   // asymmetric: stored code in [0, 2^b-1]; symmetric: signed q
 };
 
-__device__ __forceinline__ void fq_group8(const float (&v)[8], int bits, bool symmetric, int gl, FqResult& r) {
+// Round-to-nearest-even to an integer by the fp32 "magic number" method: for
+// |x| < 2^22, x + 1.5*2^23 has no fraction bits left, so the addition itself
+// rounds x to the nearest integer (ties to even), which subtracting the
+// constant recovers exactly. Here the addition is fused with the product
+// v * inv (one rounding of the exact product), which keeps the work on the
+// full-rate FMA pipe.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+template <int GL>
+__device__ __forceinline__ float group_max(float x) {
+#pragma unroll
+  for (int off = 1; off < GL; off <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+  return x;
+}
+template <int GL>
+__device__ __forceinline__ float group_min(float x) {
+#pragma unroll
+  for (int off = 1; off < GL; off <<= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, off));
+  return x;
+}
+
+template <int GL>
+__device__ __forceinline__ void fq_group8(const float (&v)[8], int bits, bool symmetric, FqResult& r) {
   if (symmetric) {
     float amax = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    for (int off = 1; off < gl; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    amax = group_max<GL>(amax);
     const float qmax = (float)((1 << (bits - 1)) - 1);
     const float qmin = -(float)(1 << (bits - 1));
     r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
     const float inv = __frcp_rn(r.delta);
     r.zero = -qmin;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) r.q[j] = fminf(fmaxf(rintf(v[j] * inv), qmin), qmax);
+    for (int j = 0; j < 8; ++j) {
+      const float t = __fmaf_rn(v[j], inv, kRoundMagic) - kRoundMagic;  // rne(v / Delta)
+      r.q[j] = fminf(fmaxf(t, qmin), qmax);
+    }
   } else {
     float mx = v[0], mn = v[0];
 #pragma unroll
@@ -53,16 +79,18 @@ __device__ __forceinline__ void fq_group8(const float (&v)[8], int bits, bool sy
       mx = fmaxf(mx, v[j]);
       mn = fminf(mn, v[j]);
     }
-    for (int off = 1; off < gl; off <<= 1) {
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-    }
+    mx = group_max<GL>(mx);
+    mn = group_min<GL>(mn);
     const float levels = (float)((1 << bits) - 1);
     r.delta = fmaxf(mx - mn, kEpsDelta) * inv_levels(bits);
     const float inv = __frcp_rn(r.delta);
-    r.zero = fminf(fmaxf(rintf(-mn * inv), 0.f), levels);
+    r.zero = fminf(fmaxf(__fmaf_rn(-mn, inv, kRoundMagic) - kRoundMagic, 0.f), levels);  // rne(-min / Delta)
+    const float off = kRoundMagic - r.zero;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) r.q[j] = fminf(fmaxf(rintf(v[j] * inv) + r.zero, 0.f), levels);
+    for (int j = 0; j < 8; ++j) {
+      const float t = __fmaf_rn(v[j], inv, kRoundMagic) - off;  // rne(v / Delta) + z
+      r.q[j] = fminf(fmaxf(t, 0.f), levels);
+    }
   }
 }
 
