@@ -18,6 +18,8 @@ using namespace awq;
 namespace {
 
 constexpr size_t kAlign = 1024;
+// search workspace header: [0, 4) device error word, [256, 260) tile counter of the GEMMs
+constexpr size_t kTileCounterOffset = 256;
 constexpr int kStatsTargetBlocks = 148 * 4;  // one wave at 4 resident blocks per SM
 constexpr int kGroupN = 8;
 
@@ -142,7 +144,7 @@ SearchLayout search_layout(int64_t d_out, int64_t d_in, int64_t N, const awq_qcf
   L.n_blocks_n = (int)cdiv(L.form == AWQ_FORM_DIRECT ? N : d_in, GEMM_BN);
   L.n_red_chunks = (int)cdiv(d_out, REDUCE_THREADS);
   L.ld_t = cdiv(N, 64) * 64;
-  size_t off = kAlign;  // [0, 1024): error word
+  size_t off = kAlign;  // [0, 1024): error word and tile counter
   L.off_s = off;      off += align_up((size_t)L.n_alpha * d_in * sizeof(float));
   L.off_inv = off;    off += align_up((size_t)L.n_alpha * d_in * sizeof(float));
   L.off_dw = off;     off += align_up((size_t)L.M * d_in * 2);
@@ -221,6 +223,7 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
   if (cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) !=
       cudaSuccess)
     return AWQ_ERR_CUDA;
+  if (cudaMemsetAsync(args.tile_counter, 0, sizeof(int), st) != cudaSuccess) return AWQ_ERR_CUDA;
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
   gemm_bf16_tcgen05<MODE><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(ta, tb, args);
   return launch_status();
@@ -354,6 +357,7 @@ awq_status awq_step_gram(const void* X, int64_t d_out, int64_t d_in, int64_t N, 
   ga.C = at<__nv_bfloat16>(ws, L.off_g);
   ga.ldC = d_in;
   ga.err = at<int>(ws, 0);
+  ga.tile_counter = at<int>(ws, kTileCounterOffset);
   const void* xt = at<void>(ws, L.off_xt);
   return run_gemm<EPI_STORE>(xt, d_in, L.ld_t, xt, d_in, L.ld_t, L.ld_t, ga, TRI_LOWER_STORE, sms, s);
 }
@@ -368,6 +372,7 @@ awq_status awq_step_contract(const void* X, int64_t d_out, int64_t d_in, int64_t
   GemmArgs ga{};
   ga.part = at<float>(ws, L.off_part);
   ga.err = at<int>(ws, 0);
+  ga.tile_counter = at<int>(ws, kTileCounterOffset);
   const void* dw = at<void>(ws, L.off_dw);
   if (L.form == AWQ_FORM_DIRECT) {
     if (!X || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;

@@ -164,11 +164,9 @@ __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* 
     const int c0 = active ? (int)(u - (long long)quad * chunks) * 8 : 0;
     const int row0 = quad * FQ_ROWS;
     float w[FQ_ROWS][8];
-    bool real[FQ_ROWS];
 #pragma unroll
     for (int r = 0; r < FQ_ROWS; ++r) {
-      real[r] = active && row0 + r < d_out;
-      if (real[r]) {
+      if (active && row0 + r < d_out) {
         unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0)), w[r]);
       } else {
 #pragma unroll
@@ -193,8 +191,9 @@ __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* 
         uint32_t out[4];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          const float d0 = real[r] ? fq_dequant(fr, 2 * h, sym) * is[2 * h] - w[r][2 * h] : 0.f;
-          const float d1 = real[r] ? fq_dequant(fr, 2 * h + 1, sym) * is[2 * h + 1] - w[r][2 * h + 1] : 0.f;
+          // rows past d_out hold w = 0, whose group dequantises to exactly 0
+          const float d0 = fq_dequant(fr, 2 * h) * is[2 * h] - w[r][2 * h];
+          const float d1 = fq_dequant(fr, 2 * h + 1) * is[2 * h + 1] - w[r][2 * h + 1];
           __nv_bfloat162 p = __floats2bfloat162_rn(d0, d1);
           out[h] = *reinterpret_cast<uint32_t*>(&p);
         }
@@ -368,7 +367,7 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
         const int row = row0 + r;
         uint32_t word = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) word |= (fq_code(fr, j, sym) & 0xFu) << (4 * j);
+        for (int j = 0; j < 8; ++j) word |= (fq_code(fr, j) & 0xFu) << (4 * j);
         __stcs(qweight + (long long)row * chunks + chunk, word);
         if ((chunk & (GL - 1)) == 0) {
           const long long gidx = (long long)row * groups + chunk / GL;

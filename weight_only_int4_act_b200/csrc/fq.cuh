@@ -28,10 +28,13 @@ __device__ __forceinline__ float inv_levels(int b) {
   return b == 4 ? (1.0f / 15.0f) : b == 3 ? (1.0f / 7.0f) : b == 2 ? (1.0f / 3.0f) : 1.0f;
 }
 
+// Codes are kept in "magic" form c = code_value + 1.5*2^23 (see below):
+// the stored code is c - lo and the dequantised value is (c - 1.5*2^23) * delta.
 struct FqResult {
   float delta;  // quantisation step of the group
   float zero;   // asymmetric: z; symmetric: 2^(b-1) (the stored zero)
-  float q[8];   // asymmetric: stored code in [0, 2^b-1]; symmetric: signed q
+  float lo;     // c of stored code 0
+  float c[8];   // clamped magic-form codes
 };
 
 // Round-to-nearest-even to an integer by the fp32 "magic number" method: for
@@ -55,53 +58,58 @@ __device__ __forceinline__ float group_min(float x) {
   return x;
 }
 
+// Three-input max / min (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float max8(const float (&v)[8]) {
+  return fmaxf(max3f(max3f(max3f(v[0], v[1], v[2]), v[3], v[4]), v[5], v[6]), v[7]);
+}
+__device__ __forceinline__ float min8(const float (&v)[8]) {
+  return fminf(min3f(min3f(min3f(v[0], v[1], v[2]), v[3], v[4]), v[5], v[6]), v[7]);
+}
+
 template <int GL>
 __device__ __forceinline__ void fq_group8(const float (&v)[8], int bits, bool symmetric, FqResult& r) {
   if (symmetric) {
-    float amax = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    float amax = fmaxf(max8(v), -min8(v));
     amax = group_max<GL>(amax);
     const float qmax = (float)((1 << (bits - 1)) - 1);
     const float qmin = -(float)(1 << (bits - 1));
     r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
     const float inv = __frcp_rn(r.delta);
     r.zero = -qmin;
+    r.lo = kRoundMagic + qmin;
+    const float hi = kRoundMagic + qmax;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float t = __fmaf_rn(v[j], inv, kRoundMagic) - kRoundMagic;  // rne(v / Delta)
-      r.q[j] = fminf(fmaxf(t, qmin), qmax);
-    }
+    for (int j = 0; j < 8; ++j)  // clamp(rne(v / Delta), qmin, qmax) + magic
+      r.c[j] = fminf(fmaxf(__fmaf_rn(v[j], inv, kRoundMagic), r.lo), hi);
   } else {
-    float mx = v[0], mn = v[0];
-#pragma unroll
-    for (int j = 1; j < 8; ++j) {
-      mx = fmaxf(mx, v[j]);
-      mn = fminf(mn, v[j]);
-    }
-    mx = group_max<GL>(mx);
-    mn = group_min<GL>(mn);
+    const float mx = group_max<GL>(max8(v));
+    const float mn = group_min<GL>(min8(v));
     const float levels = (float)((1 << bits) - 1);
     r.delta = fmaxf(mx - mn, kEpsDelta) * inv_levels(bits);
     const float inv = __frcp_rn(r.delta);
     r.zero = fminf(fmaxf(__fmaf_rn(-mn, inv, kRoundMagic) - kRoundMagic, 0.f), levels);  // rne(-min / Delta)
-    const float off = kRoundMagic - r.zero;
+    r.lo = kRoundMagic - r.zero;
+    const float hi = r.lo + levels;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float t = __fmaf_rn(v[j], inv, kRoundMagic) - off;  // rne(v / Delta) + z
-      r.q[j] = fminf(fmaxf(t, 0.f), levels);
-    }
+    for (int j = 0; j < 8; ++j)  // clamp(rne(v / Delta) + z, 0, 2^b - 1) - z + magic
+      r.c[j] = fminf(fmaxf(__fmaf_rn(v[j], inv, kRoundMagic), r.lo), hi);
   }
 }
 
-// Dequantised value v_hat of element j.
-__device__ __forceinline__ float fq_dequant(const FqResult& r, int j, bool symmetric) {
-  return symmetric ? r.q[j] * r.delta : (r.q[j] - r.zero) * r.delta;
-}
+// Dequantised value v_hat of element j ((q - z) Delta, or q Delta when symmetric).
+__device__ __forceinline__ float fq_dequant(const FqResult& r, int j) { return (r.c[j] - kRoundMagic) * r.delta; }
 
 // Stored (unsigned) code of element j.
-__device__ __forceinline__ unsigned fq_code(const FqResult& r, int j, bool symmetric) {
-  return (unsigned)(symmetric ? r.q[j] + r.zero : r.q[j]);
-}
+__device__ __forceinline__ unsigned fq_code(const FqResult& r, int j) { return (unsigned)(r.c[j] - r.lo); }
 
 }  // namespace awq

@@ -7,7 +7,8 @@
 // (128-byte swizzle, no multicast).
 //
 // Warp roles (192 threads):
-//   warp 0      one thread issues the TMA loads of A and B;
+//   warp 0      one thread takes tile indices from the global counter, publishes
+//               them to the other warps and issues the TMA loads of A and B;
 //   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
 //               one thread issues tcgen05.mma, committing each stage back to
 //               the loader and each finished tile to the epilogue;
@@ -19,8 +20,11 @@
 // The accumulator is released before the partials are written, so the next
 // tile's MMAs overlap this tile's epilogue.
 //
-// Tiles are visited in groups of `group_n` N-blocks (M-major inside a group)
-// so that the CTAs running at one time share A panels and a B slice in L2.
+// Tiles are handed out dynamically in the order of a tile index t (an atomic
+// counter; each CTA takes the next index when it starts a tile), so CTAs that
+// draw short tiles simply take more of them. Indices walk groups of `group_n`
+// N-blocks (M-major inside a group) so that the CTAs running at one time share
+// A panels and a B slice in L2.
 //
 // Block-triangular modes (the Gram form uses the symmetry of G = X^T X, with
 // 256-wide channel blocks J): TRI_LOWER_STORE computes only the tiles of G
@@ -52,7 +56,9 @@ constexpr int GEMM_TMEM_COLS = 512;
 constexpr int GEMM_SMEM_BYTES = 1024 /* alignment slack */ + GEMM_STAGES * (GEMM_A_STAGE + GEMM_B_STAGE) + 256;
 
 // error codes written to *err by the GEMM (distinct per wait site)
-constexpr int ERR_WAIT_EMPTY = 0x101, ERR_WAIT_FULL = 0x102, ERR_WAIT_TEMPTY = 0x103, ERR_WAIT_TFULL = 0x104;
+constexpr int ERR_WAIT_EMPTY = 0x101, ERR_WAIT_FULL = 0x102, ERR_WAIT_TEMPTY = 0x103, ERR_WAIT_TFULL = 0x104,
+              ERR_WAIT_SCHED = 0x105;
+constexpr int GEMM_SCHED_SLOTS = 4;  // tile indices published ahead of the MMA and epilogue warps
 
 enum TriMode { TRI_NONE = 0, TRI_LOWER_STORE = 1, TRI_K = 2 };
 
@@ -68,6 +74,7 @@ struct GemmArgs {
   __nv_bfloat16* C;            // STORE: C[M, ldC]
   long long ldC;
   int* err;                    // device error word
+  int* tile_counter;           // dynamic tile counter, zero at launch
 };
 
 // Number of tiles of the lower block triangle with n_blocks_m row tiles of
@@ -122,8 +129,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + GEMM_STAGES * GEMM_A_STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + GEMM_STAGES * GEMM_B_STAGE);
-  // bars: full[S], empty[S], tfull[2], tempty[2], drain
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * GEMM_STAGES + 5);
+  // bars: full[S], empty[S], tfull[2], tempty[2], drain, sched_full[R], sched_empty[R]
+  constexpr int NB = 2 * GEMM_STAGES + 5 + 2 * GEMM_SCHED_SLOTS;
+  volatile int* tile_ring = reinterpret_cast<volatile int*>(bars + NB);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NB) + GEMM_SCHED_SLOTS;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -133,6 +142,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   auto tfull_bar = [&](int a) { return smem_u32(bars + 2 * GEMM_STAGES + a); };
   auto tempty_bar = [&](int a) { return smem_u32(bars + 2 * GEMM_STAGES + 2 + a); };
   const uint32_t drain_bar = smem_u32(bars + 2 * GEMM_STAGES + 4);
+  auto sfull_bar = [&](int r) { return smem_u32(bars + 2 * GEMM_STAGES + 5 + r); };
+  auto sempty_bar = [&](int r) { return smem_u32(bars + 2 * GEMM_STAGES + 5 + GEMM_SCHED_SLOTS + r); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < GEMM_STAGES; ++s) {
@@ -144,6 +155,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(tempty_bar(a), 4);
     }
     mbar_init(drain_bar, 1);
+    for (int r = 0; r < GEMM_SCHED_SLOTS; ++r) {
+      mbar_init(sfull_bar(r), 1);
+      mbar_init(sempty_bar(r), 5);  // the MMA thread and one lane of each epilogue warp
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -164,12 +179,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer
+      // ---------------- tile scheduler + TMA producer
+      // Tiles are handed out dynamically (a global counter, zeroed before the
+      // launch) and published to the MMA and epilogue warps through a ring of
+      // tile indices; -1 ends the sequence.
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, last_parity = 0;  // bit s: stage s has been loaded; parity of its last load
+      int slot = 0;
+      uint32_t sphase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      while (ok) {
+        if (!mbar_wait(sempty_bar(slot), sphase ^ 1u, abort_flag, args.err, ERR_WAIT_SCHED)) break;
+        int t = atomicAdd(args.tile_counter, 1);
+        if (t >= num_tiles) t = -1;
+        tile_ring[slot] = t;
+        mbar_arrive(sfull_bar(slot));
+        if (++slot == GEMM_SCHED_SLOTS) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+        if (t < 0) break;
         int mb, nb;
         gemm_tile_coords(t, args, mb, nb);
         const int num_kb = gemm_num_kb(args, nb);
@@ -199,9 +229,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, GEMM_BN);
       int stage = 0;
       uint32_t phase = 0;
+      int slot = 0;
+      uint32_t sphase = 0;
       bool ok = true;
-      int local = 0;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x, ++local) {
+      for (int local = 0; ok; ++local) {
+        if (!mbar_wait(sfull_bar(slot), sphase, abort_flag, args.err, ERR_WAIT_SCHED)) break;
+        const int t = tile_ring[slot];
+        mbar_arrive(sempty_bar(slot));
+        if (++slot == GEMM_SCHED_SLOTS) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+        if (t < 0) break;
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.err, ERR_WAIT_TEMPTY)) break;
@@ -239,13 +278,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ---------------- epilogue (warps 2..5)
     const int quad = warp & 3;
     const int row_in_tile = quad * 32 + lane;
-    int local = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+    int slot = 0;
+    uint32_t sphase = 0;
+    for (int local = 0;; ++local) {
+      // warp-uniform decisions: the tcgen05.ld below is .sync.aligned
+      const bool have = mbar_wait(sfull_bar(slot), sphase, abort_flag, args.err, ERR_WAIT_SCHED);
+      if (!__all_sync(0xffffffffu, have)) break;
+      const int t = tile_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sempty_bar(slot));
+      if (++slot == GEMM_SCHED_SLOTS) {
+        slot = 0;
+        sphase ^= 1u;
+      }
+      if (t < 0) break;
       int mb, nb;
       gemm_tile_coords(t, args, mb, nb);
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      // warp-uniform decision: the tcgen05.ld below is .sync.aligned
       const bool ready = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, args.err, ERR_WAIT_TFULL);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
