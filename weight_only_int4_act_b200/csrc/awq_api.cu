@@ -319,21 +319,22 @@ awq_status awq_step_fake_quant(const void* W, int64_t d_out, int64_t d_in, int64
   if (!W || !aligned(W, 16)) return AWQ_ERR_INVALID_ARG;
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;
-  const long long units = (long long)(L.d_out_pad / FQ_ROWS) * (d_in / 8);
-  auto launch = [&](auto kernel) {
+  auto launch = [&](auto kernel, int cpt) {
+    const long long units = (long long)(L.d_out_pad / FQ_ROWS) * (d_in / cpt);
     const int grid = elementwise_grid(kernel, units, sms);
     kernel<<<grid, 256, 0, as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in,
                                                 L.d_out_pad, at<float>(ws, L.off_s), at<float>(ws, L.off_inv),
                                                 cfg->n_alpha, cfg->bits, cfg->symmetric,
                                                 at<__nv_bfloat16>(ws, L.off_dw));
   };
-  switch (cfg->group / 8) {
-    case 1: launch(fake_quant_delta<1>); break;
-    case 2: launch(fake_quant_delta<2>); break;
-    case 4: launch(fake_quant_delta<4>); break;
-    case 8: launch(fake_quant_delta<8>); break;
-    case 16: launch(fake_quant_delta<16>); break;
-    case 32: launch(fake_quant_delta<32>); break;
+  constexpr int C = FQ_CPT;
+  switch (cfg->group) {
+    case 8: launch(fake_quant_delta<8, FQ_ROWS, 1>, 8); break;
+    case 16: launch(fake_quant_delta<(C < 16 ? C : 16), FQ_ROWS, 16 / (C < 16 ? C : 16)>, (C < 16 ? C : 16)); break;
+    case 32: launch(fake_quant_delta<(C < 32 ? C : 32), FQ_ROWS, 32 / (C < 32 ? C : 32)>, (C < 32 ? C : 32)); break;
+    case 64: launch(fake_quant_delta<C, FQ_ROWS, 64 / C>, C); break;
+    case 128: launch(fake_quant_delta<C, FQ_ROWS, 128 / C>, C); break;
+    case 256: launch(fake_quant_delta<C, FQ_ROWS, 256 / C>, C); break;
     default: return AWQ_ERR_INVALID_ARG;
   }
   return launch_status();
@@ -438,20 +439,21 @@ awq_status awq_quantize_pack(const void* W, const float* s, int64_t d_out, int64
     return AWQ_ERR_INVALID_ARG;
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;
-  const long long units = cdiv(d_out, PACK_ROWS) * (d_in / 8);
-  auto launch = [&](auto kernel) {
+  auto launch = [&](auto kernel, int cpt) {
+    const long long units = cdiv(d_out, PACK_ROWS) * (d_in / cpt);
     const int grid = elementwise_grid(kernel, units, sms);
     kernel<<<grid, 256, 0, as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(W), s, (int)d_out, (int)d_in,
                                                 cfg->bits, cfg->symmetric, qweight, static_cast<__half*>(scales),
                                                 static_cast<__half*>(zeros));
   };
-  switch (cfg->group / 8) {
-    case 1: launch(quantize_pack<1>); break;
-    case 2: launch(quantize_pack<2>); break;
-    case 4: launch(quantize_pack<4>); break;
-    case 8: launch(quantize_pack<8>); break;
-    case 16: launch(quantize_pack<16>); break;
-    case 32: launch(quantize_pack<32>); break;
+  constexpr int C = FQ_CPT;
+  switch (cfg->group) {
+    case 8: launch(quantize_pack<8, 1>, 8); break;
+    case 16: launch(quantize_pack<(C < 16 ? C : 16), 16 / (C < 16 ? C : 16)>, (C < 16 ? C : 16)); break;
+    case 32: launch(quantize_pack<(C < 32 ? C : 32), 32 / (C < 32 ? C : 32)>, (C < 32 ? C : 32)); break;
+    case 64: launch(quantize_pack<C, 64 / C>, C); break;
+    case 128: launch(quantize_pack<C, 128 / C>, C); break;
+    case 256: launch(quantize_pack<C, 256 / C>, C); break;
     default: return AWQ_ERR_INVALID_ARG;
   }
   return launch_status();

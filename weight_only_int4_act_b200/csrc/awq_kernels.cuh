@@ -139,19 +139,39 @@ __global__ void candidate_scales(const float* __restrict__ a, int d_in, AlphaGri
 // ---------------------------------------------------------------------------
 // a3: dW[k][r][:] = Q(W_r S_k) S_k^-1 - W_r as bf16, for every alpha k.
 // ([P1] 缩放保护 W~ = sW, W^ = Q(W~)/s; [P5] §2.2 Q(WS)S^-1.)
-// One thread = 8 consecutive channels of FQ_ROWS consecutive rows: W is read
-// once and reused for every alpha, and each alpha's 8 scales are loaded once
-// for the FQ_ROWS rows. Rows d_out..d_out_pad-1 of each slice are zeros.
+// One thread = CPT consecutive channels of ROWS consecutive rows: W is read
+// once and reused for every alpha, and each alpha's scales are loaded once for
+// the ROWS rows. Rows d_out..d_out_pad-1 of each slice come out as zeros (their
+// w = 0 dequantises to exactly 0).
 // ---------------------------------------------------------------------------
-constexpr int FQ_ROWS = 4;
+#ifndef AWQ_FQ_ROWS
+#define AWQ_FQ_ROWS 4
+#endif
+#ifndef AWQ_FQ_CPT
+#define AWQ_FQ_CPT 16
+#endif
+constexpr int FQ_ROWS = AWQ_FQ_ROWS;
+constexpr int FQ_CPT = AWQ_FQ_CPT;  // channels per thread (at most; never more than g)
 
-template <int GL>
+template <int CPT>
+__device__ __forceinline__ void load_f32(const float* __restrict__ p, float (&f)[CPT]) {
+#pragma unroll
+  for (int q = 0; q < CPT / 4; ++q) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(p) + q);
+    f[4 * q] = x.x;
+    f[4 * q + 1] = x.y;
+    f[4 * q + 2] = x.z;
+    f[4 * q + 3] = x.w;
+  }
+}
+
+template <int CPT, int ROWS, int GL>
 __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* __restrict__ W, int d_out, int d_in,
-                                                        int d_out_pad, const float* __restrict__ s_all,
-                                                        const float* __restrict__ inv_all, int n_alpha, int bits,
-                                                        int symmetric, __nv_bfloat16* __restrict__ dW) {
-  const int chunks = d_in >> 3;
-  const long long total = (long long)(d_out_pad / FQ_ROWS) * chunks;
+                                                           int d_out_pad, const float* __restrict__ s_all,
+                                                           const float* __restrict__ inv_all, int n_alpha, int bits,
+                                                           int symmetric, __nv_bfloat16* __restrict__ dW) {
+  const int chunks = d_in / CPT;
+  const long long total = (long long)(d_out_pad / ROWS) * chunks;
   const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -160,46 +180,49 @@ __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* 
   for (long long base = warp_global * 32; base < total; base += n_warps * 32) {
     const long long u = base + lane;
     const bool active = u < total;
-    const int quad = active ? (int)(u / chunks) : 0;
-    const int c0 = active ? (int)(u - (long long)quad * chunks) * 8 : 0;
-    const int row0 = quad * FQ_ROWS;
-    float w[FQ_ROWS][8];
+    const int rq = active ? (int)(u / chunks) : 0;
+    const int c0 = active ? (int)(u - (long long)rq * chunks) * CPT : 0;
+    const int row0 = rq * ROWS;
+    float w[ROWS][CPT];
 #pragma unroll
-    for (int r = 0; r < FQ_ROWS; ++r) {
-      if (active && row0 + r < d_out) {
-        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0)), w[r]);
-      } else {
+    for (int r = 0; r < ROWS; ++r) {
+      const bool real = active && row0 + r < d_out;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) w[r][j] = 0.f;
+      for (int q = 0; q < CPT / 8; ++q) {
+        float f[8];
+        unpack_bf16x8(real ? __ldg(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0) + q)
+                           : make_uint4(0, 0, 0, 0),
+                      f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[r][8 * q + j] = f[j];
       }
     }
     __nv_bfloat16* out_base = dW + (long long)row0 * d_in + c0;
     for (int k = 0; k < n_alpha; ++k) {
-      float s[8], is[8];
-      const float4* sp = reinterpret_cast<const float4*>(s_all + (long long)k * d_in + c0);
-      const float4* ip = reinterpret_cast<const float4*>(inv_all + (long long)k * d_in + c0);
-      const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1), i0 = __ldg(ip), i1 = __ldg(ip + 1);
-      s[0] = s0.x; s[1] = s0.y; s[2] = s0.z; s[3] = s0.w; s[4] = s1.x; s[5] = s1.y; s[6] = s1.z; s[7] = s1.w;
-      is[0] = i0.x; is[1] = i0.y; is[2] = i0.z; is[3] = i0.w; is[4] = i1.x; is[5] = i1.y; is[6] = i1.z; is[7] = i1.w;
+      float s[CPT], is[CPT];
+      load_f32<CPT>(s_all + (long long)k * d_in + c0, s);
+      load_f32<CPT>(inv_all + (long long)k * d_in + c0, is);
 #pragma unroll
-      for (int r = 0; r < FQ_ROWS; ++r) {
-        float v[8];
+      for (int r = 0; r < ROWS; ++r) {
+        float v[CPT];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = w[r][j] * s[j];
-        FqResult fr;
-        fq_group8<GL>(v, bits, sym, fr);
-        uint32_t out[4];
+        for (int j = 0; j < CPT; ++j) v[j] = w[r][j] * s[j];
+        FqGroup<CPT> fr;
+        fq_group<CPT, GL>(v, bits, sym, fr);
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          // rows past d_out hold w = 0, whose group dequantises to exactly 0
-          const float d0 = fq_dequant(fr, 2 * h) * is[2 * h] - w[r][2 * h];
-          const float d1 = fq_dequant(fr, 2 * h + 1) * is[2 * h + 1] - w[r][2 * h + 1];
-          __nv_bfloat162 p = __floats2bfloat162_rn(d0, d1);
-          out[h] = *reinterpret_cast<uint32_t*>(&p);
+        for (int q = 0; q < CPT / 8; ++q) {
+          uint32_t out[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int j = 8 * q + 2 * h;
+            __nv_bfloat162 p = __floats2bfloat162_rn(fq_dequant(fr, j) * is[j] - w[r][j],
+                                                     fq_dequant(fr, j + 1) * is[j + 1] - w[r][j + 1]);
+            out[h] = *reinterpret_cast<uint32_t*>(&p);
+          }
+          if (active)
+            __stcs(reinterpret_cast<uint4*>(out_base + k * slice + (long long)r * d_in) + q,
+                   make_uint4(out[0], out[1], out[2], out[3]));
         }
-        if (active)
-          __stcs(reinterpret_cast<uint4*>(out_base + k * slice + (long long)r * d_in),
-                 make_uint4(out[0], out[1], out[2], out[3]));
       }
     }
   }
@@ -317,58 +340,64 @@ __global__ void loss_argmin(const double* __restrict__ block_sums, int n_chunks,
 // uint32 (channel 8w+j in bits 4j..4j+3), fp16 step and zero per group.
 // ([P2] §2.1 INT4 with fp16 scale, §4.2 packed 4-bit storage; [P4] §三.)
 // ---------------------------------------------------------------------------
-// One thread = 8 consecutive channels of PACK_ROWS consecutive rows (the 8
-// scales are loaded once for all of them; PACK_ROWS independent 16-byte loads
-// of W are in flight per thread).
+// One thread = CPT consecutive channels of PACK_ROWS consecutive rows (the
+// scales are loaded once for all of them; PACK_ROWS independent loads of W are
+// in flight per thread). Each row yields CPT/8 consecutive words.
 constexpr int PACK_ROWS = 4;
 
-template <int GL>
+template <int CPT, int GL>
 __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __restrict__ W, const float* __restrict__ s,
                                                      int d_out, int d_in, int bits, int symmetric,
                                                      uint32_t* __restrict__ qweight, __half* __restrict__ scales,
                                                      __half* __restrict__ zeros) {
-  const int chunks = d_in >> 3;
+  const int chunks = d_in / CPT;
   const int row_groups = (d_out + PACK_ROWS - 1) / PACK_ROWS;
   const long long total = (long long)row_groups * chunks;
   const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int lane = threadIdx.x & 31;
   const bool sym = symmetric != 0;
-  const int groups = d_in / (GL * 8);
+  const int groups = d_in / (GL * CPT);
+  const int words = d_in / 8;
   for (long long base = warp_global * 32; base < total; base += n_warps * 32) {
     const long long u = base + lane;
     const bool active = u < total;
     const int rg = active ? (int)(u / chunks) : 0;
     const int chunk = active ? (int)(u - (long long)rg * chunks) : 0;
-    const int c0 = chunk * 8;
+    const int c0 = chunk * CPT;
     const int row0 = rg * PACK_ROWS;
-    uint4 wraw[PACK_ROWS];
+    uint4 wraw[PACK_ROWS][CPT / 8];
 #pragma unroll
     for (int r = 0; r < PACK_ROWS; ++r)
-      wraw[r] = (active && row0 + r < d_out)
-                    ? __ldcs(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0))
-                    : make_uint4(0, 0, 0, 0);
-    float sc[8];
-    {
-      const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + c0));
-      const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + c0 + 4));
-      sc[0] = s0.x; sc[1] = s0.y; sc[2] = s0.z; sc[3] = s0.w; sc[4] = s1.x; sc[5] = s1.y; sc[6] = s1.z; sc[7] = s1.w;
-    }
+#pragma unroll
+      for (int q = 0; q < CPT / 8; ++q)
+        wraw[r][q] = (active && row0 + r < d_out)
+                         ? __ldcs(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0) + q)
+                         : make_uint4(0, 0, 0, 0);
+    float sc[CPT];
+    load_f32<CPT>(s + c0, sc);
 #pragma unroll
     for (int r = 0; r < PACK_ROWS; ++r) {
-      const bool real = active && row0 + r < d_out;
-      float v[8];
-      unpack_bf16x8(wraw[r], v);
+      float v[CPT];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] *= sc[j];
-      FqResult fr;
-      fq_group8<GL>(v, bits, sym, fr);
-      if (real) {
+      for (int q = 0; q < CPT / 8; ++q) {
+        float f[8];
+        unpack_bf16x8(wraw[r][q], f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[8 * q + j] = f[j] * sc[8 * q + j];
+      }
+      FqGroup<CPT> fr;
+      fq_group<CPT, GL>(v, bits, sym, fr);
+      if (active && row0 + r < d_out) {
         const int row = row0 + r;
-        uint32_t word = 0;
+        uint32_t* wp = qweight + (long long)row * words + c0 / 8;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) word |= (fq_code(fr, j) & 0xFu) << (4 * j);
-        __stcs(qweight + (long long)row * chunks + chunk, word);
+        for (int q = 0; q < CPT / 8; ++q) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) word |= (fq_code(fr, 8 * q + j) & 0xFu) << (4 * j);
+          __stcs(wp + q, word);
+        }
         if ((chunk & (GL - 1)) == 0) {
           const long long gidx = (long long)row * groups + chunk / GL;
           scales[gidx] = __float2half_rn(fr.delta);

@@ -1,11 +1,11 @@
 // Group-wise uniform quantiser shared by the search (fake quantisation) and
 // the pack kernel, so that both decide every code the same way.
 //
-// One thread holds 8 consecutive input channels of one row; a group of g
-// channels is g/8 consecutive lanes of a warp (g/8 a power of two <= 32, and
-// groups never straddle warps). All 32 lanes must call fq_group8 together
-// (the group reductions are full-warp shuffles); lanes without data pass
-// neutral values (zeros) and belong to groups that are wholly inactive.
+// One thread holds CPT consecutive input channels of one row; a group of g
+// channels is GL = g/CPT consecutive lanes of a warp (a power of two <= 32;
+// groups never straddle warps). All 32 lanes must call fq_group together (the
+// group reductions are full-warp shuffles); lanes without data pass zeros and
+// belong to groups that are wholly inactive.
 //
 // Quantiser ([P1] 量化基础, [P2] §2.1, [P4] §三, [P5] §2.3):
 //   symmetric : Delta = max(max|v|, eps) / (2^(b-1) - 1)
@@ -15,7 +15,7 @@
 //               q = clamp(rne(v / Delta) + z, 0, 2^b - 1),   v_hat = (q - z) Delta
 // Arithmetic is fp32; Delta is the range times the fp32 constant 1/levels,
 // 1/Delta is the correctly rounded reciprocal, and rne(v / Delta) is rounded
-// from the exact product v * (1/Delta). GL = g/8 lanes form one group.
+// from the exact product v * (1/Delta).
 #pragma once
 #include <cuda_runtime.h>
 
@@ -30,11 +30,12 @@ __device__ __forceinline__ float inv_levels(int b) {
 
 // Codes are kept in "magic" form c = code_value + 1.5*2^23 (see below):
 // the stored code is c - lo and the dequantised value is (c - 1.5*2^23) * delta.
-struct FqResult {
-  float delta;  // quantisation step of the group
-  float zero;   // asymmetric: z; symmetric: 2^(b-1) (the stored zero)
-  float lo;     // c of stored code 0
-  float c[8];   // clamped magic-form codes
+template <int CPT>
+struct FqGroup {
+  float delta;   // quantisation step of the group
+  float zero;    // asymmetric: z; symmetric: 2^(b-1) (the stored zero)
+  float lo;      // c of stored code 0
+  float c[CPT];  // clamped magic-form codes of this thread's channels
 };
 
 // Round-to-nearest-even to an integer by the fp32 "magic number" method: for
@@ -42,7 +43,8 @@ struct FqResult {
 // rounds x to the nearest integer (ties to even), which subtracting the
 // constant recovers exactly. Here the addition is fused with the product
 // v * inv (one rounding of the exact product), which keeps the work on the
-// full-rate FMA pipe.
+// full-rate FMA pipe. Larger |x| only occur in saturated (clamped) cases,
+// where the ordering, which the method preserves, is all that matters.
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 
 template <int GL>
@@ -69,18 +71,30 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
   asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-__device__ __forceinline__ float max8(const float (&v)[8]) {
-  return fmaxf(max3f(max3f(max3f(v[0], v[1], v[2]), v[3], v[4]), v[5], v[6]), v[7]);
+template <int N>
+__device__ __forceinline__ float maxN(const float (&v)[N]) {
+  float m = v[0];
+  int j = 1;
+#pragma unroll
+  for (; j + 1 < N; j += 2) m = max3f(m, v[j], v[j + 1]);
+  if (j < N) m = fmaxf(m, v[j]);
+  return m;
 }
-__device__ __forceinline__ float min8(const float (&v)[8]) {
-  return fminf(min3f(min3f(min3f(v[0], v[1], v[2]), v[3], v[4]), v[5], v[6]), v[7]);
+template <int N>
+__device__ __forceinline__ float minN(const float (&v)[N]) {
+  float m = v[0];
+  int j = 1;
+#pragma unroll
+  for (; j + 1 < N; j += 2) m = min3f(m, v[j], v[j + 1]);
+  if (j < N) m = fminf(m, v[j]);
+  return m;
 }
 
-template <int GL>
-__device__ __forceinline__ void fq_group8(const float (&v)[8], int bits, bool symmetric, FqResult& r) {
+// Quantise this thread's CPT values of a group spread over GL lanes.
+template <int CPT, int GL>
+__device__ __forceinline__ void fq_group(const float (&v)[CPT], int bits, bool symmetric, FqGroup<CPT>& r) {
   if (symmetric) {
-    float amax = fmaxf(max8(v), -min8(v));
-    amax = group_max<GL>(amax);
+    const float amax = group_max<GL>(fmaxf(maxN(v), -minN(v)));
     const float qmax = (float)((1 << (bits - 1)) - 1);
     const float qmin = -(float)(1 << (bits - 1));
     r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
@@ -89,11 +103,11 @@ __device__ __forceinline__ void fq_group8(const float (&v)[8], int bits, bool sy
     r.lo = kRoundMagic + qmin;
     const float hi = kRoundMagic + qmax;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)  // clamp(rne(v / Delta), qmin, qmax) + magic
+    for (int j = 0; j < CPT; ++j)  // clamp(rne(v / Delta), qmin, qmax) + magic
       r.c[j] = fminf(fmaxf(__fmaf_rn(v[j], inv, kRoundMagic), r.lo), hi);
   } else {
-    const float mx = group_max<GL>(max8(v));
-    const float mn = group_min<GL>(min8(v));
+    const float mx = group_max<GL>(maxN(v));
+    const float mn = group_min<GL>(minN(v));
     const float levels = (float)((1 << bits) - 1);
     r.delta = fmaxf(mx - mn, kEpsDelta) * inv_levels(bits);
     const float inv = __frcp_rn(r.delta);
@@ -101,15 +115,21 @@ __device__ __forceinline__ void fq_group8(const float (&v)[8], int bits, bool sy
     r.lo = kRoundMagic - r.zero;
     const float hi = r.lo + levels;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)  // clamp(rne(v / Delta) + z, 0, 2^b - 1) - z + magic
+    for (int j = 0; j < CPT; ++j)  // clamp(rne(v / Delta) + z, 0, 2^b - 1) - z + magic
       r.c[j] = fminf(fmaxf(__fmaf_rn(v[j], inv, kRoundMagic), r.lo), hi);
   }
 }
 
 // Dequantised value v_hat of element j ((q - z) Delta, or q Delta when symmetric).
-__device__ __forceinline__ float fq_dequant(const FqResult& r, int j) { return (r.c[j] - kRoundMagic) * r.delta; }
+template <int CPT>
+__device__ __forceinline__ float fq_dequant(const FqGroup<CPT>& r, int j) {
+  return (r.c[j] - kRoundMagic) * r.delta;
+}
 
 // Stored (unsigned) code of element j.
-__device__ __forceinline__ unsigned fq_code(const FqResult& r, int j) { return (unsigned)(r.c[j] - r.lo); }
+template <int CPT>
+__device__ __forceinline__ unsigned fq_code(const FqGroup<CPT>& r, int j) {
+  return (unsigned)(r.c[j] - r.lo);
+}
 
 }  // namespace awq

@@ -108,7 +108,13 @@ __device__ __forceinline__ void gemm_tile_coords(int t, const GemmArgs& a, int& 
   const int r = t - g * per_group;
   mb = r / width;
   nb = first + (r - mb * width);
-  if (a.tri == TRI_K) nb = a.n_blocks_n - 1 - nb;  // longest contractions first
+  if (a.tri == TRI_K) {
+    // interleave long and short contractions: positions 0, 1, 2, 3, ... take
+    // column tiles n-1, 0, n-2, 1, ..., so every group of tiles (and every
+    // CTA's run of them) mixes both and a short tile's epilogue overlaps a
+    // long tile's MMAs
+    nb = (nb & 1) ? (nb >> 1) : a.n_blocks_n - 1 - (nb >> 1);
+  }
 }
 
 __device__ __forceinline__ int gemm_num_kb(const GemmArgs& a, int nb) {
@@ -305,6 +311,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       float sum = 0.f;
 #pragma unroll 1
       for (int c = 0; c < GEMM_BN / 32; ++c) {
+        uint4 e[4];  // EPI_DOT: the 32 elements of E this chunk multiplies, fetched before the TMEM load
+        if constexpr (MODE == EPI_DOT) {
+          const int col = n0 + c * 32;
+          const __nv_bfloat16* erow = args.E + (long long)m * args.ldE + col;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            e[v] = (m < args.M && col + v * 8 < args.N) ? __ldg(reinterpret_cast<const uint4*>(erow + v * 8))
+                                                         : make_uint4(0, 0, 0, 0);
+        }
         uint32_t r[32];
         tmem_ld_32x32b_x32(taddr + c * 32, r);
         tmem_ld_wait();
@@ -315,20 +330,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             sum = fmaf(d, d, sum);
           }
         } else if constexpr (MODE == EPI_DOT) {
-          const int col = n0 + c * 32;
-          if (m < args.M) {
-            const __nv_bfloat16* erow = args.E + (long long)m * args.ldE + col;
+          // columns past N hold D = 0 (zero-filled B rows) and e = 0
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              if (col + v * 8 < args.N) {
-                const uint4 e = __ldg(reinterpret_cast<const uint4*>(erow + v * 8));
-                const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
+          for (int v = 0; v < 4; ++v) {
+            const uint32_t ew[4] = {e[v].x, e[v].y, e[v].z, e[v].w};
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  sum = fmaf(__uint_as_float(r[v * 8 + 2 * h]), bf16lo(ew[h]), sum);
-                  sum = fmaf(__uint_as_float(r[v * 8 + 2 * h + 1]), bf16hi(ew[h]), sum);
-                }
-              }
+            for (int h = 0; h < 4; ++h) {
+              sum = fmaf(__uint_as_float(r[v * 8 + 2 * h]), bf16lo(ew[h]), sum);
+              sum = fmaf(__uint_as_float(r[v * 8 + 2 * h + 1]), bf16hi(ew[h]), sum);
             }
           }
         } else {
