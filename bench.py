@@ -125,9 +125,13 @@ def tri_macs_per_row(d_in, block=256):
     return float(sum(min(block, d_in - j0) * min(d_in, j0 + block) for j0 in range(0, d_in, block)))
 
 
-def launches_per_step(form):
-    # stats 2 + scales 1 + fake-quant 1 + (transpose + Gram 2) + contraction 1 + reduce 2 + pack 1
-    return 8 + (2 if form == "gram" else 0)
+CHUNK_ALPHAS = 5  # awq_search_scales pipelines the grid in chunks of this many candidates
+
+
+def launches_per_step(form, n_alpha):
+    # stats 2 + scales 1 + per chunk (fake quant + contraction) + (transpose + Gram 2) + reduce 2 + pack 1
+    chunks = -(-n_alpha // CHUNK_ALPHAS)
+    return 6 + 2 * chunks + (2 if form == "gram" else 0)
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -161,7 +165,18 @@ def run_ours(args, rank, world, local_rank):
     cptr = ctypes.byref(cfg)
     wsp, wsn = ctypes.c_void_p(ws.data_ptr()), ws.numel()
 
+    def step_api(ev):
+        # the public calls, as a user makes them
+        ev[0].record()
+        awq.act_stats(X, ws_stats, out=a)
+        ev[1].record()
+        awq.search_scales(W, X, a, cfg, ws=ws, outputs=outs)
+        ev[2].record()
+        awq.quantize_pack(W, outs["s_best"], cfg, outputs=packed)
+        ev[3].record()
+
     def step(ev=None):
+        # the same path one step entry point at a time (no overlap), for the per-kernel breakdown
         st = B._stream()
         if ev is not None:
             ev[0].record()
@@ -187,13 +202,15 @@ def run_ours(args, rank, world, local_rank):
         if ev is not None:
             ev[6].record()
 
+    warm_ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     for _ in range(args.warmup):
         step()
+        step_api(warm_ev)
     torch.cuda.synchronize()
     awq.workspace_error(ws)
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -205,7 +222,7 @@ def run_ours(args, rank, world, local_rank):
     t_wall0 = time.perf_counter()
     for k in range(K):
         flush.fill_(k & 0xFF)  # evict L2 between timed steps (outside the step's events)
-        step(evs[k])
+        step_api(evs[k])
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -213,9 +230,19 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     awq.workspace_error(ws)
 
-    seg = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(6)] for k in range(K)])  # ms
-    step_ms = seg.sum(axis=1)
+    api = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(3)] for k in range(K)])  # ms
+    step_ms = api.sum(axis=1)
     total_ms = float(step_ms.sum())
+
+    # per-kernel breakdown: the same work one entry point at a time
+    KB = min(K, 20)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(KB)]
+    for k in range(KB):
+        flush.fill_(k & 0xFF)
+        step(kev[k])
+    torch.cuda.synchronize()
+    awq.workspace_error(ws)
+    seg = np.array([[kev[k][i].elapsed_time(kev[k][i + 1]) for i in range(6)] for k in range(KB)])
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -224,6 +251,9 @@ def run_ours(args, rank, world, local_rank):
     mean = seg.mean(axis=0)
     names = ["stats", "scales+fake_quant", "gram", "contraction", "reduce_argmin", "pack"]
     breakdown = {n: round(float(v), 4) for n, v in zip(names, mean)}
+    api_mean = api.mean(axis=0)
+    step_split = {"stats": round(float(api_mean[0]), 4), "search (overlapped)": round(float(api_mean[1]), 4),
+                  "pack": round(float(api_mean[2]), 4)}
 
     # ---- end to end through the public API with host buffers
     Wh = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -277,8 +307,8 @@ def run_ours(args, rank, world, local_rank):
     stats_bytes = N * d_in * 2 + d_in * 4
     pack_bytes = d_out * d_in * 2 + d_out * d_in // 2 + 2 * 2 * d_out * (d_in // wl.group) + d_in * 4
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    stats_gbs = stats_bytes / (breakdown["stats"] * 1e-3) / 1e9
-    pack_gbs = pack_bytes / (breakdown["pack"] * 1e-3) / 1e9
+    stats_gbs = stats_bytes / (step_split["stats"] * 1e-3) / 1e9
+    pack_gbs = pack_bytes / (step_split["pack"] * 1e-3) / 1e9
 
     line = {
         "metric": METRIC,
@@ -305,7 +335,9 @@ def run_ours(args, rank, world, local_rank):
                      "frac_of_sustained": round(achieved_tflops / peak_sustained, 4),
                      "traffic": profiled_traffic(wl.key, form),
                      "algorithmic_flops_per_launch": flops_search},
+        "step_ms": step_split,
         "breakdown_ms": breakdown,
+        "breakdown_note": "breakdown_ms: each step entry point timed alone (no overlap), " + str(KB) + " steps",
         "stats_gbs": round(stats_gbs, 1), "stats_hbm_frac": round(stats_gbs / hbm, 4),
         "pack_gbs": round(pack_gbs, 1), "pack_hbm_frac": round(pack_gbs / hbm, 4),
         "gram_tflops": round(flops_gram / (breakdown["gram"] * 1e-3) / 1e12, 2) if flops_gram else None,
@@ -313,7 +345,7 @@ def run_ours(args, rank, world, local_rank):
         "layers_per_s": round(world / (ms_per_step * 1e-3), 3),
         "e2e": {"value": round(world * n_a * K / (e2e_total * 1e-3), 2), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": launches_per_step(form) * K,
+        "gpu_launches": launches_per_step(form, n_a) * K,
         "clocks": clk,
         "wall_s_timed_region": round(t_wall, 3),
     }

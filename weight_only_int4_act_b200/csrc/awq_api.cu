@@ -311,21 +311,20 @@ awq_status awq_step_scales(const float* a, int64_t d_out, int64_t d_in, int64_t 
   return launch_status();
 }
 
-awq_status awq_step_fake_quant(const void* W, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
-                               size_t ws_bytes, awq_stream_t stream) {
-  SearchLayout L;
-  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
-  if (st != AWQ_OK) return st;
-  if (!W || !aligned(W, 16)) return AWQ_ERR_INVALID_ARG;
-  int sms = 0;
-  if ((st = check_device(&sms)) != AWQ_OK) return st;
+// Fake quantisation of grid points [k0, k1) into their slices of the dW stack.
+// max_per_sm > 0 caps the grid at that many blocks per SM (so that the kernel
+// can share the SMs with a concurrently running GEMM).
+awq_status launch_fake_quant(const void* W, int64_t d_out, int64_t d_in, const awq_qcfg* cfg, const SearchLayout& L,
+                             void* ws, int k0, int k1, int sms, int max_per_sm, cudaStream_t st) {
+  const long long slice = (long long)L.d_out_pad * d_in;
   auto launch = [&](auto kernel, int cpt) {
     const long long units = (long long)(L.d_out_pad / FQ_ROWS) * (d_in / cpt);
-    const int grid = elementwise_grid(kernel, units, sms);
-    kernel<<<grid, 256, 0, as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in,
-                                                L.d_out_pad, at<float>(ws, L.off_s), at<float>(ws, L.off_inv),
-                                                cfg->n_alpha, cfg->bits, cfg->symmetric,
-                                                at<__nv_bfloat16>(ws, L.off_dw));
+    int grid = elementwise_grid(kernel, units, sms);
+    if (max_per_sm > 0 && grid > sms * max_per_sm) grid = sms * max_per_sm;
+    kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in, L.d_out_pad,
+                                 at<float>(ws, L.off_s) + (long long)k0 * d_in,
+                                 at<float>(ws, L.off_inv) + (long long)k0 * d_in, k1 - k0, cfg->bits,
+                                 cfg->symmetric, at<__nv_bfloat16>(ws, L.off_dw) + k0 * slice);
   };
   constexpr int C = FQ_CPT;
   switch (cfg->group) {
@@ -338,6 +337,67 @@ awq_status awq_step_fake_quant(const void* W, int64_t d_out, int64_t d_in, int64
     default: return AWQ_ERR_INVALID_ARG;
   }
   return launch_status();
+}
+
+// The error contraction for grid points [k0, k1): rows [k0, k1) * d_out_pad of
+// the dW stack.
+awq_status launch_contract(const void* X, int64_t d_in, int64_t N, const SearchLayout& L, void* ws, int k0, int k1,
+                           int sms, cudaStream_t st) {
+  GemmArgs ga{};
+  const long long row0 = (long long)k0 * L.d_out_pad;
+  const long long rows = (long long)(k1 - k0) * L.d_out_pad;
+  ga.part = at<float>(ws, L.off_part) + row0;
+  ga.part_ld = L.M;
+  ga.err = at<int>(ws, 0);
+  ga.tile_counter = at<int>(ws, kTileCounterOffset);
+  const __nv_bfloat16* dw = at<__nv_bfloat16>(ws, L.off_dw) + row0 * d_in;
+  if (L.form == AWQ_FORM_DIRECT) return run_gemm<EPI_SUMSQ>(dw, rows, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, st);
+  ga.E = dw;
+  ga.ldE = d_in;
+  return run_gemm<EPI_DOT>(dw, rows, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms, st);
+}
+
+// Per device: the auxiliary stream and events with which awq_search_scales
+// overlaps the fake quantisation of one chunk of the grid with the
+// contraction of the previous chunk. Created on first use, kept until exit.
+constexpr int kChunkAlphas = 5;
+constexpr int kMaxChunks = (MAX_ALPHA + kChunkAlphas - 1) / kChunkAlphas;
+constexpr int kAuxMaxDevices = 64;
+struct DeviceAux {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t chunk_done[kMaxChunks] = {};
+};
+std::mutex g_aux_mu;
+DeviceAux g_aux[kAuxMaxDevices];
+
+awq_status device_aux(DeviceAux** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (dev < 0 || dev >= kAuxMaxDevices) return AWQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_aux_mu);
+  DeviceAux& d = g_aux[dev];
+  if (!d.stream) {
+    cudaStream_t s = nullptr;
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return AWQ_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) != cudaSuccess) return AWQ_ERR_CUDA;
+    for (int c = 0; c < kMaxChunks; ++c)
+      if (cudaEventCreateWithFlags(&d.chunk_done[c], cudaEventDisableTiming) != cudaSuccess) return AWQ_ERR_CUDA;
+    d.stream = s;
+  }
+  *out = &d;
+  return AWQ_OK;
+}
+
+awq_status awq_step_fake_quant(const void* W, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                               size_t ws_bytes, awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  if (!W || !aligned(W, 16)) return AWQ_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((st = check_device(&sms)) != AWQ_OK) return st;
+  return launch_fake_quant(W, d_out, d_in, cfg, L, ws, 0, cfg->n_alpha, sms, 0, as_stream(stream));
 }
 
 awq_status awq_step_gram(const void* X, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
@@ -368,21 +428,10 @@ awq_status awq_step_contract(const void* X, int64_t d_out, int64_t d_in, int64_t
   SearchLayout L;
   awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
   if (st != AWQ_OK) return st;
+  if (L.form == AWQ_FORM_DIRECT && (!X || !aligned(X, 16))) return AWQ_ERR_INVALID_ARG;
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;
-  GemmArgs ga{};
-  ga.part = at<float>(ws, L.off_part);
-  ga.err = at<int>(ws, 0);
-  ga.tile_counter = at<int>(ws, kTileCounterOffset);
-  const void* dw = at<void>(ws, L.off_dw);
-  if (L.form == AWQ_FORM_DIRECT) {
-    if (!X || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
-    return run_gemm<EPI_SUMSQ>(dw, L.M, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, as_stream(stream));
-  }
-  ga.E = at<__nv_bfloat16>(ws, L.off_dw);
-  ga.ldE = d_in;
-  return run_gemm<EPI_DOT>(dw, L.M, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms,
-                           as_stream(stream));
+  return launch_contract(X, d_in, N, L, ws, 0, cfg->n_alpha, sms, as_stream(stream));
 }
 
 awq_status awq_step_reduce(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws, size_t ws_bytes,
@@ -410,10 +459,31 @@ awq_status awq_search_scales(const void* W, const void* X, const float* a, int64
   if (st != AWQ_OK) return st;
   if (!W || !X || !a || !losses || !best || !s_best) return AWQ_ERR_INVALID_ARG;
   if (!aligned(W, 16) || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((st = check_device(&sms)) != AWQ_OK) return st;
+  DeviceAux* aux = nullptr;
+  if ((st = device_aux(&aux)) != AWQ_OK) return st;
+  cudaStream_t s = as_stream(stream);
   if ((st = awq_step_scales(a, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
-  if ((st = awq_step_fake_quant(W, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  // fork: the fake quantisation runs chunk by chunk on the auxiliary stream,
+  // each chunk signalling its event; the Gram product and the contraction of
+  // chunk c (which waits for chunk c's event) run on the caller's stream, so
+  // the write-bound fake quantisation of chunk c+1 overlaps the tensor-bound
+  // contraction of chunk c. The last wait joins the two streams.
+  const int n_chunks = (cfg->n_alpha + kChunkAlphas - 1) / kChunkAlphas;
+  if (cudaEventRecord(aux->fork, s) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (cudaStreamWaitEvent(aux->stream, aux->fork, 0) != cudaSuccess) return AWQ_ERR_CUDA;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int k0 = c * kChunkAlphas, k1 = k0 + kChunkAlphas < cfg->n_alpha ? k0 + kChunkAlphas : cfg->n_alpha;
+    if ((st = launch_fake_quant(W, d_out, d_in, cfg, L, ws, k0, k1, sms, 1, aux->stream)) != AWQ_OK) return st;
+    if (cudaEventRecord(aux->chunk_done[c], aux->stream) != cudaSuccess) return AWQ_ERR_CUDA;
+  }
   if ((st = awq_step_gram(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
-  if ((st = awq_step_contract(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  for (int c = 0; c < n_chunks; ++c) {
+    const int k0 = c * kChunkAlphas, k1 = k0 + kChunkAlphas < cfg->n_alpha ? k0 + kChunkAlphas : cfg->n_alpha;
+    if (cudaStreamWaitEvent(s, aux->chunk_done[c], 0) != cudaSuccess) return AWQ_ERR_CUDA;
+    if ((st = launch_contract(X, d_in, N, L, ws, k0, k1, sms, s)) != AWQ_OK) return st;
+  }
   return awq_step_reduce(d_out, d_in, N, cfg, ws, ws_bytes, losses, best, s_best, row_losses, stream);
 }
 

@@ -28,14 +28,14 @@ __device__ __forceinline__ float inv_levels(int b) {
   return b == 4 ? (1.0f / 15.0f) : b == 3 ? (1.0f / 7.0f) : b == 2 ? (1.0f / 3.0f) : 1.0f;
 }
 
-// Codes are kept in "magic" form c = code_value + 1.5*2^23 (see below):
-// the stored code is c - lo and the dequantised value is (c - 1.5*2^23) * delta.
+// Codes are kept in "magic" form c = stored code + 1.5*2^23 (see below):
+// the stored code is c - 1.5*2^23 and the dequantised value is (c - off) * delta.
 template <int CPT>
 struct FqGroup {
   float delta;   // quantisation step of the group
   float zero;    // asymmetric: z; symmetric: 2^(b-1) (the stored zero)
-  float lo;      // c of stored code 0
-  float c[CPT];  // clamped magic-form codes of this thread's channels
+  float off;     // 1.5*2^23 + z (asymmetric) or 1.5*2^23 + 2^(b-1) (symmetric)
+  float c[CPT];  // magic-form codes of this thread's channels
 };
 
 // Round-to-nearest-even to an integer by the fp32 "magic number" method: for
@@ -90,46 +90,56 @@ __device__ __forceinline__ float minN(const float (&v)[N]) {
   return m;
 }
 
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Quantise this thread's CPT values of a group spread over GL lanes.
+// The clamp to the code range is done on the FMA pipe: with span = 2^b - 1
+// codes, y = sat((v / Delta + z) / span) is clamp(v / Delta + z, 0, span) / span,
+// and fma(y, span, 1.5*2^23) rounds y * span to the nearest integer (ties to
+// even) in magic form. This equals clamp(rne(v / Delta) + z, 0, span) except
+// where v / Delta lies within ~1e-6 of a rounding boundary.
 template <int CPT, int GL>
 __device__ __forceinline__ void fq_group(const float (&v)[CPT], int bits, bool symmetric, FqGroup<CPT>& r) {
+  const float span = (float)((1 << bits) - 1);
+  const float inv_span = inv_levels(bits);
+  float a, b;  // y = sat(v * a + b)
   if (symmetric) {
     const float amax = group_max<GL>(fmaxf(maxN(v), -minN(v)));
-    const float qmax = (float)((1 << (bits - 1)) - 1);
-    const float qmin = -(float)(1 << (bits - 1));
+    const float half = (float)(1 << (bits - 1));  // -qmin
     r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
     const float inv = __frcp_rn(r.delta);
-    r.zero = -qmin;
-    r.lo = kRoundMagic + qmin;
-    const float hi = kRoundMagic + qmax;
-#pragma unroll
-    for (int j = 0; j < CPT; ++j)  // clamp(rne(v / Delta), qmin, qmax) + magic
-      r.c[j] = fminf(fmaxf(__fmaf_rn(v[j], inv, kRoundMagic), r.lo), hi);
+    r.zero = half;
+    r.off = kRoundMagic + half;
+    a = inv * inv_span;
+    b = half * inv_span;  // q - qmin = rne(v / Delta) + 2^(b-1)
   } else {
     const float mx = group_max<GL>(maxN(v));
     const float mn = group_min<GL>(minN(v));
-    const float levels = (float)((1 << bits) - 1);
-    r.delta = fmaxf(mx - mn, kEpsDelta) * inv_levels(bits);
+    r.delta = fmaxf(mx - mn, kEpsDelta) * inv_span;
     const float inv = __frcp_rn(r.delta);
-    r.zero = fminf(fmaxf(__fmaf_rn(-mn, inv, kRoundMagic) - kRoundMagic, 0.f), levels);  // rne(-min / Delta)
-    r.lo = kRoundMagic - r.zero;
-    const float hi = r.lo + levels;
-#pragma unroll
-    for (int j = 0; j < CPT; ++j)  // clamp(rne(v / Delta) + z, 0, 2^b - 1) - z + magic
-      r.c[j] = fminf(fmaxf(__fmaf_rn(v[j], inv, kRoundMagic), r.lo), hi);
+    r.zero = fminf(fmaxf(__fmaf_rn(-mn, inv, kRoundMagic) - kRoundMagic, 0.f), span);  // clamp(rne(-min / Delta))
+    r.off = kRoundMagic + r.zero;
+    a = inv * inv_span;
+    b = r.zero * inv_span;
   }
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) r.c[j] = __fmaf_rn(fma_sat(v[j], a, b), span, kRoundMagic);
 }
 
 // Dequantised value v_hat of element j ((q - z) Delta, or q Delta when symmetric).
 template <int CPT>
 __device__ __forceinline__ float fq_dequant(const FqGroup<CPT>& r, int j) {
-  return (r.c[j] - kRoundMagic) * r.delta;
+  return (r.c[j] - r.off) * r.delta;
 }
 
 // Stored (unsigned) code of element j.
 template <int CPT>
 __device__ __forceinline__ unsigned fq_code(const FqGroup<CPT>& r, int j) {
-  return (unsigned)(r.c[j] - r.lo);
+  return (unsigned)(r.c[j] - kRoundMagic);
 }
 
 }  // namespace awq

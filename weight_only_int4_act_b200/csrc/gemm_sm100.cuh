@@ -68,7 +68,8 @@ struct GemmArgs {
   int num_tiles;               // tiles visited (all, or the lower block triangle)
   int n_blocks_m, n_blocks_n;  // ceil(M/128), ceil(N/256)
   int group_n;                 // raster group width in N-blocks
-  float* part;                 // SUMSQ / DOT: [n_blocks_n][M] per-row partial sums
+  float* part;                 // SUMSQ / DOT: part[n_blk * part_ld + m], per-row partial sums
+  long long part_ld;
   const __nv_bfloat16* E;      // DOT: E[M, ldE]; element (m, n) multiplies D[m, n]
   long long ldE;
   __nv_bfloat16* C;            // STORE: C[M, ldC]
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(acc));
       if constexpr (MODE != EPI_STORE) {
-        if (m < args.M) args.part[(long long)nb * args.M + m] = sum;
+        if (m < args.M) args.part[(long long)nb * args.part_ld + m] = sum;
       }
     }
   }
