@@ -15,10 +15,9 @@
  *   - X is bf16 [N, d_in], row-major (N calibration tokens x input channels).
  *   - Groups are g consecutive input channels within one row of W.
  *   - Every pointer argument is DEVICE memory owned by the caller, unless the
- *     comment says "host". The library allocates no device memory; scratch
- *     memory is the caller's workspace. Its only state is, per device, the
- *     auxiliary stream and events awq_search_scales uses (created on its first
- *     call on that device; make that first call before any stream capture).
+ *     comment says "host". The library allocates no device memory and keeps
+ *     no state of its own beyond what awq_act_stats_noalloc documents;
+ *     scratch memory is the caller's workspace.
  *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
  *     the legacy default stream). A returned AWQ_OK means the work was
  *     validated and enqueued. Errors the device finds (a wait that timed out,
@@ -113,11 +112,7 @@ awq_status awq_act_stats_noalloc(const void* X_bf16, int64_t N, int64_t d_in, fl
  *   L_k = ||dW X^T||_F^2                                               ([P5] §1.1, §4.1)
  * then best = argmin_k L_k (lowest k on ties) and s_best = s(alpha_best).
  * The contraction runs on tcgen05 tensor cores with bf16 operands and fp32
- * accumulation, either directly (dW X^T) or through G = X^T X. The grid is
- * processed in chunks of 5 candidates: the fake quantisation of a chunk runs
- * on the library's auxiliary stream while the contraction of the previous one
- * runs on `stream` (joined back into `stream` before the reduction). Calls
- * from several host threads at once serialise on the auxiliary stream.
+ * accumulation, either directly (dW X^T) or through G = X^T X.
  * Outputs (device): losses float [n_alpha]; best int32 [1]; s_best float
  * [d_in]; row_losses float [n_alpha, d_out] (per-row losses) or NULL.
  * On non-finite losses the device sets best = -1, fills s_best with NaN and

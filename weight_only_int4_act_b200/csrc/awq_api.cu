@@ -221,7 +221,9 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
   if (tiles > INT32_MAX) return AWQ_ERR_SHAPE;
   args.num_tiles = (int)tiles;
   if (cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) !=
-      cudaSuccess)
+          cudaSuccess ||
+      cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
     return AWQ_ERR_CUDA;
   if (cudaMemsetAsync(args.tile_counter, 0, sizeof(int), st) != cudaSuccess) return AWQ_ERR_CUDA;
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
@@ -312,8 +314,7 @@ awq_status awq_step_scales(const float* a, int64_t d_out, int64_t d_in, int64_t 
 }
 
 // Fake quantisation of grid points [k0, k1) into their slices of the dW stack.
-// max_per_sm > 0 caps the grid at that many blocks per SM (so that the kernel
-// can share the SMs with a concurrently running GEMM).
+// max_per_sm > 0 caps the grid at that many blocks per SM.
 awq_status launch_fake_quant(const void* W, int64_t d_out, int64_t d_in, const awq_qcfg* cfg, const SearchLayout& L,
                              void* ws, int k0, int k1, int sms, int max_per_sm, cudaStream_t st) {
   const long long slice = (long long)L.d_out_pad * d_in;
@@ -355,38 +356,6 @@ awq_status launch_contract(const void* X, int64_t d_in, int64_t N, const SearchL
   ga.E = dw;
   ga.ldE = d_in;
   return run_gemm<EPI_DOT>(dw, rows, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms, st);
-}
-
-// Per device: the auxiliary stream and events with which awq_search_scales
-// overlaps the fake quantisation of one chunk of the grid with the
-// contraction of the previous chunk. Created on first use, kept until exit.
-constexpr int kChunkAlphas = 5;
-constexpr int kMaxChunks = (MAX_ALPHA + kChunkAlphas - 1) / kChunkAlphas;
-constexpr int kAuxMaxDevices = 64;
-struct DeviceAux {
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr;
-  cudaEvent_t chunk_done[kMaxChunks] = {};
-};
-std::mutex g_aux_mu;
-DeviceAux g_aux[kAuxMaxDevices];
-
-awq_status device_aux(DeviceAux** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
-  if (dev < 0 || dev >= kAuxMaxDevices) return AWQ_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_aux_mu);
-  DeviceAux& d = g_aux[dev];
-  if (!d.stream) {
-    cudaStream_t s = nullptr;
-    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return AWQ_ERR_CUDA;
-    if (cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) != cudaSuccess) return AWQ_ERR_CUDA;
-    for (int c = 0; c < kMaxChunks; ++c)
-      if (cudaEventCreateWithFlags(&d.chunk_done[c], cudaEventDisableTiming) != cudaSuccess) return AWQ_ERR_CUDA;
-    d.stream = s;
-  }
-  *out = &d;
-  return AWQ_OK;
 }
 
 awq_status awq_step_fake_quant(const void* W, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
@@ -459,31 +428,10 @@ awq_status awq_search_scales(const void* W, const void* X, const float* a, int64
   if (st != AWQ_OK) return st;
   if (!W || !X || !a || !losses || !best || !s_best) return AWQ_ERR_INVALID_ARG;
   if (!aligned(W, 16) || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
-  int sms = 0;
-  if ((st = check_device(&sms)) != AWQ_OK) return st;
-  DeviceAux* aux = nullptr;
-  if ((st = device_aux(&aux)) != AWQ_OK) return st;
-  cudaStream_t s = as_stream(stream);
   if ((st = awq_step_scales(a, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
-  // fork: the fake quantisation runs chunk by chunk on the auxiliary stream,
-  // each chunk signalling its event; the Gram product and the contraction of
-  // chunk c (which waits for chunk c's event) run on the caller's stream, so
-  // the write-bound fake quantisation of chunk c+1 overlaps the tensor-bound
-  // contraction of chunk c. The last wait joins the two streams.
-  const int n_chunks = (cfg->n_alpha + kChunkAlphas - 1) / kChunkAlphas;
-  if (cudaEventRecord(aux->fork, s) != cudaSuccess) return AWQ_ERR_CUDA;
-  if (cudaStreamWaitEvent(aux->stream, aux->fork, 0) != cudaSuccess) return AWQ_ERR_CUDA;
-  for (int c = 0; c < n_chunks; ++c) {
-    const int k0 = c * kChunkAlphas, k1 = k0 + kChunkAlphas < cfg->n_alpha ? k0 + kChunkAlphas : cfg->n_alpha;
-    if ((st = launch_fake_quant(W, d_out, d_in, cfg, L, ws, k0, k1, sms, 1, aux->stream)) != AWQ_OK) return st;
-    if (cudaEventRecord(aux->chunk_done[c], aux->stream) != cudaSuccess) return AWQ_ERR_CUDA;
-  }
+  if ((st = awq_step_fake_quant(W, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
   if ((st = awq_step_gram(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
-  for (int c = 0; c < n_chunks; ++c) {
-    const int k0 = c * kChunkAlphas, k1 = k0 + kChunkAlphas < cfg->n_alpha ? k0 + kChunkAlphas : cfg->n_alpha;
-    if (cudaStreamWaitEvent(s, aux->chunk_done[c], 0) != cudaSuccess) return AWQ_ERR_CUDA;
-    if ((st = launch_contract(X, d_in, N, L, ws, k0, k1, sms, s)) != AWQ_OK) return st;
-  }
+  if ((st = awq_step_contract(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
   return awq_step_reduce(d_out, d_in, N, cfg, ws, ws_bytes, losses, best, s_best, row_losses, stream);
 }
 
