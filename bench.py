@@ -119,6 +119,16 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm)}
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of a list of floats over all ranks of the default
+    process group (every rank must call it, in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu().tolist()]
+
+
 def tri_macs_per_row(d_in, block=256):
     """Multiply-adds per row of the block-triangular Gram contraction:
     sum over 256-wide column blocks J of width(J) * min(d_in, 256 (J + 1))."""
@@ -240,9 +250,9 @@ def run_ours(args, rank, world, local_rank):
     awq.workspace_error(ws)
     seg = np.array([[kev[k][i].elapsed_time(kev[k][i + 1]) for i in range(6)] for k in range(KB)])
     if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        seg = np.array(max_over_ranks(seg.ravel().tolist(), dev)).reshape(seg.shape)
+    if world > 1:
+        total_ms = max_over_ranks([total_ms], dev)[0]
     ms_per_step = total_ms / K
     mean = seg.mean(axis=0)
     names = ["stats", "scales+fake_quant", "gram", "contraction", "reduce_argmin", "pack"]
@@ -282,9 +292,7 @@ def run_ours(args, rank, world, local_rank):
         e_ms.append(e0.elapsed_time(e1))
     e2e_total = float(sum(e_ms))
     if world > 1:
-        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+        e2e_total = max_over_ranks([e2e_total], dev)[0]
     awq.workspace_error(ws)
     h2d = Wb.nbytes + Xb.nbytes
     d2h = sum(h.numel() * h.element_size() for h in host_out)

@@ -1,0 +1,83 @@
+"""Host-side logic of bench.py: the max-over-ranks timing used when one
+process per GPU runs under torchrun (checked here with 2 gloo ranks on the
+CPU), the triangular multiply-add count, launch counting, the ncu-summary
+reader, and the reference (CPU oracle) arm's JSON line."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mine = [float(rank + 1), 10.0 - rank, 3.0]
+        res = bench.max_over_ranks(mine, "cpu")
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+            json.dump(res, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo(tmp_path):
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.spawn(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    for r in range(2):
+        assert json.loads((tmp_path / f"r{r}.json").read_text()) == [2.0, 10.0, 3.0]
+
+
+def test_tri_macs_matches_block_count():
+    for d_in in (64, 256, 384, 4096, 11008):
+        brute = 0
+        for i in range(d_in):
+            brute += min(d_in, (i // 256 + 1) * 256)  # row i of G' holds columns of blocks <= its block
+        assert bench.tri_macs_per_row(d_in) == brute
+
+
+def test_launch_count():
+    assert bench.launches_per_step("direct", 20) == 8
+    assert bench.launches_per_step("gram", 20) == 10
+
+
+def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "contract_gram_CX.md").write_text(
+        f"- source_sha256: `{bench.kernel_source_hash()}`\n- traffic_bytes_per_launch: `123`\n")
+    (prof / "contract_gram_CY.md").write_text("- source_sha256: `0000`\n- traffic_bytes_per_launch: `456`\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "weight_only_int4_act_b200" / "csrc").mkdir(parents=True)
+    for f in ("gemm_sm100.cuh", "ptx.cuh"):
+        src = os.path.join(ROOT, "weight_only_int4_act_b200", "csrc", f)
+        (tmp_path / "weight_only_int4_act_b200" / "csrc" / f).write_bytes(open(src, "rb").read())
+    assert bench.profiled_traffic("CX", "gram") == 123.0
+    assert bench.profiled_traffic("CY", "gram") is None
+    assert bench.profiled_traffic("CZ", "gram") is None
+
+
+def test_reference_arm_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "C1",
+                          "--steps", "1", "--warmup", "3", "--ref-rows", "64"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == bench.UNIT and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["higher_is_better"] is True
