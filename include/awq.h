@@ -126,6 +126,27 @@ awq_status awq_search_scales(const void* W_bf16, const void* X_bf16, const float
                              float* losses, int32_t* best, float* s_best, float* row_losses,
                              awq_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * The search for several linear layers that read the same activations X
+ * (for example the q/k/v projections, or gate/up): W is their row
+ * concatenation [d_out, d_in] with layer i holding seg_rows[i] consecutive
+ * rows (HOST array, n_seg in 1..16, sum = d_out). The statistics, the Gram
+ * product and one fake-quant and contraction launch serve all layers; each
+ * layer gets its own losses and choice:
+ *   losses float [n_seg, n_alpha], best int32 [n_seg], s_best float
+ *   [n_seg, d_in], row_losses as in awq_search_scales (or NULL).
+ * Layers whose scales are folded into one shared preceding operation need a
+ * single shared choice: that is awq_search_scales on the same concatenated W
+ * (its loss is the sum over the layers). Workspace: awq_search_workspace_size
+ * with the total d_out. Errors as awq_search_scales, plus
+ * AWQ_ERR_INVALID_ARG for n_seg out of range and AWQ_ERR_SHAPE when the
+ * segment sizes do not sum to d_out.
+ * ------------------------------------------------------------------------- */
+awq_status awq_search_scales_segmented(const void* W_bf16, const void* X_bf16, const float* a, int64_t d_out,
+                                       int64_t d_in, int64_t N, const awq_qcfg* cfg, int32_t n_seg,
+                                       const int64_t* seg_rows, void* ws, size_t ws_bytes, float* losses,
+                                       int32_t* best, float* s_best, float* row_losses, awq_stream_t stream);
+
 /* The contraction form awq_search_scales will use for these sizes (1 direct,
  * 2 Gram): AUTO picks the one with fewer multiply-adds, n_alpha*d_out*d_in*N
  * versus (N + n_alpha*d_out) * T(d_in), where T(d_in) ~ d_in^2/2 counts the

@@ -117,3 +117,22 @@ def test_python_binding_refuses_cpu_tensors():
     X = torch.zeros((4, 16), dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA tensor"):
         awq.act_stats(X)
+
+
+def test_segmented_search_validation():
+    lib = awq.lib()
+    cfg = awq.make_cfg(4, 128, False, 20)
+    c = ctypes.byref(cfg)
+    big = 1 << 40
+
+    def call(rows, d_out=256):
+        arr = (ctypes.c_int64 * max(len(rows), 1))(*rows)
+        return lib.awq_search_scales_segmented(FAKE, FAKE, FAKE, d_out, 512, 256, c, len(rows), ctypes.cast(arr, ctypes.c_void_p),
+                                               FAKE, big, FAKE, FAKE, FAKE, None, None)
+    assert call([]) == 1                      # n_seg < 1
+    assert call([16] * 17, d_out=272) == 1    # n_seg > 16
+    assert call([100, 100]) == 2              # rows do not sum to d_out
+    assert call([200, 100]) == 2              # overshoot
+    assert call([256, 0]) == 2                # empty layer
+    assert lib.awq_search_scales_segmented(FAKE, FAKE, FAKE, 256, 512, 256, c, 1, None, FAKE, big, FAKE, FAKE, FAKE,
+                                           None, None) == 1

@@ -24,7 +24,7 @@ EXPORTED = (
     "awq_status_str", "awq_stats_workspace_size", "awq_act_stats", "awq_search_workspace_size",
     "awq_search_scales", "awq_search_form", "awq_workspace_error", "awq_quantize_pack",
     "awq_step_scales", "awq_step_fake_quant", "awq_step_gram", "awq_step_contract", "awq_step_reduce",
-    "awq_debug_copy_dw", "awq_act_stats_noalloc",
+    "awq_debug_copy_dw", "awq_act_stats_noalloc", "awq_search_scales_segmented",
 )
 
 
@@ -70,6 +70,9 @@ def lib() -> ctypes.CDLL:
             "awq_search_form": (c_int32, [c_int64, c_int64, c_int64, cfgp]),
             "awq_search_scales": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, cfgp,
                                             c_void_p, c_size_t, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+            "awq_search_scales_segmented": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, cfgp,
+                                                      c_int32, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p,
+                                                      c_void_p, c_void_p, c_void_p]),
             "awq_workspace_error": (c_int32, [c_void_p, c_void_p]),
             "awq_quantize_pack": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_void_p, c_void_p,
                                             c_void_p, c_void_p]),
@@ -187,6 +190,33 @@ def search_scales(W, X, a, cfg: QCfg, ws=None, row_losses=False, outputs=None):
     _check(lib().awq_search_scales(_ptr(W), _ptr(X), _ptr(a), d_out, d_in, N, ctypes.byref(cfg), _ptr(ws),
                                    ws.numel(), _ptr(o["losses"]), _ptr(o["best"]), _ptr(o["s_best"]),
                                    _ptr(o["row_losses"]), _stream()), "awq_search_scales")
+    return dict(o, ws=ws)
+
+
+def search_scales_segmented(W, X, a, cfg: QCfg, seg_rows, ws=None, row_losses=False):
+    """Per-layer search for layers sharing X; W is their row concatenation and
+    seg_rows the row count of each layer. Returns dict(losses float32[n_seg,
+    n_alpha], best int32[n_seg], s_best float32[n_seg, d_in], row_losses, ws)."""
+    torch = _torch()
+    _req(W, torch.bfloat16, None, "W")
+    d_out, d_in = W.shape
+    _req(X, torch.bfloat16, None, "X")
+    N = X.shape[0]
+    if X.shape[1] != d_in:
+        raise ValueError("X must have d_in columns")
+    _req(a, torch.float32, (d_in,), "a")
+    n_seg = len(seg_rows)
+    rows = (ctypes.c_int64 * max(n_seg, 1))(*[int(r) for r in seg_rows])
+    if ws is None:
+        ws = workspace(search_workspace_size(d_out, d_in, N, cfg))
+    o = dict(losses=torch.empty((n_seg, cfg.n_alpha), dtype=torch.float32, device=W.device),
+             best=torch.empty(n_seg, dtype=torch.int32, device=W.device),
+             s_best=torch.empty((n_seg, d_in), dtype=torch.float32, device=W.device),
+             row_losses=torch.empty((cfg.n_alpha, d_out), dtype=torch.float32, device=W.device) if row_losses else None)
+    _check(lib().awq_search_scales_segmented(_ptr(W), _ptr(X), _ptr(a), d_out, d_in, N, ctypes.byref(cfg), n_seg,
+                                             ctypes.cast(rows, c_void_p), _ptr(ws), ws.numel(), _ptr(o["losses"]),
+                                             _ptr(o["best"]), _ptr(o["s_best"]), _ptr(o["row_losses"]), _stream()),
+           "awq_search_scales_segmented")
     return dict(o, ws=ws)
 
 

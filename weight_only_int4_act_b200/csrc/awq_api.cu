@@ -112,7 +112,7 @@ struct SearchLayout {
   int n_blocks_n;   // column tiles of the contraction
   int n_red_chunks; // blocks per alpha in the row reduction
   long long ld_t;   // padded token count of X^T (Gram)
-  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_xt, off_g, total;
+  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_seg, off_xt, off_g, total;
 };
 
 // sum over 256-wide column blocks J of width(J) * min(d_in, 256 (J + 1)): the
@@ -151,6 +151,7 @@ SearchLayout search_layout(int64_t d_out, int64_t d_in, int64_t N, const awq_qcf
   L.off_part = off;   off += align_up((size_t)L.n_blocks_n * L.M * sizeof(float));
   L.off_blk = off;    off += align_up((size_t)L.n_alpha * L.n_red_chunks * sizeof(double));
   L.off_loss64 = off; off += align_up((size_t)L.n_alpha * sizeof(double));
+  L.off_seg = off;    off += align_up((size_t)MAX_ALPHA * MAX_SEG * sizeof(double));
   if (L.form == AWQ_FORM_GRAM) {
     L.off_xt = off;   off += align_up((size_t)d_in * L.ld_t * 2);
     L.off_g = off;    off += align_up((size_t)d_in * d_in * 2);
@@ -433,6 +434,39 @@ awq_status awq_search_scales(const void* W, const void* X, const float* a, int64
   if ((st = awq_step_gram(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
   if ((st = awq_step_contract(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
   return awq_step_reduce(d_out, d_in, N, cfg, ws, ws_bytes, losses, best, s_best, row_losses, stream);
+}
+
+awq_status awq_search_scales_segmented(const void* W, const void* X, const float* a, int64_t d_out, int64_t d_in,
+                                       int64_t N, const awq_qcfg* cfg, int32_t n_seg, const int64_t* seg_rows,
+                                       void* ws, size_t ws_bytes, float* losses, int32_t* best, float* s_best,
+                                       float* row_losses, awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  if (!W || !X || !a || !losses || !best || !s_best || !seg_rows) return AWQ_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
+  if (n_seg < 1 || n_seg > MAX_SEG) return AWQ_ERR_INVALID_ARG;
+  SegTable seg{};
+  int64_t acc = 0;
+  for (int i = 0; i < n_seg; ++i) {
+    if (seg_rows[i] < 1) return AWQ_ERR_SHAPE;
+    seg.start[i] = (int)acc;
+    acc += seg_rows[i];
+    if (acc > d_out) return AWQ_ERR_SHAPE;
+  }
+  if (acc != d_out) return AWQ_ERR_SHAPE;
+  seg.start[n_seg] = (int)acc;
+  if ((st = awq_step_scales(a, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  if ((st = awq_step_fake_quant(W, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  if ((st = awq_step_gram(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  if ((st = awq_step_contract(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  segment_loss_reduce<<<dim3(n_seg, L.n_alpha), REDUCE_THREADS, 0, s>>>(
+      at<float>(ws, L.off_part), L.n_blocks_n, L.M, (int)d_out, L.d_out_pad, seg, row_losses, at<double>(ws, L.off_seg));
+  if ((st = launch_status()) != AWQ_OK) return st;
+  segment_argmin<<<1, 32 * MAX_SEG, 0, s>>>(at<double>(ws, L.off_seg), n_seg, L.n_alpha, at<float>(ws, L.off_s),
+                                            (int)d_in, losses, best, s_best, at<int>(ws, 0));
+  return launch_status();
 }
 
 awq_status awq_workspace_error(void* ws, awq_stream_t stream) {

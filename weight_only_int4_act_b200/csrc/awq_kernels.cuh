@@ -336,6 +336,77 @@ __global__ void loss_argmin(const double* __restrict__ block_sums, int n_chunks,
 }
 
 // ---------------------------------------------------------------------------
+// a6 for several layers sharing X (rows of W split into segments, one layer
+// each): fp64 loss per (segment, alpha) in a fixed order, then an argmin per
+// segment. part layout as for row_loss_reduce.
+// ---------------------------------------------------------------------------
+constexpr int MAX_SEG = 16;
+
+struct SegTable {
+  int start[MAX_SEG + 1];  // segment s holds rows [start[s], start[s+1])
+};
+
+__global__ void __launch_bounds__(REDUCE_THREADS) segment_loss_reduce(const float* __restrict__ part, int n_blocks_n,
+                                                                      long long M, int d_out, int d_out_pad,
+                                                                      SegTable seg, float* __restrict__ row_losses,
+                                                                      double* __restrict__ seg_sums) {
+  __shared__ double red[REDUCE_THREADS];
+  const int sg = blockIdx.x, k = blockIdx.y;
+  double acc = 0.0;
+  for (int r = seg.start[sg] + threadIdx.x; r < seg.start[sg + 1]; r += REDUCE_THREADS) {
+    const long long m = (long long)k * d_out_pad + r;
+    double s = 0.0;
+    for (int nb = 0; nb < n_blocks_n; ++nb) s += (double)part[(long long)nb * M + m];
+    if (row_losses) row_losses[(long long)k * d_out + r] = (float)s;
+    acc += s;
+  }
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = REDUCE_THREADS / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) seg_sums[(long long)k * MAX_SEG + sg] = red[0];
+}
+
+// One warp per segment: losses[sg][k], warp-shuffle argmin (lowest k on ties),
+// s_best[sg][:] = s(alpha_best).
+__global__ void segment_argmin(const double* __restrict__ seg_sums, int n_seg, int n_alpha,
+                               const float* __restrict__ s_all, int d_in, float* __restrict__ losses,
+                               int* __restrict__ best_out, float* __restrict__ s_best, int* err) {
+  const int sg = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (sg >= n_seg) return;
+  double bv = INFINITY;
+  int bi = MAX_ALPHA;
+  bool finite = true;
+  for (int k = lane; k < n_alpha; k += 32) {
+    const double v = seg_sums[(long long)k * MAX_SEG + sg];
+    losses[(long long)sg * n_alpha + k] = (float)v;
+    if (!isfinite(v)) finite = false;
+    if (v < bv) {
+      bv = v;
+      bi = k;
+    }
+  }
+  for (int off = 16; off > 0; off >>= 1) {
+    const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+    if (ov < bv || (ov == bv && oi < bi)) {
+      bv = ov;
+      bi = oi;
+    }
+  }
+  finite = __all_sync(0xffffffffu, finite);
+  const int b = finite ? bi : -1;
+  if (lane == 0) {
+    best_out[sg] = b;
+    if (!finite && err) atomicCAS(err, 0, ERR_NONFINITE);
+  }
+  for (int i = lane; i < d_in; i += 32)
+    s_best[(long long)sg * d_in + i] = b >= 0 ? s_all[(long long)b * d_in + i] : __int_as_float(0x7fc00000);
+}
+
+// ---------------------------------------------------------------------------
 // a7: pack. Codes of Q(W S) (same quantiser as the search), 8 nibbles per
 // uint32 (channel 8w+j in bits 4j..4j+3), fp16 step and zero per group.
 // ([P2] §2.1 INT4 with fp16 scale, §4.2 packed 4-bit storage; [P4] §三.)
