@@ -136,8 +136,8 @@ def tri_macs_per_row(d_in, block=256):
 
 
 def launches_per_step(form, n_alpha):
-    # stats 2 + scales 1 + fake quant 1 + (transpose + Gram 2) + contraction 1 + reduce 2 + pack 1
-    return 8 + (2 if form == "gram" else 0)
+    # stats 2 + scales 1 + fake quant 1 + (Gram 1) + contraction 1 + reduce 2 + pack 1
+    return 8 + (1 if form == "gram" else 0)
 
 
 # ----------------------------------------------------------------------------- our arm

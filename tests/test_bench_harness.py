@@ -53,7 +53,7 @@ def test_tri_macs_matches_block_count():
 
 def test_launch_count():
     assert bench.launches_per_step("direct", 20) == 8
-    assert bench.launches_per_step("gram", 20) == 10
+    assert bench.launches_per_step("gram", 20) == 9
 
 
 def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):

@@ -111,8 +111,7 @@ struct SearchLayout {
   long long M;      // rows of the dW stack
   int n_blocks_n;   // column tiles of the contraction
   int n_red_chunks; // blocks per alpha in the row reduction
-  long long ld_t;   // padded token count of X^T (Gram)
-  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_seg, off_xt, off_g, total;
+  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_seg, off_g, total;
 };
 
 // sum over 256-wide column blocks J of width(J) * min(d_in, 256 (J + 1)): the
@@ -143,7 +142,6 @@ SearchLayout search_layout(int64_t d_out, int64_t d_in, int64_t N, const awq_qcf
   L.M = (long long)L.n_alpha * L.d_out_pad;
   L.n_blocks_n = (int)cdiv(L.form == AWQ_FORM_DIRECT ? N : d_in, GEMM_BN);
   L.n_red_chunks = (int)cdiv(d_out, REDUCE_THREADS);
-  L.ld_t = cdiv(N, 64) * 64;
   size_t off = kAlign;  // [0, 1024): error word and tile counter
   L.off_s = off;      off += align_up((size_t)L.n_alpha * d_in * sizeof(float));
   L.off_inv = off;    off += align_up((size_t)L.n_alpha * d_in * sizeof(float));
@@ -153,7 +151,6 @@ SearchLayout search_layout(int64_t d_out, int64_t d_in, int64_t N, const awq_qcf
   L.off_loss64 = off; off += align_up((size_t)L.n_alpha * sizeof(double));
   L.off_seg = off;    off += align_up((size_t)MAX_ALPHA * MAX_SEG * sizeof(double));
   if (L.form == AWQ_FORM_GRAM) {
-    L.off_xt = off;   off += align_up((size_t)d_in * L.ld_t * 2);
     L.off_g = off;    off += align_up((size_t)d_in * d_in * 2);
   }
   L.total = off;
@@ -204,12 +201,18 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 }
 
 // D = A[M, K] * B[Nr, K]^T with the given epilogue.
-template <int MODE>
+// MN = true: A and B are row-major [K, M] / [K, Nr] matrices read transposed.
+template <int MODE, bool MN = false>
 awq_status run_gemm(const void* A, long long M, long long lda, const void* B, long long Nr, long long ldb, long long K,
                     GemmArgs args, int tri, int num_sms, cudaStream_t st) {
   CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K, lda, GEMM_BM)) return AWQ_ERR_CUDA;
-  if (!make_map(&tb, B, Nr, K, ldb, GEMM_BN)) return AWQ_ERR_CUDA;
+  if (MN) {
+    if (!make_map(&ta, A, K, M, lda, GEMM_BK)) return AWQ_ERR_CUDA;
+    if (!make_map(&tb, B, K, Nr, ldb, GEMM_BK)) return AWQ_ERR_CUDA;
+  } else {
+    if (!make_map(&ta, A, M, K, lda, GEMM_BM)) return AWQ_ERR_CUDA;
+    if (!make_map(&tb, B, Nr, K, ldb, GEMM_BN)) return AWQ_ERR_CUDA;
+  }
   args.M = (int)M;
   args.N = (int)Nr;
   args.K = (int)K;
@@ -221,14 +224,14 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
                                                  : (long long)args.n_blocks_m * args.n_blocks_n;
   if (tiles > INT32_MAX) return AWQ_ERR_SHAPE;
   args.num_tiles = (int)tiles;
-  if (cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE>, cudaFuncAttributePreferredSharedMemoryCarveout,
+  if (cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE, MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           GEMM_SMEM_BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE, MN>, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared) != cudaSuccess)
     return AWQ_ERR_CUDA;
   if (cudaMemsetAsync(args.tile_counter, 0, sizeof(int), st) != cudaSuccess) return AWQ_ERR_CUDA;
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-  gemm_bf16_tcgen05<MODE><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(ta, tb, args);
+  gemm_bf16_tcgen05<MODE, MN><<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(ta, tb, args);
   return launch_status();
 }
 
@@ -379,18 +382,13 @@ awq_status awq_step_gram(const void* X, int64_t d_out, int64_t d_in, int64_t N, 
   if (!X || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;
-  cudaStream_t s = as_stream(stream);
-  dim3 tgrid((unsigned)(L.ld_t / 64), (unsigned)cdiv(d_in, 64));
-  transpose_bf16<<<tgrid, dim3(64, 4), 0, s>>>(static_cast<const __nv_bfloat16*>(X), N, (int)d_in, L.ld_t,
-                                               at<__nv_bfloat16>(ws, L.off_xt));
-  if ((st = launch_status()) != AWQ_OK) return st;
   GemmArgs ga{};
   ga.C = at<__nv_bfloat16>(ws, L.off_g);
   ga.ldC = d_in;
   ga.err = at<int>(ws, 0);
   ga.tile_counter = at<int>(ws, kTileCounterOffset);
-  const void* xt = at<void>(ws, L.off_xt);
-  return run_gemm<EPI_STORE>(xt, d_in, L.ld_t, xt, d_in, L.ld_t, L.ld_t, ga, TRI_LOWER_STORE, sms, s);
+  // G = X^T X with both operands read transposed from X [N, d_in] (MN-major)
+  return run_gemm<EPI_STORE, true>(X, d_in, d_in, X, d_in, d_in, N, ga, TRI_LOWER_STORE, sms, as_stream(stream));
 }
 
 awq_status awq_step_contract(const void* X, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,

@@ -1,7 +1,6 @@
 // SIMT kernels of the AWQ search path (everything except the tensor-core
-// contraction): activation statistics, candidate scales, the fake-quantised
-// dW stack, the transpose feeding the Gram product, the fixed-order loss
-// reduction with argmin, and the pack.
+// products): activation statistics, candidate scales, the fake-quantised dW
+// stack, the fixed-order loss reduction with argmin, and the pack.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -225,30 +224,6 @@ __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* 
         }
       }
     }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// a4 feed: XT[i][t] = X[t][i] (tokens padded with zeros to ld_t columns), so
-// that G = X^T X is a K-major product of XT with itself.
-// ---------------------------------------------------------------------------
-__global__ void transpose_bf16(const __nv_bfloat16* __restrict__ X, long long N, int d_in, long long ld_t,
-                               __nv_bfloat16* __restrict__ XT) {
-  __shared__ __nv_bfloat16 tile[64][65];
-  const long long t0 = (long long)blockIdx.x * 64;
-  const int i0 = blockIdx.y * 64;
-  for (int k = threadIdx.y; k < 64; k += blockDim.y) {
-    const long long t = t0 + k;
-    const int i = i0 + threadIdx.x;
-    __nv_bfloat16 v = __float2bfloat16(0.f);
-    if (t < N && i < d_in) v = X[t * d_in + i];
-    tile[k][threadIdx.x] = v;
-  }
-  __syncthreads();
-  for (int k = threadIdx.y; k < 64; k += blockDim.y) {
-    const int i = i0 + k;
-    const long long t = t0 + threadIdx.x;
-    if (i < d_in && t < ld_t) XT[(long long)i * ld_t + t] = tile[threadIdx.x][k];
   }
 }
 

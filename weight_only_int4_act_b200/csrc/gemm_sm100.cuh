@@ -53,6 +53,7 @@ constexpr int GEMM_THREADS = 192;
 constexpr int GEMM_A_STAGE = GEMM_BM * GEMM_BK * 2;  // 16 KB
 constexpr int GEMM_B_STAGE = GEMM_BN * GEMM_BK * 2;  // 32 KB
 constexpr int GEMM_TMEM_COLS = 512;
+constexpr int GEMM_MN_CHUNK = 64 * GEMM_BK * 2;  // MN-major: one 64-wide chunk of 64 k-rows (8 KB)
 constexpr int GEMM_SMEM_BYTES = 1024 /* alignment slack */ + GEMM_STAGES * (GEMM_A_STAGE + GEMM_B_STAGE) + 256;
 
 // error codes written to *err by the GEMM (distinct per wait site)
@@ -127,7 +128,12 @@ __device__ __forceinline__ int gemm_num_kb(const GemmArgs& a, int nb) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-template <int MODE>
+// MN = false: A [M, K] and B [N, K] row-major (K-major operands), one TMA box
+// of 64 x 128 (A) and 64 x 256 (B) rows per stage.
+// MN = true: A and B are the same row-major [K, M] matrix read transposed
+// (MN-major operands; G = X^T X straight from X), boxes of 64 (M or N) x 64
+// (K) loaded at 64-column offsets: 2 for A and 4 for B per stage.
+template <int MODE, bool MN = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const GemmArgs args) {
@@ -216,8 +222,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(full_bar(stage), GEMM_A_STAGE + GEMM_B_STAGE);
-          tma_load_2d(smem_u32(sA + stage * GEMM_A_STAGE), &tmA, full_bar(stage), kb * GEMM_BK, mb * GEMM_BM);
-          tma_load_2d(smem_u32(sB + stage * GEMM_B_STAGE), &tmB, full_bar(stage), kb * GEMM_BK, nb * GEMM_BN);
+          if constexpr (MN) {
+#pragma unroll
+            for (int c = 0; c < GEMM_BM / 64; ++c)
+              tma_load_2d(smem_u32(sA + stage * GEMM_A_STAGE + c * GEMM_MN_CHUNK), &tmA, full_bar(stage),
+                          mb * GEMM_BM + c * 64, kb * GEMM_BK);
+#pragma unroll
+            for (int c = 0; c < GEMM_BN / 64; ++c)
+              tma_load_2d(smem_u32(sB + stage * GEMM_B_STAGE + c * GEMM_MN_CHUNK), &tmB, full_bar(stage),
+                          nb * GEMM_BN + c * 64, kb * GEMM_BK);
+          } else {
+            tma_load_2d(smem_u32(sA + stage * GEMM_A_STAGE), &tmA, full_bar(stage), kb * GEMM_BK, mb * GEMM_BM);
+            tma_load_2d(smem_u32(sB + stage * GEMM_B_STAGE), &tmB, full_bar(stage), kb * GEMM_BK, nb * GEMM_BN);
+          }
           issued |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == GEMM_STAGES) {
@@ -233,7 +250,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer
-      constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, GEMM_BN);
+      constexpr uint32_t IDESC = idesc_bf16_f32(GEMM_BM, GEMM_BN, MN);
       int stage = 0;
       uint32_t phase = 0;
       int slot = 0;
@@ -266,8 +283,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t b_base = smem_u32(sB + stage * GEMM_B_STAGE);
 #pragma unroll
           for (int k = 0; k < GEMM_BK / 16; ++k) {
-            mma_bf16(d_tmem, desc_kmajor_sw128(a_base + k * 32), desc_kmajor_sw128(b_base + k * 32), IDESC,
-                     (kb | k) != 0);
+            // K-major: 16 elements = 32 B along the swizzled row; MN-major: 16 rows of 128 B
+            const uint64_t ad = MN ? desc_mnmajor_sw128(a_base + k * 2048, GEMM_MN_CHUNK)
+                                   : desc_kmajor_sw128(a_base + k * 32);
+            const uint64_t bd = MN ? desc_mnmajor_sw128(b_base + k * 2048, GEMM_MN_CHUNK)
+                                   : desc_kmajor_sw128(b_base + k * 32);
+            mma_bf16(d_tmem, ad, bd, IDESC, (kb | k) != 0);
           }
           mma_commit(empty_bar(stage));
           if (++stage == GEMM_STAGES) {

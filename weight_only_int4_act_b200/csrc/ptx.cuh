@@ -162,11 +162,27 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 D, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+// Shared-memory matrix descriptor for an MN-major operand tile stored with the
+// 128-byte swizzle: for each k (a 128-byte row) 64 consecutive M (or N)
+// elements; 8-row atoms of 1024 B (stride byte offset); successive 64-wide
+// MN chunks `mn_chunk_bytes` apart (leading byte offset).
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t mn_chunk_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((mn_chunk_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, shape M x N; both
+// operands K-major, or both MN-major ("transposed", bits 15 and 16).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool mn_major = false) {
   return (1u << 4)                     // D format: f32
          | (1u << 7)                   // A format: bf16
          | (1u << 10)                  // B format: bf16
+         | (mn_major ? (3u << 15) : 0u)
          | ((uint32_t)(N >> 3) << 17)  // N / 8
          | ((uint32_t)(M >> 4) << 24); // M / 16
 }
