@@ -11,6 +11,7 @@
 
 #include "../../include/awq.h"
 #include "awq_kernels.cuh"
+#include "gemm_pair_sm100.cuh"
 #include "gemm_sm100.cuh"
 
 using namespace awq;
@@ -235,6 +236,36 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
   return launch_status();
 }
 
+// The contraction on CTA pairs (gemm_pair_sm100.cuh): 256 x 256 tiles.
+template <int MODE>
+awq_status run_gemm_pair(const void* A, long long M, long long lda, const void* B, long long Nr, long long ldb,
+                         long long K, GemmArgs args, int tri, int num_sms, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, A, M, K, lda, 128)) return AWQ_ERR_CUDA;
+  if (!make_map(&tb, B, Nr, K, ldb, 128)) return AWQ_ERR_CUDA;
+  args.M = (int)M;
+  args.N = (int)Nr;
+  args.K = (int)K;
+  args.n_blocks_m = (int)cdiv(M, PAIR_BM);
+  args.n_blocks_n = (int)cdiv(Nr, PAIR_BN);
+  args.group_n = kGroupN < args.n_blocks_n ? kGroupN : args.n_blocks_n;
+  args.tri = tri;
+  const long long tiles = (long long)args.n_blocks_m * args.n_blocks_n;
+  if (tiles > INT32_MAX) return AWQ_ERR_SHAPE;
+  args.num_tiles = (int)tiles;
+  if (cudaFuncSetAttribute(gemm_pair_bf16_tcgen05<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           PAIR_SMEM_BYTES) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  if (cudaMemsetAsync(args.tile_counter, 0, sizeof(int), st) != cudaSuccess) return AWQ_ERR_CUDA;
+  const long long pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
+  gemm_pair_bf16_tcgen05<MODE><<<(unsigned)(2 * pairs), GEMM_THREADS, PAIR_SMEM_BYTES, st>>>(ta, tb, args);
+  return launch_status();
+}
+
+#ifndef AWQ_GEMM_PAIR
+#define AWQ_GEMM_PAIR 1
+#endif
+
 // Grid of a grid-stride kernel with 256-thread blocks: enough blocks for the
 // work, at most one wave of resident blocks.
 template <typename K>
@@ -356,9 +387,14 @@ awq_status launch_contract(const void* X, int64_t d_in, int64_t N, const SearchL
   ga.err = at<int>(ws, 0);
   ga.tile_counter = at<int>(ws, kTileCounterOffset);
   const __nv_bfloat16* dw = at<__nv_bfloat16>(ws, L.off_dw) + row0 * d_in;
-  if (L.form == AWQ_FORM_DIRECT) return run_gemm<EPI_SUMSQ>(dw, rows, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, st);
+  if (L.form == AWQ_FORM_DIRECT) {
+    if (AWQ_GEMM_PAIR) return run_gemm_pair<EPI_SUMSQ>(dw, rows, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, st);
+    return run_gemm<EPI_SUMSQ>(dw, rows, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, st);
+  }
   ga.E = dw;
   ga.ldE = d_in;
+  if (AWQ_GEMM_PAIR)
+    return run_gemm_pair<EPI_DOT>(dw, rows, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms, st);
   return run_gemm<EPI_DOT>(dw, rows, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms, st);
 }
 

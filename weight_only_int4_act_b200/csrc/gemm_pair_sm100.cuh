@@ -1,0 +1,294 @@
+// The loss contraction on CTA pairs (tcgen05 cta_group::2) for sm_100a.
+//
+// Same product and epilogues as gemm_sm100.cuh (EPI_SUMSQ, EPI_DOT; TRI_NONE
+// or TRI_K), but each 256 x 256 tile is computed by a cluster of two CTAs on
+// two SMs: CTA r of the pair loads rows [128 r, 128 r + 128) of the tile's A
+// panel and of its B panel (64-wide K stages, TMA, no multicast), and one
+// thread of the even CTA issues M=256 N=256 K=16 MMAs that read both CTAs'
+// shared memory and accumulate 128 rows x 256 columns in each CTA's TMEM.
+// Per SM and K step that is 32 KB of operand traffic instead of 48 KB for
+// the same MMA work.
+//
+// Coordination inside the pair:
+//   full[s]    even CTA only: armed by the even producer with both CTAs'
+//              bytes; both CTAs' TMA loads complete on it (cta_group::2 form);
+//   empty[s]   in each CTA, released by the MMA commit multicast to both;
+//   tfull[a]   in each CTA, MMA commit multicast to both;
+//   tempty[a]  even CTA only, 8 arrivals (the epilogue warps of both CTAs);
+//   tile ring  the even producer takes tile indices from the global counter,
+//              writes them into both CTAs' rings and arrives on both sfull;
+//              sempty (even CTA) counts 10 readers (even MMA + 4 even
+//              epilogue warps + odd producer + 4 odd epilogue warps).
+// All waits are bounded (ptx.cuh); the CTAs meet at a cluster barrier before
+// freeing TMEM (both CTAs, cta_group::2) and exiting.
+#pragma once
+#include "gemm_sm100.cuh"
+
+namespace awq {
+
+constexpr int PAIR_BM = 256;  // tile rows (128 per CTA)
+constexpr int PAIR_BN = 256;  // tile columns (B rows, 128 per CTA)
+constexpr int PAIR_BK = 64;
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_A_STAGE = 128 * PAIR_BK * 2;  // 16 KB per CTA
+constexpr int PAIR_B_STAGE = 128 * PAIR_BK * 2;  // 16 KB per CTA
+constexpr int PAIR_SLOTS = 4;
+constexpr int PAIR_SMEM_BYTES = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 512;
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+    gemm_pair_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + PAIR_STAGES * PAIR_A_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + PAIR_STAGES * PAIR_B_STAGE);
+  // full[S], empty[S], tfull[2], tempty[2], drain, sfull[R], sempty[R]
+  constexpr int NB = 2 * PAIR_STAGES + 5 + 2 * PAIR_SLOTS;
+  volatile int* tile_ring = reinterpret_cast<volatile int*>(bars + NB);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NB) + PAIR_SLOTS;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank() & 1u;
+  const bool even = rank == 0;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + PAIR_STAGES + s); };
+  auto tfull_bar = [&](int a) { return smem_u32(bars + 2 * PAIR_STAGES + a); };
+  auto tempty_bar = [&](int a) { return smem_u32(bars + 2 * PAIR_STAGES + 2 + a); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * PAIR_STAGES + 4);
+  auto sfull_bar = [&](int r) { return smem_u32(bars + 2 * PAIR_STAGES + 5 + r); };
+  auto sempty_bar = [&](int r) { return smem_u32(bars + 2 * PAIR_STAGES + 5 + PAIR_SLOTS + r); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PAIR_STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 8);
+    }
+    mbar_init(drain_bar, 1);
+    for (int r = 0; r < PAIR_SLOTS; ++r) {
+      mbar_init(sfull_bar(r), 1);
+      mbar_init(sempty_bar(r), 10);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), GEMM_TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = args.num_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- tile scheduler (even CTA) + TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, last_parity = 0;
+      int slot = 0;
+      uint32_t sphase = 0;
+      bool ok = true;
+      while (ok) {
+        int t;
+        if (even) {
+          if (!mbar_wait(sempty_bar(slot), sphase ^ 1u, abort_flag, args.err, ERR_WAIT_SCHED)) break;
+          t = atomicAdd(args.tile_counter, 1);
+          if (t >= num_tiles) t = -1;
+          tile_ring[slot] = t;
+          st_shared_remote(mapa_shared(smem_u32((const void*)(tile_ring + slot)), 1), t);
+          mbar_arrive(sfull_bar(slot));
+          mbar_arrive_remote(mapa_shared(sfull_bar(slot), 1));
+        } else {
+          if (!mbar_wait(sfull_bar(slot), sphase, abort_flag, args.err, ERR_WAIT_SCHED)) break;
+          t = tile_ring[slot];
+          mbar_arrive_remote(mapa_shared(sempty_bar(slot), 0));
+        }
+        if (++slot == PAIR_SLOTS) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+        if (t < 0) break;
+        int mb, nb;
+        gemm_tile_coords(t, args, mb, nb);
+        const int num_kb = gemm_num_kb(args, nb);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.err, ERR_WAIT_EMPTY)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_even = mapa_shared(full_bar(stage), 0);
+          if (even) mbar_arrive_expect_tx(full_bar(stage), 2 * (PAIR_A_STAGE + PAIR_B_STAGE));
+          tma_load_2d_pair(smem_u32(sA + stage * PAIR_A_STAGE), &tmA, full_even, kb * PAIR_BK,
+                           mb * PAIR_BM + (int)rank * 128);
+          tma_load_2d_pair(smem_u32(sB + stage * PAIR_B_STAGE), &tmB, full_even, kb * PAIR_BK,
+                           nb * PAIR_BN + (int)rank * 128);
+          issued |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == PAIR_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (even) {
+        // loads land on the even CTA's full barriers: wait for every armed one
+        for (int s = 0; s < PAIR_STAGES; ++s)
+          if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (last_parity >> s) & 1u);
+      } else if (*abort_flag) {
+        // on an aborted run, give this CTA's unconsumed loads time to land
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && even) {
+      // ---------------- MMA issuer (even CTA)
+      constexpr uint32_t IDESC = idesc_bf16_f32(PAIR_BM, PAIR_BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int slot = 0;
+      uint32_t sphase = 0;
+      bool ok = true;
+      for (int local = 0; ok; ++local) {
+        if (!mbar_wait(sfull_bar(slot), sphase, abort_flag, args.err, ERR_WAIT_SCHED)) break;
+        const int t = tile_ring[slot];
+        mbar_arrive(sempty_bar(slot));
+        if (++slot == PAIR_SLOTS) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+        if (t < 0) break;
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.err, ERR_WAIT_TEMPTY)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * PAIR_BN;
+        int mb, nb;
+        gemm_tile_coords(t, args, mb, nb);
+        const int num_kb = gemm_num_kb(args, nb);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, args.err, ERR_WAIT_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * PAIR_A_STAGE);
+          const uint32_t b_base = smem_u32(sB + stage * PAIR_B_STAGE);
+#pragma unroll
+          for (int k = 0; k < PAIR_BK / 16; ++k)
+            mma_bf16_pair(d_tmem, desc_kmajor_sw128(a_base + k * 32), desc_kmajor_sw128(b_base + k * 32), IDESC,
+                          (kb | k) != 0);
+          mma_commit_pair(empty_bar(stage), 0x3);
+          if (++stage == PAIR_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) mma_commit_pair(tfull_bar(acc), 0x3);
+      }
+      mma_commit_pair(drain_bar, 0x1);
+      mbar_wait_drain(drain_bar, 0);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 of both CTAs)
+    const int quad = warp & 3;
+    const int row_in_tile = quad * 32 + lane;
+    int slot = 0;
+    uint32_t sphase = 0;
+    for (int local = 0;; ++local) {
+      const bool have = mbar_wait(sfull_bar(slot), sphase, abort_flag, args.err, ERR_WAIT_SCHED);
+      if (!__all_sync(0xffffffffu, have)) break;
+      const int t = tile_ring[slot];
+      __syncwarp();
+      if (lane == 0) {
+        if (even)
+          mbar_arrive(sempty_bar(slot));
+        else
+          mbar_arrive_remote(mapa_shared(sempty_bar(slot), 0));
+      }
+      if (++slot == PAIR_SLOTS) {
+        slot = 0;
+        sphase ^= 1u;
+      }
+      if (t < 0) break;
+      int mb, nb;
+      gemm_tile_coords(t, args, mb, nb);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      const bool ready = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, args.err, ERR_WAIT_TFULL);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * PAIR_BN;
+      const int m = mb * PAIR_BM + (int)rank * 128 + row_in_tile;
+      const int n0 = nb * PAIR_BN;
+      float sum = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < PAIR_BN / 32; ++c) {
+        uint4 e[4];
+        if constexpr (MODE == EPI_DOT) {
+          const int col = n0 + c * 32;
+          const __nv_bfloat16* erow = args.E + (long long)m * args.ldE + col;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            e[v] = (m < args.M && col + v * 8 < args.N) ? __ldg(reinterpret_cast<const uint4*>(erow + v * 8))
+                                                         : make_uint4(0, 0, 0, 0);
+        }
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c * 32, r);
+        tmem_ld_wait();
+        if constexpr (MODE == EPI_SUMSQ) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float d = __uint_as_float(r[j]);
+            sum = fmaf(d, d, sum);
+          }
+        } else {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint32_t ew[4] = {e[v].x, e[v].y, e[v].z, e[v].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              sum = fmaf(__uint_as_float(r[v * 8 + 2 * h]), bf16lo(ew[h]), sum);
+              sum = fmaf(__uint_as_float(r[v * 8 + 2 * h + 1]), bf16hi(ew[h]), sum);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (even)
+          mbar_arrive(tempty_bar(acc));
+        else
+          mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
+      }
+      if (m < args.M) args.part[(long long)nb * args.part_ld + m] = sum;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // all MMAs drained, all TMEM reads and remote arrivals done in both CTAs
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, GEMM_TMEM_COLS);
+  }
+}
+
+}  // namespace awq
