@@ -50,7 +50,7 @@ def load_peaks():
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("gemm_sm100.cuh", "ptx.cuh"):
+    for f in ("gemm_pair_sm100.cuh", "gemm_sm100.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "weight_only_int4_act_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -331,8 +331,8 @@ def run_ours(args, rank, world, local_rank):
                    "group": wl.group, "symmetric": wl.symmetric, "n_alpha": n_a, "form": form,
                    "l2": "flushed: 256 MiB write between timed steps, outside the step events",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "roofline": {"kernel": "gemm_bf16_tcgen05 " + ("(direct, sum-of-squares epilogue)" if form == "direct"
-                                                     else "(block-triangular Gram, dot epilogue)"),
+        "roofline": {"kernel": "gemm_pair_bf16_tcgen05 (CTA pairs, " + ("direct, sum-of-squares epilogue)" if form == "direct"
+                                                                 else "block-triangular Gram, dot epilogue)"),
                      "bound": "tensor", "achieved": round(achieved_tflops, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
                      "peak_kind": f"bf16 dense burst ({peaks.get('source')})",

@@ -29,11 +29,15 @@ namespace awq {
 constexpr int PAIR_BM = 256;  // tile rows (128 per CTA)
 constexpr int PAIR_BN = 256;  // tile columns (B rows, 128 per CTA)
 constexpr int PAIR_BK = 64;
-constexpr int PAIR_STAGES = 6;
+#ifndef AWQ_PAIR_STAGES
+#define AWQ_PAIR_STAGES 6
+#endif
+constexpr int PAIR_STAGES = AWQ_PAIR_STAGES;
 constexpr int PAIR_A_STAGE = 128 * PAIR_BK * 2;  // 16 KB per CTA
 constexpr int PAIR_B_STAGE = 128 * PAIR_BK * 2;  // 16 KB per CTA
 constexpr int PAIR_SLOTS = 4;
 constexpr int PAIR_SMEM_BYTES = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 512;
+static_assert(PAIR_SMEM_BYTES <= 232448, "shared memory per CTA");
 
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
