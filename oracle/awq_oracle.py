@@ -96,7 +96,7 @@ def candidate_scales(a: np.ndarray, alpha: float, eps_a: float = EPS_A,
 # step a3: group-wise quantiser and fake quantisation
 # ---------------------------------------------------------------------------
 def quantize_groups(V: np.ndarray, bits: int, group: int, symmetric: bool,
-                    eps_delta: float = EPS_DELTA):
+                    eps_delta: float = EPS_DELTA, clip: float = 1.0):
     """Uniform group-wise quantisation of V[rows, d_in] along d_in.
 
     Returns (V_hat, codes, delta, zero): V_hat the dequantised values, codes
@@ -117,6 +117,13 @@ def quantize_groups(V: np.ndarray, bits: int, group: int, symmetric: bool,
         v_hat = (q_i - z) * Delta.
     rne = round half to even ([P5] §2.3 "round"; the demo's np.round is
     half-to-even too).
+
+    Clipping ([P5] 参考资料 note: the practical algorithm searches a restricted
+    parameterisation "possibly combined with clipping"; the pages give no
+    formula): with clip ratio c in (0, 1], the group's range is shrunk before
+    the step is taken — max|v| -> c max|v| (symmetric), max v -> c max v and
+    min v -> c min v (asymmetric) — and values outside the shrunk range clip to
+    the extreme codes. c = 1 is the plain quantiser.
     """
     V = np.asarray(V, dtype=np.float64)
     rows, d_in = V.shape
@@ -126,15 +133,15 @@ def quantize_groups(V: np.ndarray, bits: int, group: int, symmetric: bool,
     if symmetric:
         qmax = 2 ** (bits - 1) - 1
         qmin = -(2 ** (bits - 1))
-        delta = np.maximum(np.abs(G).max(axis=-1), eps_delta) / qmax
+        delta = np.maximum(clip * np.abs(G).max(axis=-1), eps_delta) / qmax
         q = np.clip(np.rint(G / delta[..., None]), qmin, qmax)
         Vh = q * delta[..., None]
         codes = (q - qmin).astype(np.int64)
         zero = np.full(delta.shape, float(-qmin))
     else:
         levels = 2 ** bits - 1
-        mx = G.max(axis=-1)
-        mn = G.min(axis=-1)
+        mx = clip * G.max(axis=-1)
+        mn = clip * G.min(axis=-1)
         delta = np.maximum(mx - mn, eps_delta) / levels
         zero = np.clip(np.rint(-mn / delta), 0, levels)
         q = np.clip(np.rint(G / delta[..., None]) + zero[..., None], 0, levels)
@@ -143,7 +150,7 @@ def quantize_groups(V: np.ndarray, bits: int, group: int, symmetric: bool,
     return Vh.reshape(rows, d_in), codes.reshape(rows, d_in), delta, zero
 
 
-def fake_quant(W: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool):
+def fake_quant(W: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool, clip: float = 1.0):
     """W_hat = Q(W S) S^-1 for W[rows, d_in] (float64) and scales s[d_in].
 
     [P1] 缩放保护: W~_i = s_i W_i, W^_i = Q(W~_i) / s_i; [P5] §2.2: Q(WS)S^-1.
@@ -151,13 +158,14 @@ def fake_quant(W: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: b
     """
     s = np.asarray(s, dtype=np.float64)
     V = W * s[None, :]
-    Vh, codes, delta, zero = quantize_groups(V, bits, group, symmetric)
+    Vh, codes, delta, zero = quantize_groups(V, bits, group, symmetric, clip=clip)
     return Vh / s[None, :], codes, delta, zero
 
 
-def delta_weight(W: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool) -> np.ndarray:
+def delta_weight(W: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool,
+                 clip: float = 1.0) -> np.ndarray:
     """Delta W = Q(W S) S^-1 - W, formed before any contraction."""
-    What = fake_quant(W, s, bits, group, symmetric)[0]
+    What = fake_quant(W, s, bits, group, symmetric, clip)[0]
     return What - W
 
 
@@ -249,6 +257,26 @@ def search(W_bits: np.ndarray, X_bits: np.ndarray, a: np.ndarray, bits: int, gro
                 alphas=alphas, row_losses=per_row if rows is not None else None)
 
 
+def search_candidates(W_bits: np.ndarray, X_bits: np.ndarray, s_cand: np.ndarray, bits: int, group: int,
+                      symmetric: bool, clips=None, form: str = "direct", G: np.ndarray | None = None):
+    """Loss of arbitrary candidates: candidate k uses scales s_cand[k] and clip
+    ratio clips[k] (default 1); L_k = ||(Q(W S_k) S_k^-1 - W) X^T||_F^2 and the
+    lowest-index argmin, as in search(). Covers the clipping search (the same s
+    with several clip ratios) and other candidate sets (e.g. a salience mask
+    with a fixed scale factor, [P1] 显著识别 and its Python demo)."""
+    W = widen_bf16(W_bits)
+    s_cand = np.atleast_2d(np.asarray(s_cand, dtype=np.float64))
+    n = s_cand.shape[0]
+    clips = np.ones(n) if clips is None else np.asarray(clips, dtype=np.float64)
+    if form == "gram" and G is None:
+        G = gram(X_bits)
+    losses = np.zeros(n)
+    for k in range(n):
+        dW = delta_weight(W, s_cand[k], bits, group, symmetric, clips[k])
+        losses[k] = (row_losses_gram(dW, G) if form == "gram" else row_losses_direct(dW, X_bits)).sum()
+    return dict(losses=losses, best=choose(losses))
+
+
 def choose(losses: np.ndarray) -> int:
     """argmin over the grid; the lowest index among exact ties."""
     losses = np.asarray(losses, dtype=np.float64)
@@ -289,7 +317,7 @@ def to_fp16(x: np.ndarray) -> np.ndarray:
     return np.asarray(x, dtype=np.float64).astype(np.float16)
 
 
-def pack(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool):
+def pack(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool, clip: float = 1.0):
     """Codes of Q(W S) at the chosen scales, packed; fp16 step and zero point.
 
     Returns (qweight uint32[rows, d_in/8], scales fp16[rows, d_in/g],
@@ -298,12 +326,12 @@ def pack(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bo
     rounded to fp16 (reading: the pages give an fp16 scale, [P2] §2.1).
     """
     W = widen_bf16(W_bits)
-    _, codes, delta, zero = fake_quant(W, s, bits, group, symmetric)
+    _, codes, delta, zero = fake_quant(W, s, bits, group, symmetric, clip)
     return pack_codes(codes), to_fp16(delta), to_fp16(zero), codes, delta, zero
 
 
 def boundary_mask(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool,
-                  band: float = 1e-4) -> np.ndarray:
+                  band: float = 1e-4, clip: float = 1.0) -> np.ndarray:
     """Elements whose code the float64 oracle decides within ``band`` of a
     rounding boundary: v/Delta (or -min/Delta for the zero point of the
     element's group) lies within ``band`` of a half-integer. A float32
@@ -313,11 +341,11 @@ def boundary_mask(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symm
     rows, d_in = V.shape
     G = V.reshape(rows, d_in // group, group)
     if symmetric:
-        delta = np.maximum(np.abs(G).max(axis=-1), EPS_DELTA) / (2 ** (bits - 1) - 1)
+        delta = np.maximum(clip * np.abs(G).max(axis=-1), EPS_DELTA) / (2 ** (bits - 1) - 1)
         r = G / delta[..., None]
         near = np.abs(r - np.floor(r) - 0.5) < band
     else:
-        mx, mn = G.max(axis=-1), G.min(axis=-1)
+        mx, mn = clip * G.max(axis=-1), clip * G.min(axis=-1)
         delta = np.maximum(mx - mn, EPS_DELTA) / (2 ** bits - 1)
         r = G / delta[..., None]
         near = np.abs(r - np.floor(r) - 0.5) < band

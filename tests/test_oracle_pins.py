@@ -442,3 +442,61 @@ def test_pack_layer_consistency():
     ref = O.fake_quant(O.widen_bf16(W), s, 4, 128, False)[0] * s
     assert np.allclose(Vh, ref, rtol=1e-14, atol=1e-18)
     assert np.array_equal(zr.astype(np.float64), zero)
+
+
+# ---------------------------------------------------------------------------
+# clipping and arbitrary candidates
+# ---------------------------------------------------------------------------
+def test_clip_one_is_plain_quantiser():
+    rng = np.random.default_rng(20)
+    V = rng.standard_normal((50, 128))
+    for sym in (False, True):
+        a = O.quantize_groups(V, 4, 128, sym)
+        b = O.quantize_groups(V, 4, 128, sym, clip=1.0)
+        assert all(np.array_equal(x, y) for x, y in zip(a, b))
+
+
+def test_clip_closed_forms():
+    """With ratio c the step is c*range/(2^b-1) (asymmetric) or
+    c*max|v|/(2^(b-1)-1) (symmetric), and values beyond the shrunk range take
+    the extreme codes."""
+    V = np.array([[-1.0, -0.2, 0.1, 0.4, 2.0, 0.0, 0.3, -0.5]])
+    _, codes, delta, zero = O.quantize_groups(V, 4, 8, False, clip=0.5)
+    assert delta[0, 0] == pytest.approx(0.5 * 3.0 / 15.0)
+    assert zero[0, 0] == np.rint(0.5 / delta[0, 0])       # -min' / Delta = 0.5 / 0.1 = 5
+    assert codes[0, 4] == 15 and codes[0, 0] == 0           # 2.0 > 1.0 = max', -1.0 < -0.5 = min'
+    _, codes, delta, _ = O.quantize_groups(V, 4, 8, True, clip=0.25)
+    assert delta[0, 0] == pytest.approx(0.25 * 2.0 / 7.0)
+    assert codes[0, 4] == 15 and codes[0, 0] == 0           # 2.0 and -1.0 clip to q = 7 and q = -8
+
+
+def test_clip_brute_force_codes():
+    """Clipped codes are the nearest dequantised grid points (exact ties excluded)."""
+    rng = np.random.default_rng(21)
+    V = rng.standard_normal((200, 16))
+    for sym, bits in ((False, 4), (True, 3)):
+        Vh, codes, delta, zero = O.quantize_groups(V, bits, 16, sym, clip=0.7)
+        n = 2 ** bits
+        for r in range(V.shape[0]):
+            offs = 2 ** (bits - 1) if sym else zero[r, 0]
+            cands = (np.arange(n) - offs) * delta[r, 0]
+            for i in range(16):
+                dist = np.abs(cands - V[r, i])
+                o = np.argsort(dist)
+                if dist[o[1]] - dist[o[0]] < 1e-12:
+                    continue
+                assert codes[r, i] == o[0]
+
+
+def test_search_candidates_matches_search():
+    """The alpha grid given as explicit candidates reproduces search()."""
+    W, X = make_inputs(WORKLOADS["C1"])
+    a = O.act_stats(X)
+    ref = O.search(W, X, a, 4, 128, False, 5)
+    s_cand = np.stack([O.candidate_scales(a, al) for al in O.alpha_grid(5)])
+    got = O.search_candidates(W, X, s_cand, 4, 128, False)
+    assert np.allclose(got["losses"], ref["losses"], rtol=1e-14) and got["best"] == ref["best"]
+    # clip ratio 1 changes nothing; clipping a lot increases the loss
+    clipped = O.search_candidates(W, X, np.stack([s_cand[2]] * 3), 4, 128, False, clips=[1.0, 0.9, 0.3])
+    assert clipped["losses"][0] == pytest.approx(ref["losses"][2], rel=1e-14)
+    assert clipped["losses"][2] > clipped["losses"][0]
