@@ -173,6 +173,32 @@ awq_status awq_quantize_pack(const void* W_bf16, const float* s, int64_t d_out, 
                              const awq_qcfg* cfg, uint32_t* qweight, void* scales_f16, void* zeros_f16,
                              awq_stream_t stream);
 
+/* Pack with a clip ratio clip in (0, 1]: each group's range is shrunk by clip
+ * before the step is taken (symmetric: c max|v|; asymmetric: c max v and
+ * c min v) and values beyond it take the extreme codes. clip = 1 is
+ * awq_quantize_pack. AWQ_ERR_INVALID_ARG for clip outside (0, 1]. */
+awq_status awq_quantize_pack_clipped(const void* W_bf16, const float* s, int64_t d_out, int64_t d_in,
+                                     const awq_qcfg* cfg, float clip, uint32_t* qweight, void* scales_f16,
+                                     void* zeros_f16, awq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * The search over caller-given candidates instead of the a^alpha grid
+ * ([P5] 参考资料: the practical algorithm searches a restricted
+ * parameterisation of the scales, possibly combined with clipping).
+ * Candidate k uses the scale vector s_cand[k] (DEVICE float [n, d_in], every
+ * entry > 0) and the clip ratio clips[k] (HOST float [n] in (0, 1], or NULL
+ * for no clipping), n = cfg->n_alpha (cfg->alphas is ignored). For example:
+ * the clipping search is n copies of s_best with a grid of clip ratios; a
+ * salience mask ([P1] 显著识别) is s_i = factor on the channels above a
+ * percentile of a and 1 elsewhere. Outputs as in awq_search_scales, with
+ * s_best = the chosen candidate's scales; a non-positive scale is recorded as
+ * AWQ_ERR_NONFINITE. Workspace: awq_search_workspace_size.
+ * ------------------------------------------------------------------------- */
+awq_status awq_search_candidates(const void* W_bf16, const void* X_bf16, const float* s_cand, const float* clips,
+                                 int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                                 size_t ws_bytes, float* losses, int32_t* best, float* s_best, float* row_losses,
+                                 awq_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * The search, one step at a time (awq_search_scales is exactly these calls
  * in this order). They share the search workspace; offsets are internal.

@@ -1,6 +1,6 @@
 """AWQ calibration and scale search on B200 (sm_100a): a C-ABI CUDA library
 (include/awq.h) and its Python binding."""
 from .binding import (  # noqa: F401
-    AwqError, QCfg, make_cfg, lib, act_stats, search_scales, search_scales_segmented, quantize_pack, workspace_error,
+    AwqError, QCfg, make_cfg, lib, act_stats, search_scales, search_scales_segmented, search_candidates, quantize_pack, workspace_error,
     stats_workspace_size, search_workspace_size, search_form, workspace, debug_dw, step, status_str,
 )

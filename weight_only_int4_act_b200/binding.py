@@ -24,7 +24,8 @@ EXPORTED = (
     "awq_status_str", "awq_stats_workspace_size", "awq_act_stats", "awq_search_workspace_size",
     "awq_search_scales", "awq_search_form", "awq_workspace_error", "awq_quantize_pack",
     "awq_step_scales", "awq_step_fake_quant", "awq_step_gram", "awq_step_contract", "awq_step_reduce",
-    "awq_debug_copy_dw", "awq_act_stats_noalloc", "awq_search_scales_segmented",
+    "awq_debug_copy_dw", "awq_act_stats_noalloc", "awq_search_scales_segmented", "awq_search_candidates",
+    "awq_quantize_pack_clipped",
 )
 
 
@@ -73,6 +74,11 @@ def lib() -> ctypes.CDLL:
             "awq_search_scales_segmented": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, cfgp,
                                                       c_int32, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p,
                                                       c_void_p, c_void_p, c_void_p]),
+            "awq_search_candidates": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64,
+                                                cfgp, c_void_p, c_size_t, c_void_p, c_void_p, c_void_p, c_void_p,
+                                                c_void_p]),
+            "awq_quantize_pack_clipped": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_float, c_void_p,
+                                                    c_void_p, c_void_p, c_void_p]),
             "awq_workspace_error": (c_int32, [c_void_p, c_void_p]),
             "awq_quantize_pack": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_void_p, c_void_p,
                                             c_void_p, c_void_p]),
@@ -220,6 +226,34 @@ def search_scales_segmented(W, X, a, cfg: QCfg, seg_rows, ws=None, row_losses=Fa
     return dict(o, ws=ws)
 
 
+def search_candidates(W, X, s_cand, cfg: QCfg, clips=None, ws=None, row_losses=False):
+    """Losses of explicit candidates: scale vectors s_cand float32 [n, d_in] (CUDA)
+    and optional clip ratios (host sequence of n floats in (0, 1]); n must equal
+    cfg.n_alpha. Returns dict(losses, best, s_best, row_losses, ws)."""
+    torch = _torch()
+    _req(W, torch.bfloat16, None, "W")
+    d_out, d_in = W.shape
+    _req(X, torch.bfloat16, None, "X")
+    N = X.shape[0]
+    _req(s_cand, torch.float32, (cfg.n_alpha, d_in), "s_cand")
+    carr = None
+    if clips is not None:
+        if len(clips) != cfg.n_alpha:
+            raise ValueError("need one clip ratio per candidate")
+        carr = (c_float * len(clips))(*[float(c) for c in clips])
+    if ws is None:
+        ws = workspace(search_workspace_size(d_out, d_in, N, cfg))
+    o = dict(losses=torch.empty(cfg.n_alpha, dtype=torch.float32, device=W.device),
+             best=torch.empty(1, dtype=torch.int32, device=W.device),
+             s_best=torch.empty(d_in, dtype=torch.float32, device=W.device),
+             row_losses=torch.empty((cfg.n_alpha, d_out), dtype=torch.float32, device=W.device) if row_losses else None)
+    _check(lib().awq_search_candidates(_ptr(W), _ptr(X), _ptr(s_cand), ctypes.cast(carr, c_void_p) if carr else None,
+                                       d_out, d_in, N, ctypes.byref(cfg), _ptr(ws), ws.numel(), _ptr(o["losses"]),
+                                       _ptr(o["best"]), _ptr(o["s_best"]), _ptr(o["row_losses"]), _stream()),
+           "awq_search_candidates")
+    return dict(o, ws=ws)
+
+
 def workspace_error(ws):
     """Raise AwqError if a kernel recorded an error in the workspace (synchronises)."""
     _check(lib().awq_workspace_error(_ptr(ws), _stream()), "device")
@@ -241,7 +275,7 @@ def debug_dw(ws, d_out, d_in, N, cfg, k):
 
 
 # --------------------------------------------------------------------------- a7
-def quantize_pack(W, s, cfg: QCfg, outputs=None):
+def quantize_pack(W, s, cfg: QCfg, outputs=None, clip=1.0):
     """(qweight int32 view of uint32 [d_out, d_in/8], scales fp16 [d_out, d_in/g], zeros fp16 [d_out, d_in/g])."""
     torch = _torch()
     _req(W, torch.bfloat16, None, "W")
@@ -253,6 +287,10 @@ def quantize_pack(W, s, cfg: QCfg, outputs=None):
                    torch.empty((d_out, ng), dtype=torch.float16, device=W.device),
                    torch.empty((d_out, ng), dtype=torch.float16, device=W.device))
     q, sc, zr = outputs
-    _check(lib().awq_quantize_pack(_ptr(W), _ptr(s), d_out, d_in, ctypes.byref(cfg), _ptr(q), _ptr(sc), _ptr(zr),
-                                   _stream()), "awq_quantize_pack")
+    if clip == 1.0:
+        _check(lib().awq_quantize_pack(_ptr(W), _ptr(s), d_out, d_in, ctypes.byref(cfg), _ptr(q), _ptr(sc), _ptr(zr),
+                                       _stream()), "awq_quantize_pack")
+    else:
+        _check(lib().awq_quantize_pack_clipped(_ptr(W), _ptr(s), d_out, d_in, ctypes.byref(cfg), float(clip), _ptr(q),
+                                               _ptr(sc), _ptr(zr), _stream()), "awq_quantize_pack_clipped")
     return q, sc, zr

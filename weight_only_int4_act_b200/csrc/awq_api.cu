@@ -351,7 +351,12 @@ awq_status awq_step_scales(const float* a, int64_t d_out, int64_t d_in, int64_t 
 // Fake quantisation of grid points [k0, k1) into their slices of the dW stack.
 // max_per_sm > 0 caps the grid at that many blocks per SM.
 awq_status launch_fake_quant(const void* W, int64_t d_out, int64_t d_in, const awq_qcfg* cfg, const SearchLayout& L,
-                             void* ws, int k0, int k1, int sms, int max_per_sm, cudaStream_t st) {
+                             void* ws, int k0, int k1, int sms, int max_per_sm, cudaStream_t st,
+                             const ClipTable* clip_table = nullptr) {
+  ClipTable clips;
+  for (int k = 0; k < MAX_ALPHA; ++k) clips.c[k] = 1.0f;
+  if (clip_table)
+    for (int k = k0; k < k1; ++k) clips.c[k - k0] = clip_table->c[k];
   const long long slice = (long long)L.d_out_pad * d_in;
   auto launch = [&](auto kernel, int cpt) {
     const long long units = (long long)(L.d_out_pad / FQ_ROWS) * (d_in / cpt);
@@ -360,7 +365,7 @@ awq_status launch_fake_quant(const void* W, int64_t d_out, int64_t d_in, const a
     kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in, L.d_out_pad,
                                  at<float>(ws, L.off_s) + (long long)k0 * d_in,
                                  at<float>(ws, L.off_inv) + (long long)k0 * d_in, k1 - k0, cfg->bits,
-                                 cfg->symmetric, at<__nv_bfloat16>(ws, L.off_dw) + k0 * slice);
+                                 cfg->symmetric, at<__nv_bfloat16>(ws, L.off_dw) + k0 * slice, clips);
   };
   constexpr int C = FQ_CPT;
   switch (cfg->group) {
@@ -515,11 +520,12 @@ awq_status awq_workspace_error(void* ws, awq_stream_t stream) {
   return word == ERR_NONFINITE ? AWQ_ERR_NONFINITE : AWQ_ERR_DEVICE;
 }
 
-awq_status awq_quantize_pack(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
-                             uint32_t* qweight, void* scales, void* zeros, awq_stream_t stream) {
+awq_status awq_quantize_pack_clipped(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
+                                     float clip, uint32_t* qweight, void* scales, void* zeros, awq_stream_t stream) {
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if ((st = check_layer_shape(d_out, d_in, cfg)) != AWQ_OK) return st;
+  if (!(clip > 0.f && clip <= 1.f)) return AWQ_ERR_INVALID_ARG;
   if (!W || !s || !qweight || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
   if (!aligned(W, 16) || !aligned(s, 16) || !aligned(qweight, 4) || !aligned(scales, 2) || !aligned(zeros, 2))
     return AWQ_ERR_INVALID_ARG;
@@ -530,7 +536,7 @@ awq_status awq_quantize_pack(const void* W, const float* s, int64_t d_out, int64
     const int grid = elementwise_grid(kernel, units, sms);
     kernel<<<grid, 256, 0, as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(W), s, (int)d_out, (int)d_in,
                                                 cfg->bits, cfg->symmetric, qweight, static_cast<__half*>(scales),
-                                                static_cast<__half*>(zeros));
+                                                static_cast<__half*>(zeros), clip);
   };
   constexpr int C = FQ_CPT;
   switch (cfg->group) {
@@ -543,6 +549,41 @@ awq_status awq_quantize_pack(const void* W, const float* s, int64_t d_out, int64
     default: return AWQ_ERR_INVALID_ARG;
   }
   return launch_status();
+}
+
+awq_status awq_quantize_pack(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
+                             uint32_t* qweight, void* scales, void* zeros, awq_stream_t stream) {
+  return awq_quantize_pack_clipped(W, s, d_out, d_in, cfg, 1.0f, qweight, scales, zeros, stream);
+}
+
+awq_status awq_search_candidates(const void* W, const void* X, const float* s_cand, const float* clips,
+                                 int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                                 size_t ws_bytes, float* losses, int32_t* best, float* s_best, float* row_losses,
+                                 awq_stream_t stream) {
+  SearchLayout L;
+  awq_status st = check_search_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  if (!W || !X || !s_cand || !losses || !best || !s_best) return AWQ_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
+  ClipTable table;
+  for (int k = 0; k < MAX_ALPHA; ++k) table.c[k] = 1.0f;
+  if (clips)
+    for (int k = 0; k < cfg->n_alpha; ++k) {
+      if (!(clips[k] > 0.f && clips[k] <= 1.f)) return AWQ_ERR_INVALID_ARG;
+      table.c[k] = clips[k];
+    }
+  int sms = 0;
+  if ((st = check_device(&sms)) != AWQ_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return AWQ_ERR_CUDA;
+  const long long n = (long long)cfg->n_alpha * d_in;
+  set_candidate_scales<<<(unsigned)(cdiv(n, 256) < 4 * sms ? cdiv(n, 256) : 4 * sms), 256, 0, s>>>(
+      s_cand, n, at<float>(ws, L.off_s), at<float>(ws, L.off_inv), at<int>(ws, 0));
+  if ((st = launch_status()) != AWQ_OK) return st;
+  if ((st = launch_fake_quant(W, d_out, d_in, cfg, L, ws, 0, cfg->n_alpha, sms, 0, s, &table)) != AWQ_OK) return st;
+  if ((st = awq_step_gram(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  if ((st = awq_step_contract(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
+  return awq_step_reduce(d_out, d_in, N, cfg, ws, ws_bytes, losses, best, s_best, row_losses, stream);
 }
 
 awq_status awq_debug_copy_dw(const void* ws, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, int32_t k,

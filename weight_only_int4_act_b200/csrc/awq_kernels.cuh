@@ -135,6 +135,18 @@ __global__ void candidate_scales(const float* __restrict__ a, int d_in, AlphaGri
   }
 }
 
+// Candidate scales given by the caller: s_all = s_cand, inv_all = 1 / s_cand;
+// a non-positive or non-finite scale is recorded as a non-finite error.
+__global__ void set_candidate_scales(const float* __restrict__ s_cand, long long n, float* __restrict__ s_all,
+                                     float* __restrict__ inv_all, int* err) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = s_cand[i];
+    if (!(v > 0.f) || !isfinite(v)) atomicCAS(err, 0, ERR_NONFINITE);
+    s_all[i] = v;
+    inv_all[i] = 1.0f / v;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // a3: dW[k][r][:] = Q(W_r S_k) S_k^-1 - W_r as bf16, for every alpha k.
 // ([P1] 缩放保护 W~ = sW, W^ = Q(W~)/s; [P5] §2.2 Q(WS)S^-1.)
@@ -164,11 +176,16 @@ __device__ __forceinline__ void load_f32(const float* __restrict__ p, float (&f)
   }
 }
 
+struct ClipTable {
+  float c[MAX_ALPHA];  // clip ratio of each candidate (1: none)
+};
+
 template <int CPT, int ROWS, int GL>
 __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* __restrict__ W, int d_out, int d_in,
                                                            int d_out_pad, const float* __restrict__ s_all,
                                                            const float* __restrict__ inv_all, int n_alpha, int bits,
-                                                           int symmetric, __nv_bfloat16* __restrict__ dW) {
+                                                           int symmetric, __nv_bfloat16* __restrict__ dW,
+                                                           ClipTable clips) {
   const int chunks = d_in / CPT;
   const long long total = (long long)(d_out_pad / ROWS) * chunks;
   const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -207,7 +224,7 @@ __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* 
 #pragma unroll
         for (int j = 0; j < CPT; ++j) v[j] = w[r][j] * s[j];
         FqGroup<CPT> fr;
-        fq_group<CPT, GL>(v, bits, sym, fr);
+        fq_group<CPT, GL>(v, bits, sym, fr, clips.c[k]);
 #pragma unroll
         for (int q = 0; q < CPT / 8; ++q) {
           uint32_t out[4];
@@ -395,7 +412,7 @@ template <int CPT, int GL>
 __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __restrict__ W, const float* __restrict__ s,
                                                      int d_out, int d_in, int bits, int symmetric,
                                                      uint32_t* __restrict__ qweight, __half* __restrict__ scales,
-                                                     __half* __restrict__ zeros) {
+                                                     __half* __restrict__ zeros, float clip) {
   const int chunks = d_in / CPT;
   const int row_groups = (d_out + PACK_ROWS - 1) / PACK_ROWS;
   const long long total = (long long)row_groups * chunks;
@@ -433,7 +450,7 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
         for (int j = 0; j < 8; ++j) v[8 * q + j] = f[j] * sc[8 * q + j];
       }
       FqGroup<CPT> fr;
-      fq_group<CPT, GL>(v, bits, sym, fr);
+      fq_group<CPT, GL>(v, bits, sym, fr, clip);
       if (active && row0 + r < d_out) {
         const int row = row0 + r;
         uint32_t* wp = qweight + (long long)row * words + c0 / 8;

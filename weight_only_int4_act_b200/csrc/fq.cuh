@@ -102,13 +102,15 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
 // and fma(y, span, 1.5*2^23) rounds y * span to the nearest integer (ties to
 // even) in magic form. This equals clamp(rne(v / Delta) + z, 0, span) except
 // where v / Delta lies within ~1e-6 of a rounding boundary.
+// clip in (0, 1] shrinks the group's range before the step is taken (1: none).
 template <int CPT, int GL>
-__device__ __forceinline__ void fq_group(const float (&v)[CPT], int bits, bool symmetric, FqGroup<CPT>& r) {
+__device__ __forceinline__ void fq_group(const float (&v)[CPT], int bits, bool symmetric, FqGroup<CPT>& r,
+                                         float clip = 1.0f) {
   const float span = (float)((1 << bits) - 1);
   const float inv_span = inv_levels(bits);
   float a, b;  // y = sat(v * a + b)
   if (symmetric) {
-    const float amax = group_max<GL>(fmaxf(maxN(v), -minN(v)));
+    const float amax = clip * group_max<GL>(fmaxf(maxN(v), -minN(v)));
     const float half = (float)(1 << (bits - 1));  // -qmin
     r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
     const float inv = __frcp_rn(r.delta);
@@ -117,8 +119,8 @@ __device__ __forceinline__ void fq_group(const float (&v)[CPT], int bits, bool s
     a = inv * inv_span;
     b = half * inv_span;  // q - qmin = rne(v / Delta) + 2^(b-1)
   } else {
-    const float mx = group_max<GL>(maxN(v));
-    const float mn = group_min<GL>(minN(v));
+    const float mx = clip * group_max<GL>(maxN(v));
+    const float mn = clip * group_min<GL>(minN(v));
     r.delta = fmaxf(mx - mn, kEpsDelta) * inv_span;
     const float inv = __frcp_rn(r.delta);
     r.zero = fminf(fmaxf(__fmaf_rn(-mn, inv, kRoundMagic) - kRoundMagic, 0.f), span);  // clamp(rne(-min / Delta))
