@@ -49,17 +49,19 @@ def test_clip_search_and_clipped_pack(name, wl):
     s_star = O.candidate_scales(a, 0.5).astype(np.float32)
     s_cand = np.stack([s_star] * len(CLIPS))
     Wb, W, cfg, best, ref = _run(wl, s_cand, CLIPS)
-    c = CLIPS[best]
-    q, sc, zr = awq.quantize_pack(W, torch.from_numpy(s_star).cuda(), cfg, clip=c)
-    torch.cuda.synchronize()
     s64 = s_star.astype(np.float64)
-    _, sc_ref, zr_ref, codes_ref, _, _ = O.pack(Wb, s64, wl.bits, wl.group, wl.symmetric, clip=c)
-    near = O.boundary_mask(Wb, s64, wl.bits, wl.group, wl.symmetric, clip=c)
-    codes = unpack_words(q, wl.d_in)
-    assert not ((codes != codes_ref) & ~near).any()
-    sc_g = sc.cpu().numpy().astype(np.float64)
-    assert np.all(np.abs(sc_g - sc_ref.astype(np.float64)) <= 2.0 ** -10 * np.abs(sc_ref.astype(np.float64)))
-    print(name, "best clip", c, "losses", ref["losses"])
+    for c in sorted({CLIPS[best], 0.8, 0.55}):
+        q, sc, zr = awq.quantize_pack(W, torch.from_numpy(s_star).cuda(), cfg, clip=c)
+        torch.cuda.synchronize()
+        _, sc_ref, zr_ref, codes_ref, _, _ = O.pack(Wb, s64, wl.bits, wl.group, wl.symmetric, clip=c)
+        near = O.boundary_mask(Wb, s64, wl.bits, wl.group, wl.symmetric, clip=c)
+        codes = unpack_words(q, wl.d_in)
+        assert not ((codes != codes_ref) & ~near).any(), c
+        sc_g = sc.cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(sc_g - sc_ref.astype(np.float64)) <= 2.0 ** -10 * np.abs(sc_ref.astype(np.float64)))
+        gnear = near.reshape(wl.d_out, -1, wl.group).any(axis=-1)
+        assert not ((zr.cpu().numpy() != zr_ref) & ~gnear).any(), c
+    print(name, "best clip", CLIPS[best], "losses", ref["losses"])
 
 
 def test_salience_mask_candidates():
