@@ -130,6 +130,7 @@ def quantize_groups(V: np.ndarray, bits: int, group: int, symmetric: bool,
     if d_in % group:
         raise ValueError("d_in must be a multiple of the group size")
     G = V.reshape(rows, d_in // group, group)
+    clip = np.broadcast_to(np.asarray(clip, dtype=np.float64), (rows, d_in // group))  # scalar or per group
     if symmetric:
         qmax = 2 ** (bits - 1) - 1
         qmin = -(2 ** (bits - 1))
@@ -275,6 +276,34 @@ def search_candidates(W_bits: np.ndarray, X_bits: np.ndarray, s_cand: np.ndarray
         dW = delta_weight(W, s_cand[k], bits, group, symmetric, clips[k])
         losses[k] = (row_losses_gram(dW, G) if form == "gram" else row_losses_direct(dW, X_bits)).sum()
     return dict(losses=losses, best=choose(losses))
+
+
+def group_clip_errors(W_bits: np.ndarray, X_bits: np.ndarray, s: np.ndarray, bits: int, group: int,
+                      symmetric: bool, clips, G: np.ndarray | None = None) -> np.ndarray:
+    """Per-group output error of each clip ratio, err[c, r, j] =
+    sum_t (sum_{i in group j} dW_c[r, i] X[t, i])^2, i.e. the output error the
+    group would cause with only its own inputs (the block-diagonal part of
+    dW G dW^T), with dW_c = Q(W S; clip c) S^-1 - W. This is the per-group
+    reading of the clipping search ([P5] 参考资料 note): each group of each row
+    then takes the ratio with the smallest error."""
+    W = widen_bf16(W_bits)
+    rows, d_in = W.shape
+    ng = d_in // group
+    if G is None:
+        G = gram(X_bits)
+    out = np.zeros((len(clips), rows, ng))
+    for ci, c in enumerate(clips):
+        dW = delta_weight(W, s, bits, group, symmetric, c)
+        for j in range(ng):
+            blk = dW[:, j * group:(j + 1) * group]
+            Gb = G[j * group:(j + 1) * group, j * group:(j + 1) * group]
+            out[ci, :, j] = np.einsum("ri,ri->r", blk @ Gb, blk)
+    return out
+
+
+def group_clip_choice(err: np.ndarray) -> np.ndarray:
+    """Index of the smallest error per (row, group), the lowest index on ties."""
+    return np.argmin(err, axis=0)
 
 
 def choose(losses: np.ndarray) -> int:

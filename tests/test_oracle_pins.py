@@ -500,3 +500,37 @@ def test_search_candidates_matches_search():
     clipped = O.search_candidates(W, X, np.stack([s_cand[2]] * 3), 4, 128, False, clips=[1.0, 0.9, 0.3])
     assert clipped["losses"][0] == pytest.approx(ref["losses"][2], rel=1e-14)
     assert clipped["losses"][2] > clipped["losses"][0]
+
+
+def test_per_group_clip_clamp_matches_scalar():
+    """A per-group clip array applies each group's own ratio."""
+    rng = np.random.default_rng(22)
+    V = rng.standard_normal((6, 32))
+    clip = np.array([[1.0, 0.5]] * 6)
+    full = O.quantize_groups(V, 4, 16, False, clip=clip)
+    for j, c in enumerate((1.0, 0.5)):
+        part = O.quantize_groups(V[:, 16 * j:16 * (j + 1)], 4, 16, False, clip=c)
+        assert np.array_equal(full[0][:, 16 * j:16 * (j + 1)], part[0])
+
+
+def test_group_clip_errors_brute_force():
+    """err[c, r, j] equals the direct per-group output error with a triple loop
+    over tokens and the group's channels."""
+    rng = np.random.default_rng(23)
+    Wb = gen.f64_to_bf16_bits(rng.standard_normal((3, 32)) * 0.05)
+    Xb = gen.f64_to_bf16_bits(rng.standard_normal((5, 32)) * np.linspace(0.5, 3, 32))
+    s = O.candidate_scales(O.act_stats(Xb), 0.4)
+    clips = [1.0, 0.8, 0.6]
+    err = O.group_clip_errors(Wb, Xb, s, 4, 16, False, clips)
+    W, X = O.widen_bf16(Wb), O.widen_bf16(Xb)
+    for ci, c in enumerate(clips):
+        dW = O.delta_weight(W, s, 4, 16, False, c)
+        for r in range(3):
+            for j in range(2):
+                tot = 0.0
+                for t in range(5):
+                    tot += sum(dW[r, i] * X[t, i] for i in range(16 * j, 16 * j + 16)) ** 2
+                assert err[ci, r, j] == pytest.approx(tot, rel=1e-12, abs=1e-300)
+    best = O.group_clip_choice(err)
+    assert best.shape == (3, 2)
+    assert np.all(err[best, np.arange(3)[:, None], np.arange(2)[None, :]] <= err[0] + 0.0)
