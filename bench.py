@@ -36,6 +36,7 @@ METRIC = "AWQ search: alpha-candidate layer evals/s, TFLOP/s vs bf16 peak; stats
 UNIT = "alpha-candidate layer evals/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 L2_FLUSH_BYTES = 256 << 20
+GROUP_CLIPS = [1.0, 0.95, 0.9, 0.85, 0.8, 0.75, 0.7, 0.6, 0.5]  # ratios of the per-group clipping pass
 
 
 def load_peaks():
@@ -59,7 +60,7 @@ def kernel_source_hash():
 def profiled_traffic(config_key, form):
     """Per-launch DRAM bytes of the contraction from the committed ncu summary,
     if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", f"contract_{form}_{config_key}.md")
+    path = os.path.join(ROOT, "profiles", f"contract_pair_{form}_{config_key}.md")
     if not os.path.exists(path):
         return None
     vals = {}
@@ -297,6 +298,44 @@ def run_ours(args, rank, world, local_rank):
     h2d = Wb.nbytes + Xb.nbytes
     d2h = sum(h.numel() * h.element_size() for h in host_out)
 
+    # ---- per-group clipping with the chosen scales (a follow-on pass, timed apart from the step)
+    gclip = None
+    if wl.group >= 32 and not args.no_group_clip:
+        ccfg = awq.make_cfg(wl.bits, wl.group, wl.symmetric, len(GROUP_CLIPS))
+        cws = awq.workspace(awq.group_clip_workspace_size(d_out, d_in, N, ccfg))
+        best_clip = torch.empty((d_out, ng), dtype=torch.uint8, device=dev)
+        cp = (ctypes.c_float * len(GROUP_CLIPS))(*GROUP_CLIPS)
+
+        def clip_step():
+            st = B._stream()
+            B._check(L.awq_search_group_clip(ctypes.c_void_p(W.data_ptr()), ctypes.c_void_p(X.data_ptr()),
+                                             ctypes.c_void_p(outs["s_best"].data_ptr()), ctypes.cast(cp, ctypes.c_void_p),
+                                             d_out, d_in, N, ctypes.byref(ccfg), ctypes.c_void_p(cws.data_ptr()),
+                                             cws.numel(), ctypes.c_void_p(best_clip.data_ptr()), None, st),
+                     "awq_search_group_clip")
+            awq.quantize_pack_group_clip(W, outs["s_best"], GROUP_CLIPS, best_clip, ccfg, outputs=packed)
+
+        for _ in range(3):
+            clip_step()
+        torch.cuda.synchronize()
+        g_ms = []
+        for k in range(KB):
+            flush.fill_(k & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            clip_step()
+            e1.record()
+            e1.synchronize()
+            g_ms.append(e0.elapsed_time(e1))
+        awq.workspace_error(cws)
+        gms = float(np.mean(g_ms))
+        if world > 1:
+            gms = max_over_ranks([gms], dev)[0]
+        gclip = {"clips": GROUP_CLIPS, "ms_per_pass": round(gms, 4),
+                 "clip_group_evals_per_s": round(world * len(GROUP_CLIPS) * d_out * ng / (gms * 1e-3), 1),
+                 "note": "search_group_clip + quantize_pack_group_clip with s_best, " + str(KB) + " passes, L2 flushed"}
+        del cws
+
     peaks = load_peaks()
     n_a = wl.n_alpha
     flops_direct = 2.0 * n_a * d_out * d_in * N
@@ -349,6 +388,7 @@ def run_ours(args, rank, world, local_rank):
         "layers_per_s": round(world / (ms_per_step * 1e-3), 3),
         "e2e": {"value": round(world * n_a * K / (e2e_total * 1e-3), 2), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "group_clip": gclip,
         "gpu_launches": launches_per_step(form, n_a) * K,
         "clocks": clk,
         "wall_s_timed_region": round(t_wall, 3),
@@ -433,6 +473,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--cpu-rows", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-group-clip", action="store_true", help="skip the per-group clipping pass")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -200,6 +200,41 @@ awq_status awq_search_candidates(const void* W_bf16, const void* X_bf16, const f
                                  awq_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Per-group clipping search ([P5] 参考资料 note: the clipping search, read per
+ * quantisation group). With the scales s fixed (DEVICE float [d_in], every
+ * entry > 0, e.g. s_best of the scale search), clip candidate c (ratio
+ * clips[c], HOST float [n] in (0, 1], n = cfg->n_alpha <= 64; cfg->alphas is
+ * ignored) gives dW_c = Q(W S; clips[c]) S^-1 - W. For row r and group j
+ * (columns j*g .. j*g+g-1) its error is the group's own output error
+ *   err[c, r, j] = sum_t (sum_{i in j} dW_c[r, i] X[t, i])^2
+ *               = dW_c[r, j] G_jj dW_c[r, j]^T,    G = X^T X,
+ * i.e. the block-diagonal part of the layer error dW G dW^T. Computed as:
+ * the diagonal 256-blocks of G on the tensor cores (masked to the groups),
+ * every candidate's dW stack, one contraction of dW against those blocks with
+ * per-32-column partials, then a float64 sum per group and the argmin.
+ *   best_clip   DEVICE uint8 [d_out, d_in/g]: index of the smallest error,
+ *               the lowest index on exact ties.
+ *   group_err   DEVICE float [n, d_out, d_in/g] or NULL: the errors.
+ * Requires g >= 32 (AWQ_ERR_UNSUPPORTED otherwise). Workspace:
+ * awq_group_clip_workspace_size; non-finite errors or a non-positive scale
+ * are recorded as AWQ_ERR_NONFINITE (awq_workspace_error). Asynchronous.
+ * ------------------------------------------------------------------------- */
+size_t awq_group_clip_workspace_size(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg);
+awq_status awq_search_group_clip(const void* W_bf16, const void* X_bf16, const float* s, const float* clips,
+                                 int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
+                                 size_t ws_bytes, uint8_t* best_clip, float* group_err, awq_stream_t stream);
+
+/* awq_quantize_pack with a clip ratio per (row, group): group j of row r uses
+ * clips[best_clip[r * (d_in/g) + j]] (clips HOST float [n_clips] in (0, 1],
+ * n_clips <= 64; best_clip DEVICE uint8 [d_out, d_in/g], entries < n_clips,
+ * e.g. the output of awq_search_group_clip; an entry >= n_clips means no
+ * clipping). Outputs as in awq_quantize_pack. AWQ_ERR_INVALID_ARG for a ratio
+ * outside (0, 1], n_clips outside [1, 64] or a NULL table. */
+awq_status awq_quantize_pack_group_clip(const void* W_bf16, const float* s, const float* clips, int32_t n_clips,
+                                        const uint8_t* best_clip, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
+                                        uint32_t* qweight, void* scales_f16, void* zeros_f16, awq_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * The search, one step at a time (awq_search_scales is exactly these calls
  * in this order). They share the search workspace; offsets are internal.
  * ------------------------------------------------------------------------- */
@@ -210,7 +245,8 @@ awq_status awq_step_scales(const float* a, int64_t d_out, int64_t d_in, int64_t 
  * workspace (rows padded to a multiple of 128 with zeros). */
 awq_status awq_step_fake_quant(const void* W_bf16, int64_t d_out, int64_t d_in, int64_t N,
                                const awq_qcfg* cfg, void* ws, size_t ws_bytes, awq_stream_t stream);
-/* a4 (Gram form only): X^T into the workspace, then G = X^T X (bf16). */
+/* a4 (Gram form only): the lower block triangle of G = X^T X (bf16, strictly
+ * lower 256-blocks doubled) into the workspace. */
 awq_status awq_step_gram(const void* X_bf16, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg,
                          void* ws, size_t ws_bytes, awq_stream_t stream);
 /* a5: the tensor-core contraction with the fused squared-sum epilogue, per

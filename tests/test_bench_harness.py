@@ -59,9 +59,9 @@ def test_launch_count():
 def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "contract_gram_CX.md").write_text(
+    (prof / "contract_pair_gram_CX.md").write_text(
         f"- source_sha256: `{bench.kernel_source_hash()}`\n- traffic_bytes_per_launch: `123`\n")
-    (prof / "contract_gram_CY.md").write_text("- source_sha256: `0000`\n- traffic_bytes_per_launch: `456`\n")
+    (prof / "contract_pair_gram_CY.md").write_text("- source_sha256: `0000`\n- traffic_bytes_per_launch: `456`\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     (tmp_path / "weight_only_int4_act_b200" / "csrc").mkdir(parents=True)
     for f in ("gemm_pair_sm100.cuh", "gemm_sm100.cuh", "ptx.cuh"):

@@ -136,3 +136,36 @@ def test_segmented_search_validation():
     assert call([256, 0]) == 2                # empty layer
     assert lib.awq_search_scales_segmented(FAKE, FAKE, FAKE, 256, 512, 256, c, 1, None, FAKE, big, FAKE, FAKE, FAKE,
                                            None, None) == 1
+
+
+def test_group_clip_validation():
+    lib = awq.lib()
+    big = 1 << 40
+    cfg = awq.make_cfg(4, 128, False, 4)
+    c = ctypes.byref(cfg)
+    clips = (ctypes.c_float * 4)(1.0, 0.9, 0.8, 0.7)
+    cp = ctypes.cast(clips, ctypes.c_void_p)
+    need = awq.group_clip_workspace_size(256, 512, 256, cfg)
+    # the candidate stack of 4 x 256 x 512 bf16 and the 512 x 256 diagonal blocks of G
+    assert need >= 4 * 256 * 512 * 2 + 512 * 256 * 2
+    assert awq.group_clip_workspace_size(200, 512, 256, cfg) == need  # rows pad to 128
+    assert awq.group_clip_workspace_size(256, 512, 256, awq.make_cfg(4, 16, False, 4)) == 0  # g < 32
+
+    def call(cfg_=cfg, clips_=cp, ws_bytes=big, best=FAKE, d_in=512):
+        return lib.awq_search_group_clip(FAKE, FAKE, FAKE, clips_, 256, d_in, 256, ctypes.byref(cfg_), FAKE,
+                                         ws_bytes, best, None, None)
+    assert call(cfg_=awq.make_cfg(4, 16, False, 4)) == 7          # AWQ_ERR_UNSUPPORTED
+    assert call(ws_bytes=need - 1) == 3                           # AWQ_ERR_WORKSPACE
+    assert call(best=None) == 1
+    assert call(clips_=None) == 1
+    assert call(d_in=500) == 2
+    bad = (ctypes.c_float * 4)(1.0, 0.9, 1.5, 0.7)
+    assert call(clips_=ctypes.cast(bad, ctypes.c_void_p)) == 1
+    # pack with a clip per group
+    pk = lib.awq_quantize_pack_group_clip
+    assert pk(FAKE, FAKE, None, 4, FAKE, 256, 512, c, FAKE, FAKE, FAKE, None) == 1
+    assert pk(FAKE, FAKE, cp, 0, FAKE, 256, 512, c, FAKE, FAKE, FAKE, None) == 1
+    assert pk(FAKE, FAKE, cp, 65, FAKE, 256, 512, c, FAKE, FAKE, FAKE, None) == 1
+    assert pk(FAKE, FAKE, cp, 4, None, 256, 512, c, FAKE, FAKE, FAKE, None) == 1
+    assert pk(FAKE, FAKE, ctypes.cast(bad, ctypes.c_void_p), 4, FAKE, 256, 512, c, FAKE, FAKE, FAKE, None) == 1
+    assert pk(FAKE, FAKE, cp, 4, FAKE, 256, 500, c, FAKE, FAKE, FAKE, None) == 2

@@ -25,7 +25,8 @@ EXPORTED = (
     "awq_search_scales", "awq_search_form", "awq_workspace_error", "awq_quantize_pack",
     "awq_step_scales", "awq_step_fake_quant", "awq_step_gram", "awq_step_contract", "awq_step_reduce",
     "awq_debug_copy_dw", "awq_act_stats_noalloc", "awq_search_scales_segmented", "awq_search_candidates",
-    "awq_quantize_pack_clipped",
+    "awq_quantize_pack_clipped", "awq_group_clip_workspace_size", "awq_search_group_clip",
+    "awq_quantize_pack_group_clip",
 )
 
 
@@ -79,6 +80,11 @@ def lib() -> ctypes.CDLL:
                                                 c_void_p]),
             "awq_quantize_pack_clipped": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_float, c_void_p,
                                                     c_void_p, c_void_p, c_void_p]),
+            "awq_group_clip_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, cfgp]),
+            "awq_search_group_clip": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64,
+                                                cfgp, c_void_p, c_size_t, c_void_p, c_void_p, c_void_p]),
+            "awq_quantize_pack_group_clip": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_int64,
+                                                       c_int64, cfgp, c_void_p, c_void_p, c_void_p, c_void_p]),
             "awq_workspace_error": (c_int32, [c_void_p, c_void_p]),
             "awq_quantize_pack": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_void_p, c_void_p,
                                             c_void_p, c_void_p]),
@@ -252,6 +258,59 @@ def search_candidates(W, X, s_cand, cfg: QCfg, clips=None, ws=None, row_losses=F
                                        _ptr(o["best"]), _ptr(o["s_best"]), _ptr(o["row_losses"]), _stream()),
            "awq_search_candidates")
     return dict(o, ws=ws)
+
+
+def group_clip_workspace_size(d_out, d_in, N, cfg: QCfg) -> int:
+    return int(lib().awq_group_clip_workspace_size(d_out, d_in, N, ctypes.byref(cfg)))
+
+
+def _clip_array(clips, n):
+    if len(clips) != n:
+        raise ValueError("need one clip ratio per candidate")
+    return (c_float * n)(*[float(c) for c in clips])
+
+
+def search_group_clip(W, X, s, clips, cfg: QCfg, ws=None, group_err=False):
+    """Per-(row, group) clip choice with the scales s fixed: clips is a host
+    sequence of cfg.n_alpha ratios. Returns dict(best_clip uint8 [d_out, d_in/g],
+    group_err float32 [n, d_out, d_in/g] or None, ws)."""
+    torch = _torch()
+    _req(W, torch.bfloat16, None, "W")
+    d_out, d_in = W.shape
+    _req(X, torch.bfloat16, None, "X")
+    N = X.shape[0]
+    _req(s, torch.float32, (d_in,), "s")
+    carr = _clip_array(clips, cfg.n_alpha)
+    if ws is None:
+        ws = workspace(group_clip_workspace_size(d_out, d_in, N, cfg))
+    ng = d_in // cfg.group if cfg.group > 0 else 0
+    o = dict(best_clip=torch.empty((d_out, ng), dtype=torch.uint8, device=W.device),
+             group_err=torch.empty((cfg.n_alpha, d_out, ng), dtype=torch.float32, device=W.device)
+             if group_err else None)
+    _check(lib().awq_search_group_clip(_ptr(W), _ptr(X), _ptr(s), ctypes.cast(carr, c_void_p), d_out, d_in, N,
+                                       ctypes.byref(cfg), _ptr(ws), ws.numel(), _ptr(o["best_clip"]),
+                                       _ptr(o["group_err"]), _stream()), "awq_search_group_clip")
+    return dict(o, ws=ws)
+
+
+def quantize_pack_group_clip(W, s, clips, best_clip, cfg: QCfg, outputs=None):
+    """quantize_pack with group j of row r clipped at clips[best_clip[r, j]]."""
+    torch = _torch()
+    _req(W, torch.bfloat16, None, "W")
+    d_out, d_in = W.shape
+    _req(s, torch.float32, (d_in,), "s")
+    ng = d_in // cfg.group if cfg.group > 0 else 0
+    _req(best_clip, torch.uint8, (d_out, ng), "best_clip")
+    carr = _clip_array(clips, len(clips))
+    if outputs is None:
+        outputs = (torch.empty((d_out, d_in // 8), dtype=torch.int32, device=W.device),
+                   torch.empty((d_out, ng), dtype=torch.float16, device=W.device),
+                   torch.empty((d_out, ng), dtype=torch.float16, device=W.device))
+    q, sc, zr = outputs
+    _check(lib().awq_quantize_pack_group_clip(_ptr(W), _ptr(s), ctypes.cast(carr, c_void_p), len(clips),
+                                              _ptr(best_clip), d_out, d_in, ctypes.byref(cfg), _ptr(q), _ptr(sc),
+                                              _ptr(zr), _stream()), "awq_quantize_pack_group_clip")
+    return q, sc, zr
 
 
 def workspace_error(ws):

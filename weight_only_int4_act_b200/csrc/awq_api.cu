@@ -212,7 +212,8 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
     if (!make_map(&tb, B, K, Nr, ldb, GEMM_BK)) return AWQ_ERR_CUDA;
   } else {
     if (!make_map(&ta, A, M, K, lda, GEMM_BM)) return AWQ_ERR_CUDA;
-    if (!make_map(&tb, B, Nr, K, ldb, GEMM_BN)) return AWQ_ERR_CUDA;
+    // TRI_DIAG: B is the compact [Nr, 256] diagonal-block matrix
+    if (!make_map(&tb, B, Nr, tri == TRI_DIAG ? GEMM_BN : K, ldb, GEMM_BN)) return AWQ_ERR_CUDA;
   }
   args.M = (int)M;
   args.N = (int)Nr;
@@ -222,7 +223,8 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
   args.group_n = kGroupN < args.n_blocks_n ? kGroupN : args.n_blocks_n;
   args.tri = tri;
   const long long tiles = tri == TRI_LOWER_STORE ? tri_lower_tiles(args.n_blocks_m)
-                                                 : (long long)args.n_blocks_m * args.n_blocks_n;
+                          : tri == TRI_DIAG_STORE ? args.n_blocks_m
+                                                  : (long long)args.n_blocks_m * args.n_blocks_n;
   if (tiles > INT32_MAX) return AWQ_ERR_SHAPE;
   args.num_tiles = (int)tiles;
   if (cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE, MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -508,6 +510,107 @@ awq_status awq_search_scales_segmented(const void* W, const void* X, const float
   return launch_status();
 }
 
+namespace {
+// Workspace of the per-group clipping search (cfg->n_alpha = number of clip ratios).
+struct ClipLayout {
+  int n, d_out_pad, n_chunks;  // candidates, padded rows, 32-column chunks of the partials
+  long long M;
+  size_t off_s, off_inv, off_dw, off_part, off_g, total;
+};
+
+ClipLayout clip_layout(int64_t d_out, int64_t d_in, const awq_qcfg* cfg) {
+  ClipLayout L{};
+  L.n = cfg->n_alpha;
+  L.d_out_pad = (int)(cdiv(d_out, GEMM_BM) * GEMM_BM);
+  L.M = (long long)L.n * L.d_out_pad;
+  L.n_chunks = (int)cdiv(d_in, GEMM_BN) * (GEMM_BN / 32);
+  size_t off = kAlign;
+  L.off_s = off;    off += align_up((size_t)L.n * d_in * sizeof(float));
+  L.off_inv = off;  off += align_up((size_t)L.n * d_in * sizeof(float));
+  L.off_dw = off;   off += align_up((size_t)L.M * d_in * 2);
+  L.off_part = off; off += align_up((size_t)L.n_chunks * L.M * sizeof(float));
+  L.off_g = off;    off += align_up((size_t)d_in * GEMM_BN * 2);
+  L.total = off;
+  return L;
+}
+
+awq_status check_clip_common(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, const void* ws,
+                             size_t ws_bytes, ClipLayout* L) {
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_layer_shape(d_out, d_in, cfg)) != AWQ_OK) return st;
+  if ((st = check_tokens(N)) != AWQ_OK) return st;
+  if (cfg->group < 32) return AWQ_ERR_UNSUPPORTED;  // errors are gathered per 32-column chunk
+  if (!ws || !aligned(ws, 256)) return AWQ_ERR_INVALID_ARG;
+  *L = clip_layout(d_out, d_in, cfg);
+  if (ws_bytes < L->total) return AWQ_ERR_WORKSPACE;
+  return AWQ_OK;
+}
+}  // namespace
+
+size_t awq_group_clip_workspace_size(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg) {
+  ClipLayout L;
+  if (check_clip_common(d_out, d_in, N, cfg, reinterpret_cast<void*>(256), SIZE_MAX, &L) != AWQ_OK) return 0;
+  return L.total;
+}
+
+awq_status awq_search_group_clip(const void* W, const void* X, const float* s, const float* clips, int64_t d_out,
+                                 int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws, size_t ws_bytes,
+                                 uint8_t* best_clip, float* group_err, awq_stream_t stream) {
+  ClipLayout L;
+  awq_status st = check_clip_common(d_out, d_in, N, cfg, ws, ws_bytes, &L);
+  if (st != AWQ_OK) return st;
+  if (!W || !X || !s || !clips || !best_clip) return AWQ_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
+  ClipTable table{};
+  for (int k = 0; k < L.n; ++k) {
+    if (!(clips[k] > 0.f && clips[k] <= 1.f)) return AWQ_ERR_INVALID_ARG;
+    table.c[k] = clips[k];
+  }
+  int sms = 0;
+  if ((st = check_device(&sms)) != AWQ_OK) return st;
+  cudaStream_t cs = as_stream(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(int), cs) != cudaSuccess) return AWQ_ERR_CUDA;
+  repeat_scales<<<2 * sms, 256, 0, cs>>>(s, (int)d_in, L.n, at<float>(ws, L.off_s), at<float>(ws, L.off_inv),
+                                         at<int>(ws, 0));
+  if ((st = launch_status()) != AWQ_OK) return st;
+  // candidates: the same scales, one clip ratio each
+  SearchLayout SL{};
+  SL.d_out_pad = L.d_out_pad;
+  SL.off_s = L.off_s;
+  SL.off_inv = L.off_inv;
+  SL.off_dw = L.off_dw;
+  if ((st = launch_fake_quant(W, d_out, d_in, cfg, SL, ws, 0, L.n, sms, 0, cs, &table)) != AWQ_OK) return st;
+  // diagonal 256-blocks of G = X^T X, masked to each quantisation group, compact [d_in, 256]
+  GemmArgs gs{};
+  gs.C = at<__nv_bfloat16>(ws, L.off_g);
+  gs.ldC = GEMM_BN;
+  gs.err = at<int>(ws, 0);
+  gs.tile_counter = at<int>(ws, kTileCounterOffset);
+  gs.group = cfg->group;
+  // entries outside the stored diagonal (columns past d_in) must read as 0
+  if (cudaMemsetAsync(gs.C, 0, (size_t)d_in * GEMM_BN * 2, cs) != cudaSuccess) return AWQ_ERR_CUDA;
+  if ((st = run_gemm<EPI_STORE, true>(X, d_in, d_in, X, d_in, d_in, N, gs, TRI_DIAG_STORE, sms, cs)) != AWQ_OK)
+    return st;
+  // per (row, 32-column chunk) errors of every candidate: dW[:, J] G_J dW[:, J]^T restricted to the groups
+  GemmArgs ga{};
+  ga.part = at<float>(ws, L.off_part);
+  ga.part_ld = L.M;
+  ga.err = at<int>(ws, 0);
+  ga.tile_counter = at<int>(ws, kTileCounterOffset);
+  ga.E = at<__nv_bfloat16>(ws, L.off_dw);
+  ga.ldE = d_in;
+  if ((st = run_gemm<EPI_DOT32>(at<void>(ws, L.off_dw), L.M, d_in, at<void>(ws, L.off_g), d_in, GEMM_BN, d_in, ga,
+                                TRI_DIAG, sms, cs)) != AWQ_OK)
+    return st;
+  const int ng = (int)(d_in / cfg->group);
+  const long long units = (long long)ng * d_out;
+  group_clip_argmin<<<(unsigned)(cdiv(units, 256) < 8 * sms ? cdiv(units, 256) : 8 * sms), 256, 0, cs>>>(
+      at<float>(ws, L.off_part), L.M, (int)d_out, L.d_out_pad, ng, cfg->group / 32, L.n, best_clip, group_err,
+      at<int>(ws, 0));
+  return launch_status();
+}
+
 awq_status awq_workspace_error(void* ws, awq_stream_t stream) {
   if (!ws) return AWQ_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
@@ -520,8 +623,9 @@ awq_status awq_workspace_error(void* ws, awq_stream_t stream) {
   return word == ERR_NONFINITE ? AWQ_ERR_NONFINITE : AWQ_ERR_DEVICE;
 }
 
-awq_status awq_quantize_pack_clipped(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
-                                     float clip, uint32_t* qweight, void* scales, void* zeros, awq_stream_t stream) {
+awq_status pack_impl(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg, float clip,
+                     const uint8_t* group_clip, const ClipTable& gtable, uint32_t* qweight, void* scales, void* zeros,
+                     awq_stream_t stream) {
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if ((st = check_layer_shape(d_out, d_in, cfg)) != AWQ_OK) return st;
@@ -536,7 +640,7 @@ awq_status awq_quantize_pack_clipped(const void* W, const float* s, int64_t d_ou
     const int grid = elementwise_grid(kernel, units, sms);
     kernel<<<grid, 256, 0, as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(W), s, (int)d_out, (int)d_in,
                                                 cfg->bits, cfg->symmetric, qweight, static_cast<__half*>(scales),
-                                                static_cast<__half*>(zeros), clip);
+                                                static_cast<__half*>(zeros), clip, group_clip, gtable);
   };
   constexpr int C = FQ_CPT;
   switch (cfg->group) {
@@ -551,9 +655,28 @@ awq_status awq_quantize_pack_clipped(const void* W, const float* s, int64_t d_ou
   return launch_status();
 }
 
+awq_status awq_quantize_pack_clipped(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
+                                     float clip, uint32_t* qweight, void* scales, void* zeros, awq_stream_t stream) {
+  ClipTable none{};
+  return pack_impl(W, s, d_out, d_in, cfg, clip, nullptr, none, qweight, scales, zeros, stream);
+}
+
 awq_status awq_quantize_pack(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
                              uint32_t* qweight, void* scales, void* zeros, awq_stream_t stream) {
   return awq_quantize_pack_clipped(W, s, d_out, d_in, cfg, 1.0f, qweight, scales, zeros, stream);
+}
+
+awq_status awq_quantize_pack_group_clip(const void* W, const float* s, const float* clips, int32_t n_clips,
+                                        const uint8_t* best_clip, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
+                                        uint32_t* qweight, void* scales, void* zeros, awq_stream_t stream) {
+  if (!clips || !best_clip || n_clips < 1 || n_clips > MAX_ALPHA) return AWQ_ERR_INVALID_ARG;
+  ClipTable table;
+  for (int k = 0; k < MAX_ALPHA; ++k) table.c[k] = 1.0f;  // indices past n_clips: no clipping
+  for (int k = 0; k < n_clips; ++k) {
+    if (!(clips[k] > 0.f && clips[k] <= 1.f)) return AWQ_ERR_INVALID_ARG;
+    table.c[k] = clips[k];
+  }
+  return pack_impl(W, s, d_out, d_in, cfg, 1.0f, best_clip, table, qweight, scales, zeros, stream);
 }
 
 awq_status awq_search_candidates(const void* W, const void* X, const float* s_cand, const float* clips,

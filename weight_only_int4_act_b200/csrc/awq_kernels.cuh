@@ -399,6 +399,51 @@ __global__ void segment_argmin(const double* __restrict__ seg_sums, int n_seg, i
 }
 
 // ---------------------------------------------------------------------------
+// Per-group clipping search. s_all[k] = s, inv_all[k] = 1/s for k < n.
+// ---------------------------------------------------------------------------
+__global__ void repeat_scales(const float* __restrict__ s, int d_in, int n, float* __restrict__ s_all,
+                              float* __restrict__ inv_all, int* err) {
+  const long long total = (long long)n * d_in;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float v = s[i % d_in];
+    if (!(v > 0.f) || !isfinite(v)) atomicCAS(err, 0, ERR_NONFINITE);
+    s_all[i] = v;
+    inv_all[i] = 1.0f / v;
+  }
+}
+
+// err[c][r][j] = sum of the group's 32-column partials (fp64, in order) for
+// clip candidate c; best[r][j] = argmin over c (lowest index on ties).
+// part layout: part[chunk32 * part_ld + c * d_out_pad + r]. One thread per
+// (group j, row r), rows fastest.
+__global__ void group_clip_argmin(const float* __restrict__ part, long long part_ld, int d_out, int d_out_pad,
+                                  int n_groups, int chunks_per_group, int n_clip, uint8_t* __restrict__ best,
+                                  float* __restrict__ group_err, int* err) {
+  const long long total = (long long)n_groups * d_out;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int j = (int)(i / d_out), r = (int)(i - (long long)j * d_out);
+    double bv = INFINITY;
+    int bi = 0;
+    bool finite = true;
+    for (int c = 0; c < n_clip; ++c) {
+      double e = 0.0;
+      for (int u = 0; u < chunks_per_group; ++u)
+        e += (double)part[(long long)(j * chunks_per_group + u) * part_ld + (long long)c * d_out_pad + r];
+      if (!isfinite(e)) finite = false;
+      if (group_err) group_err[((long long)c * d_out + r) * n_groups + j] = (float)e;
+      if (e < bv) {
+        bv = e;
+        bi = c;
+      }
+    }
+    if (!finite) atomicCAS(err, 0, ERR_NONFINITE);
+    best[(long long)r * n_groups + j] = (uint8_t)bi;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // a7: pack. Codes of Q(W S) (same quantiser as the search), 8 nibbles per
 // uint32 (channel 8w+j in bits 4j..4j+3), fp16 step and zero per group.
 // ([P2] §2.1 INT4 with fp16 scale, §4.2 packed 4-bit storage; [P4] §三.)
@@ -412,7 +457,8 @@ template <int CPT, int GL>
 __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __restrict__ W, const float* __restrict__ s,
                                                      int d_out, int d_in, int bits, int symmetric,
                                                      uint32_t* __restrict__ qweight, __half* __restrict__ scales,
-                                                     __half* __restrict__ zeros, float clip) {
+                                                     __half* __restrict__ zeros, float clip,
+                                                     const uint8_t* __restrict__ group_clip, ClipTable clips) {
   const int chunks = d_in / CPT;
   const int row_groups = (d_out + PACK_ROWS - 1) / PACK_ROWS;
   const long long total = (long long)row_groups * chunks;
@@ -449,8 +495,14 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[8 * q + j] = f[j] * sc[8 * q + j];
       }
+      // per-group clip ratio (index into clips) when given, else the scalar one
+      float c = clip;
+      if (group_clip && active && row0 + r < d_out) {
+        const int idx = group_clip[(long long)(row0 + r) * groups + chunk / GL];
+        c = idx < MAX_ALPHA ? clips.c[idx] : 1.0f;
+      }
       FqGroup<CPT> fr;
-      fq_group<CPT, GL>(v, bits, sym, fr, clip);
+      fq_group<CPT, GL>(v, bits, sym, fr, c);
       if (active && row0 + r < d_out) {
         const int row = row0 + r;
         uint32_t* wp = qweight + (long long)row * words + c0 / 8;

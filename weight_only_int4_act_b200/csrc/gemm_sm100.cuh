@@ -17,6 +17,7 @@
 //     EPI_SUMSQ  part[n_blk][m] = sum_{n in tile} D[m,n]^2         (||dW X^T||^2)
 //     EPI_DOT    part[n_blk][m] = sum_{n in tile} D[m,n] E[m,n]    (trace(dW G dW^T))
 //     EPI_STORE  C[m, n] = bf16(D[m, n])                            (G = X^T X)
+//     EPI_DOT32  as EPI_DOT, one partial per 32-column chunk          (per-group errors)
 // The accumulator is released before the partials are written, so the next
 // tile's MMAs overlap this tile's epilogue.
 //
@@ -43,7 +44,7 @@
 
 namespace awq {
 
-enum EpiMode { EPI_SUMSQ = 0, EPI_DOT = 1, EPI_STORE = 2 };
+enum EpiMode { EPI_SUMSQ = 0, EPI_DOT = 1, EPI_STORE = 2, EPI_DOT32 = 3 };
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BN = 256;
@@ -61,7 +62,11 @@ constexpr int ERR_WAIT_EMPTY = 0x101, ERR_WAIT_FULL = 0x102, ERR_WAIT_TEMPTY = 0
               ERR_WAIT_SCHED = 0x105;
 constexpr int GEMM_SCHED_SLOTS = 4;  // tile indices published ahead of the MMA and epilogue warps
 
-enum TriMode { TRI_NONE = 0, TRI_LOWER_STORE = 1, TRI_K = 2 };
+// TRI_DIAG_STORE: only the diagonal 256-blocks of G, stored compactly as
+// C[m, j] = G[m, 256*(m/256) + j] (ldC = 256) with the entries whose row and
+// column fall in different quantisation groups set to 0; TRI_DIAG: column
+// tile J contracts k in [256J, 256J+256) of A against that compact B.
+enum TriMode { TRI_NONE = 0, TRI_LOWER_STORE = 1, TRI_K = 2, TRI_DIAG_STORE = 3, TRI_DIAG = 4 };
 
 struct GemmArgs {
   int M, N, K;                 // problem size (rows of A, rows of B, contraction length)
@@ -77,6 +82,7 @@ struct GemmArgs {
   long long ldC;
   int* err;                    // device error word
   int* tile_counter;           // dynamic tile counter, zero at launch
+  int group;                   // TRI_DIAG_STORE: quantisation group size (divides 256)
 };
 
 // Number of tiles of the lower block triangle with n_blocks_m row tiles of
@@ -87,6 +93,11 @@ __host__ __device__ inline long long tri_lower_tiles(long long n_blocks_m) {
 }
 
 __device__ __forceinline__ void gemm_tile_coords(int t, const GemmArgs& a, int& mb, int& nb) {
+  if (a.tri == TRI_DIAG_STORE) {
+    mb = t;
+    nb = t >> 1;
+    return;
+  }
   if (a.tri == TRI_LOWER_STORE) {
     // rows 2q and 2q+1 each hold q+1 tiles; tiles before row 2q: q(q+1)
     int q = (int)((sqrtf(4.0f * (float)t + 1.0f) - 1.0f) * 0.5f);
@@ -122,6 +133,7 @@ __device__ __forceinline__ void gemm_tile_coords(int t, const GemmArgs& a, int& 
 __device__ __forceinline__ int gemm_num_kb(const GemmArgs& a, int nb) {
   int k = a.K;
   if (a.tri == TRI_K) k = min(k, (nb + 1) * GEMM_BN);
+  if (a.tri == TRI_DIAG) k = min(GEMM_BN, a.K - nb * GEMM_BN);
   return (k + GEMM_BK - 1) / GEMM_BK;
 }
 
@@ -232,7 +244,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               tma_load_2d(smem_u32(sB + stage * GEMM_B_STAGE + c * GEMM_MN_CHUNK), &tmB, full_bar(stage),
                           nb * GEMM_BN + c * 64, kb * GEMM_BK);
           } else {
-            tma_load_2d(smem_u32(sA + stage * GEMM_A_STAGE), &tmA, full_bar(stage), kb * GEMM_BK, mb * GEMM_BM);
+            const int ka = (args.tri == TRI_DIAG ? nb * GEMM_BN : 0) + kb * GEMM_BK;  // TRI_DIAG: B is compact
+            tma_load_2d(smem_u32(sA + stage * GEMM_A_STAGE), &tmA, full_bar(stage), ka, mb * GEMM_BM);
             tma_load_2d(smem_u32(sB + stage * GEMM_B_STAGE), &tmB, full_bar(stage), kb * GEMM_BK, nb * GEMM_BN);
           }
           issued |= 1u << stage;
@@ -333,8 +346,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       float sum = 0.f;
 #pragma unroll 1
       for (int c = 0; c < GEMM_BN / 32; ++c) {
-        uint4 e[4];  // EPI_DOT: the 32 elements of E this chunk multiplies, fetched before the TMEM load
-        if constexpr (MODE == EPI_DOT) {
+        uint4 e[4];  // EPI_DOT(32): the 32 elements of E this chunk multiplies, fetched before the TMEM load
+        if constexpr (MODE == EPI_DOT || MODE == EPI_DOT32) {
           const int col = n0 + c * 32;
           const __nv_bfloat16* erow = args.E + (long long)m * args.ldE + col;
 #pragma unroll
@@ -351,7 +364,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const float d = __uint_as_float(r[j]);
             sum = fmaf(d, d, sum);
           }
-        } else if constexpr (MODE == EPI_DOT) {
+        } else if constexpr (MODE == EPI_DOT || MODE == EPI_DOT32) {
           // columns past N hold D = 0 (zero-filled B rows) and e = 0
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -362,19 +375,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               sum = fmaf(__uint_as_float(r[v * 8 + 2 * h + 1]), bf16hi(ew[h]), sum);
             }
           }
+          if constexpr (MODE == EPI_DOT32) {  // one partial per 32-column chunk
+            if (m < args.M) args.part[(long long)(nb * (GEMM_BN / 32) + c) * args.part_ld + m] = sum;
+            sum = 0.f;
+          }
         } else {
           const int col = n0 + c * 32;
+          const bool diag = args.tri == TRI_DIAG_STORE;
           const float scale = (args.tri == TRI_LOWER_STORE && nb < (mb >> 1)) ? 2.0f : 1.0f;
           if (m < args.M) {
-            __nv_bfloat16* crow = args.C + (long long)m * args.ldC + col;
+            __nv_bfloat16* crow = args.C + (long long)m * args.ldC + (diag ? col - n0 : col);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               if (col + v * 8 < args.N) {
+                // TRI_DIAG_STORE keeps only entries of the row's own quantisation group
+                const float keep = (!diag || (m / args.group) == ((col + v * 8) / args.group)) ? scale : 0.0f;
                 uint32_t w[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                  __nv_bfloat162 p = __floats2bfloat162_rn(scale * __uint_as_float(r[v * 8 + 2 * h]),
-                                                           scale * __uint_as_float(r[v * 8 + 2 * h + 1]));
+                  __nv_bfloat162 p = __floats2bfloat162_rn(keep * __uint_as_float(r[v * 8 + 2 * h]),
+                                                           keep * __uint_as_float(r[v * 8 + 2 * h + 1]));
                   w[h] = *reinterpret_cast<uint32_t*>(&p);
                 }
                 *reinterpret_cast<uint4*>(crow + v * 8) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -386,7 +406,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(acc));
-      if constexpr (MODE != EPI_STORE) {
+      if constexpr (MODE == EPI_SUMSQ || MODE == EPI_DOT) {
         if (m < args.M) args.part[(long long)nb * args.part_ld + m] = sum;
       }
     }
