@@ -11,16 +11,19 @@ Pages cited (by title and section):
   [P1] "AWQ量化" tutorial (aiqz.cc): 量化基础 (uniform quantiser), 激活感知
        (importance Omega_i), 缩放保护 (scale-quantise-restore), 误差分析,
        GPTQ对比 (AWQ objective).
-  [P2] "AWQ量化技术解析：激活感知的权重量化革命" (kwkr.cn): §2.1 (INT4 clip to
-       [-8, 7], fp16 scale), §4.2 (two 4-bit values per byte).
-  [P3] "大模型的开发应用（十八）：大模型量化：GPTQ与AWQ" (ewbang.com): AWQ 二.2
-       (grid search of alpha on [0, 1]).
+  [P2] "AWQ量化技术解析：激活感知的权重量化革命" (kwkr.cn): §1.2 (dequantise
+       on the fly, W_int4 x scale_fp16), §2.1 (INT4 clip to [-8, 7], fp16
+       scale), §4.2 (two 4-bit values per byte).
+  [P3] "大模型的开发应用（十八）：大模型量化：GPTQ与AWQ" (ewbang.com): AWQ 二.1
+       (the layer computes Q(W s)(X / s)), 二.2 (grid search of alpha on
+       [0, 1]), 二.3 (INT4 storage, dequantised for the product).
   [P4] "AWQ 量化全流程拆解：将 70B 大模型塞进单张消费级 GPU" (lnrq.cn): §三
        quant_config (zero_point, q_group_size = 128, w_bit = 4).
   [P5] "AWQ" (scholia-log, inference-quantization/2_AWQ): §1.1 (Delta Y =
        Delta W X), §1.2 (a_i = E|x_i|), §2.1 (W X = (W S)(S^-1 X)), §2.3
        (Q(w) = Delta round(w / Delta)), §3.1-3.3 (worked examples, groups),
-       §4.1 (s_i = a_i^alpha and the boxed objective).
+       §4.1 (s_i = a_i^alpha and the boxed objective), §4.3 (diagonal S:
+       S^-1 folds into the adjacent norm or linear layer).
 
 Conventions. W is [d_out, d_in] (rows are output channels), X is [N, d_in]
 (tokens x input channels), so the layer output for token t is W x_t and the
@@ -382,3 +385,73 @@ def boundary_mask(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symm
         zn = np.abs(rz - np.floor(rz) - 0.5) < band
         near |= zn[..., None]
     return near.reshape(rows, d_in)
+
+
+# ---------------------------------------------------------------------------
+# inference side: S^-1 folded into the producer of X, dequantisation of the
+# packed format, and the W4A16 product
+# ---------------------------------------------------------------------------
+def to_bf16_bits(x32: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns, round to nearest even (NaN stays NaN)."""
+    u = np.asarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    rounded = (u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    nan = np.isnan(np.asarray(x32, dtype=np.float32))
+    out = rounded.astype(np.uint16)
+    out[nan] = ((u[nan] >> np.uint64(16)) | np.uint64(0x40)).astype(np.uint16)
+    return out
+
+
+def fold_inv_scales(p_bits: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """Absorb S^-1 into the operation that produces X.
+
+    [P5] §4.3 (why S is diagonal): S^-1 x is a per-channel scaling that can be
+    folded into the adjacent LayerNorm or Linear, so X' = X S^-1 costs nothing
+    at run time; [P3] AWQ 二.1: the layer then computes Q(W s)(X / s).
+    p_bits holds that producer's bf16 parameters with the channel on the
+    first axis: a norm's weight or bias [d_in], or the previous linear
+    layer's weight [d_in, d_prev] / bias [d_in]. Entry (i, ...) becomes
+    p / s_i, rounded to bf16. Reading: the quotient is taken in float32 (the
+    kernel's precision; float32 division is correctly rounded on both sides),
+    so the bf16 rounding decides the same value on both sides.
+    """
+    p = widen_bf16(p_bits).astype(np.float32)
+    s32 = np.asarray(s, dtype=np.float32)
+    shape = (-1,) + (1,) * (p.ndim - 1)
+    return to_bf16_bits(p / s32.reshape(shape))
+
+
+def unpack_codes(qweight: np.ndarray, d_in: int) -> np.ndarray:
+    """Inverse of pack_codes: code of channel 8w+j = bits 4j..4j+3 of word w."""
+    q = np.asarray(qweight).view(np.uint32).astype(np.uint64)
+    rows = q.shape[0]
+    codes = np.zeros((rows, d_in), dtype=np.int64)
+    for j in range(8):
+        codes[:, j::8] = ((q >> np.uint64(4 * j)) & np.uint64(0xF)).astype(np.int64)
+    return codes
+
+
+def dequant_packed(qweight: np.ndarray, scales_f16: np.ndarray, zeros_f16: np.ndarray, group: int,
+                   d_in: int) -> np.ndarray:
+    """W_hat[r, i] = (code - z) * Delta of the group, from the stored format.
+
+    [P2] §1.2: the weights are dequantised on the fly as W_int4 x scale_fp16;
+    with a zero point (asymmetric, [P4] §三 zero_point) the code is first
+    offset by z. Symmetric codes are stored as q + 2^(b-1) with zero 2^(b-1)
+    (this library's layout), so the same formula covers both quantisers.
+    The result is W_hat = Q(W S) in the scaled space (float64, exact from the
+    fp16 step and zero point)."""
+    codes = unpack_codes(qweight, d_in).astype(np.float64)
+    delta = np.repeat(np.asarray(scales_f16, dtype=np.float64), group, axis=1)
+    zero = np.repeat(np.asarray(zeros_f16, dtype=np.float64), group, axis=1)
+    return (codes - zero) * delta
+
+
+def w4a16_matmul(Xp_bits: np.ndarray, qweight: np.ndarray, scales_f16: np.ndarray, zeros_f16: np.ndarray,
+                 group: int) -> np.ndarray:
+    """Y[t, o] = sum_i X'[t, i] W_hat[o, i]: the quantised layer applied to
+    activations that already carry S^-1 ([P5] §2.1 W X = (W S)(S^-1 X);
+    [P3] AWQ 二.3: weights stored in INT4, dequantised for the product).
+    Float64, exact products of the bf16 activations and the dequantised weights."""
+    Xp = widen_bf16(Xp_bits)
+    W_hat = dequant_packed(qweight, scales_f16, zeros_f16, group, Xp.shape[1])
+    return Xp @ W_hat.T

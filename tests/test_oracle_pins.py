@@ -534,3 +534,124 @@ def test_group_clip_errors_brute_force():
     best = O.group_clip_choice(err)
     assert best.shape == (3, 2)
     assert np.all(err[best, np.arange(3)[:, None], np.arange(2)[None, :]] <= err[0] + 0.0)
+
+
+# ---------------------------------------------------------------------------
+# inference side: fold, unpack, dequantise, W4A16 product
+# ---------------------------------------------------------------------------
+def test_bf16_rounding_matches_torch():
+    """to_bf16_bits is round-to-nearest-even; torch's CPU float32 -> bfloat16
+    conversion is the library routine it must equal (ties included)."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(30)
+    x = (rng.standard_normal(20000) * np.exp(rng.standard_normal(20000) * 4)).astype(np.float32)
+    ties = (np.arange(1, 2001, dtype=np.uint32) << np.uint32(16)) | np.uint32(0x8000)  # exact midpoints
+    x = np.concatenate([x, ties.view(np.float32), np.array([0.0, -0.0, np.inf, -np.inf], dtype=np.float32)])
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.to_bf16_bits(x), ref)
+
+
+def test_fold_matches_library_and_special_cases():
+    """p / s_i per channel (first axis), fp32 quotient rounded to bf16: equals
+    torch's float32 division + bfloat16 rounding; s = 1 leaves p unchanged and a
+    power-of-two s only moves the exponent."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(31)
+    p = gen.f64_to_bf16_bits(rng.standard_normal((64, 24)))
+    s = np.exp(rng.standard_normal(64)).astype(np.float32)
+    ref = (torch.from_numpy(O.widen_bf16(p).astype(np.float32)) / torch.from_numpy(s)[:, None]).to(torch.bfloat16)
+    assert np.array_equal(O.fold_inv_scales(p, s), ref.view(torch.int16).numpy().view(np.uint16))
+    vec = p[:, 0]
+    assert np.array_equal(O.fold_inv_scales(vec, np.ones(64, dtype=np.float32)), vec)
+    folded = O.widen_bf16(O.fold_inv_scales(vec, np.full(64, 4.0, dtype=np.float32)))
+    assert np.array_equal(folded, O.widen_bf16(vec) / 4.0)
+
+
+def test_unpack_inverts_pack_codes():
+    rng = np.random.default_rng(32)
+    codes = rng.integers(0, 16, size=(5, 64))
+    assert np.array_equal(O.unpack_codes(O.pack_codes(codes), 64), codes)
+
+
+@pytest.mark.parametrize("symmetric,bits", [(False, 4), (True, 4), (False, 3), (True, 2)])
+def test_dequant_of_pack_is_fake_quant_up_to_fp16_step(symmetric, bits):
+    """dequant_packed(pack(W, s)) reproduces Q(W S) from quantize_groups, and
+    the difference is exactly (code - z)(fp16(Delta) - Delta): the zero point
+    is an integer <= 15, exact in fp16, so the fp16 step is the only rounding."""
+    rng = np.random.default_rng(33 + bits)
+    Wb = gen.f64_to_bf16_bits(rng.standard_normal((6, 256)) * 0.02)
+    s = np.exp(rng.standard_normal(256) * 0.5)
+    qw, sc, zr, codes, delta, zero = O.pack(Wb, s, bits, 64, symmetric)
+    Vh = O.quantize_groups(O.widen_bf16(Wb) * s[None, :], bits, 64, symmetric)[0]
+    deq = O.dequant_packed(qw, sc, zr, 64, 256)
+    assert np.array_equal(zr.astype(np.float64), zero)
+    expected = (codes - np.repeat(zero, 64, axis=1)) * np.repeat(sc.astype(np.float64) - delta, 64, axis=1)
+    assert np.allclose(deq - Vh, expected, rtol=0, atol=1e-12 * np.abs(Vh).max())
+    assert np.all(np.abs(deq - Vh) <= (2 ** bits - 1) * 2.0 ** -11 * np.repeat(delta, 64, axis=1) + 1e-15)
+
+
+def test_w4a16_exact_on_the_grid():
+    """Weights already on the asymmetric grid with a power-of-two step (every
+    group holds codes 0 and 15) and s = 1: the pack is lossless, so the
+    quantised layer equals the plain product."""
+    rng = np.random.default_rng(34)
+    rows, d_in, g = 8, 128, 32
+    codes = rng.integers(0, 16, size=(rows, d_in))
+    codes[:, ::g] = 0
+    codes[:, 1::g] = 15
+    z = rng.integers(1, 15, size=(rows, d_in // g))
+    W = (codes - np.repeat(z, g, axis=1)) * 2.0 ** -6
+    Wb = gen.f64_to_bf16_bits(W)
+    assert np.array_equal(O.widen_bf16(Wb), W)
+    qw, sc, zr, c2, _, _ = O.pack(Wb, np.ones(d_in), 4, g, False)
+    assert np.array_equal(c2, codes)
+    Xb = gen.f64_to_bf16_bits(rng.standard_normal((5, d_in)))
+    Y = O.w4a16_matmul(Xb, qw, sc, zr, g)
+    assert np.allclose(Y, O.widen_bf16(Xb) @ W.T, rtol=1e-13, atol=0)
+
+
+def test_w4a16_brute_force():
+    """Triple loop with the nibbles taken out of the words one by one."""
+    rng = np.random.default_rng(35)
+    rows, d_in, g, N = 3, 32, 16, 2
+    Wb = gen.f64_to_bf16_bits(rng.standard_normal((rows, d_in)) * 0.1)
+    qw, sc, zr, _, _, _ = O.pack(Wb, np.ones(d_in), 4, g, False)
+    Xb = gen.f64_to_bf16_bits(rng.standard_normal((N, d_in)))
+    X = O.widen_bf16(Xb)
+    Y = O.w4a16_matmul(Xb, qw, sc, zr, g)
+    words = qw.view(np.uint32)
+    for t in range(N):
+        for o in range(rows):
+            acc = 0.0
+            for i in range(d_in):
+                code = (int(words[o, i // 8]) >> (4 * (i % 8))) & 0xF
+                acc += X[t, i] * (code - float(zr[o, i // g])) * float(sc[o, i // g])
+            assert Y[t, o] == pytest.approx(acc, rel=1e-12, abs=1e-14)
+
+
+def test_p5_worked_example_through_the_inference_path():
+    """AWQ (scholia-log) §3.1 数值例子, run the way a deployed layer runs it:
+    symmetric INT4 group with w_max = 1 and w_i = 0.05 (x_i = 10). Unscaled, the
+    code of w_i is 0 and the output error is -0.5; with s_i = 4 folded into the
+    activation (x' = 2.5) and the stored fp16 step, the output error is the
+    printed -0.143."""
+    ex = GOLD["int4_group_example"]
+    d_in = 8
+    W = np.zeros((1, d_in))
+    W[0, 0], W[0, 1] = ex["w_max"], ex["w_i"]
+    Wb = gen.f64_to_bf16_bits(W)
+    x = np.zeros((1, d_in))
+    x[0, 1] = ex["x_i"]
+    xb = gen.f64_to_bf16_bits(x)
+    y_true = float((O.widen_bf16(xb) @ O.widen_bf16(Wb).T)[0, 0])
+    for s_i, code, dy, tol in ((1.0, ex["unscaled_code"], ex["unscaled_dy"], 1e-3),
+                               (ex["s_i"], ex["scaled_code"], ex["scaled_dy_printed"], 5e-4)):
+        s = np.ones(d_in, dtype=np.float32)
+        s[1] = s_i
+        qw, sc, zr, codes, _, _ = O.pack(Wb, s.astype(np.float64), ex["bits"], d_in, True)
+        assert codes[0, 1] - zr[0, 0] == code
+        assert float(sc[0, 0]) == pytest.approx(ex["delta_printed"], abs=5e-4)
+        xp = O.fold_inv_scales(xb.T, s).T  # the producer of x carries 1/s
+        assert O.widen_bf16(xp)[0, 1] == pytest.approx(ex["x_i"] / s_i)
+        y = float(O.w4a16_matmul(xp, qw, sc, zr, d_in)[0, 0])
+        assert y - y_true == pytest.approx(dy, abs=tol)
