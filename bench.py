@@ -336,6 +336,62 @@ def run_ours(args, rank, world, local_rank):
                  "note": "search_group_clip + quantize_pack_group_clip with s_best, " + str(KB) + " passes, L2 flushed"}
         del cws
 
+    # ---- inference side: the packed layer applied by the W4A16 kernel (timed apart from the step)
+    w4 = None
+    if d_in % 32 == 0 and not args.no_w4a16:
+        pk = awq.quantize_pack(W, outs["s_best"], cfg)
+        Xt = X.t().contiguous()
+        awq.fold_inv_scales(outs["s_best"], Xt)  # activations carrying S^-1
+        Xp_all = Xt.t().contiguous()
+        del Xt
+        peaks_ = load_peaks()
+        hbm_ = peaks_.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        tc_ = peaks_.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        w4 = {}
+        for label, n_tok in (("decode_16", 16), ("prefill_N", N)):
+            Xp = Xp_all[:n_tok].contiguous()
+            wsw = awq.workspace(awq.w4a16_workspace_size(n_tok, d_out, d_in, cfg))
+            Yw = torch.empty((n_tok, d_out), dtype=torch.bfloat16, device=dev)
+
+            def run_w4():
+                awq.w4a16_gemm(Xp, *pk, cfg, ws=wsw, out=Yw)
+
+            def run_dense():
+                torch.matmul(Xp, W.t(), out=Yw)
+
+            res = {}
+            for nm, fn in (("w4a16", run_w4), ("bf16_dense_cublas", run_dense)):
+                for _ in range(3):
+                    fn()
+                torch.cuda.synchronize()
+                tms = []
+                for k in range(KB):
+                    flush.fill_(k & 0xFF)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    fn()
+                    e1.record()
+                    e1.synchronize()
+                    tms.append(e0.elapsed_time(e1))
+                res[nm] = float(np.mean(tms))
+            awq.workspace_error(wsw)
+            byts = d_out * d_in // 2 + 4 * d_out * ng + n_tok * d_in * 2 + n_tok * d_out * 2
+            flops = 2.0 * n_tok * d_out * d_in
+            ms = res["w4a16"]
+            entry = {"tokens": n_tok, "ms": round(ms, 4), "bf16_dense_cublas_ms": round(res["bf16_dense_cublas"], 4),
+                     "speedup_vs_bf16_dense": round(res["bf16_dense_cublas"] / ms, 3),
+                     "gbs": round(byts / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(byts / (ms * 1e-3) / 1e9 / hbm_, 4),
+                     "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                     "tensor_frac": round(flops / (ms * 1e-3) / 1e12 / tc_, 4),
+                     "algorithmic_bytes": int(byts), "flops": flops}
+            entry["bound"] = "hbm" if flops / byts < tc_ * 1e12 / (hbm_ * 1e9) else "tensor"
+            w4[label] = entry
+            del wsw, Yw, Xp
+        w4["note"] = ("awq_w4a16_gemm on this layer's packed weights (s_best), activations folded by "
+                      "awq_fold_inv_scales; " + str(KB) + " runs each, L2 flushed; cuBLAS bf16 dense on the "
+                      "unquantised W for context")
+        del Xp_all, pk
+
     peaks = load_peaks()
     n_a = wl.n_alpha
     flops_direct = 2.0 * n_a * d_out * d_in * N
@@ -389,11 +445,56 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(world * n_a * K / (e2e_total * 1e-3), 2), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "group_clip": gclip,
+        "w4a16": w4,
         "gpu_launches": launches_per_step(form, n_a) * K,
         "clocks": clk,
         "wall_s_timed_region": round(t_wall, 3),
     }
     return line
+
+
+# ----------------------------------------------------------------------------- W4A16 alone
+def run_w4a16_only(args):
+    """The W4A16 kernel alone on the workload's layer shape with `--tokens`
+    tokens: W packed at s = 1 by the library's own pack, activations from the
+    workload's generator. For profiling the kernel on its own."""
+    import torch
+    import weight_only_int4_act_b200 as awq
+    from awq_inputs import gen
+
+    wl = WORKLOADS[args.config]
+    dev = torch.device("cuda", 0)
+    Wb = gen.make_weight(wl.seed, wl.d_out, wl.d_in, wl.w_std)
+    Xb = gen.make_activations(wl.seed, args.tokens, wl.d_in, wl.x_kind, wl.x_lognormal_sigma, wl.outlier_count,
+                              wl.outlier_factor)
+    W = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).to(dev)
+    X = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).to(dev)
+    cfg = awq.make_cfg(wl.bits, wl.group, wl.symmetric, 1)
+    pk = awq.quantize_pack(W, torch.ones(wl.d_in, dtype=torch.float32, device=dev), cfg)
+    ws = awq.workspace(awq.w4a16_workspace_size(args.tokens, wl.d_out, wl.d_in, cfg))
+    Y = torch.empty((args.tokens, wl.d_out), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        awq.w4a16_gemm(X, *pk, cfg, ws=ws, out=Y)
+    torch.cuda.synchronize()
+    ms = []
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        awq.w4a16_gemm(X, *pk, cfg, ws=ws, out=Y)
+        e1.record()
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    awq.workspace_error(ws)
+    t = float(np.mean(ms))
+    byts = wl.d_out * wl.d_in // 2 + 4 * wl.d_out * (wl.d_in // wl.group) + args.tokens * (wl.d_in + wl.d_out) * 2
+    return {"metric": "W4A16 product (awq_w4a16_gemm)", "value": round(t, 4), "unit": "ms",
+            "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
+            "config": {"workload": f"{wl.key} layer {wl.d_out}x{wl.d_in}, {args.tokens} tokens",
+                       "bits": wl.bits, "group": wl.group, "l2": "flushed between runs"},
+            "gbs": round(byts / (t * 1e-3) / 1e9, 1),
+            "tflops": round(2.0 * args.tokens * wl.d_out * wl.d_in / (t * 1e-3) / 1e12, 2)}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -474,6 +575,9 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-group-clip", action="store_true", help="skip the per-group clipping pass")
+    ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 inference-side timing")
+    ap.add_argument("--only", default=None, choices=["w4a16"], help="time one component alone (its own JSON line)")
+    ap.add_argument("--tokens", type=int, default=16, help="tokens for --only w4a16")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -482,6 +586,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = WORKLOADS[args.config]
+
+    if args.only == "w4a16":
+        if rank == 0:
+            print(json.dumps(run_w4a16_only(args)), flush=True)
+        return
 
     if args.impl == "reference":
         if rank == 0:

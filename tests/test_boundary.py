@@ -169,3 +169,32 @@ def test_group_clip_validation():
     assert pk(FAKE, FAKE, cp, 4, None, 256, 512, c, FAKE, FAKE, FAKE, None) == 1
     assert pk(FAKE, FAKE, ctypes.cast(bad, ctypes.c_void_p), 4, FAKE, 256, 512, c, FAKE, FAKE, FAKE, None) == 1
     assert pk(FAKE, FAKE, cp, 4, FAKE, 256, 500, c, FAKE, FAKE, FAKE, None) == 2
+
+
+def test_w4a16_and_fold_validation():
+    lib = awq.lib()
+    big = 1 << 40
+    cfg = awq.make_cfg(4, 128, False, 1)
+    c = ctypes.byref(cfg)
+    # decode shape: few output tiles, so K is split and the workspace holds fp32 partials
+    small = awq.w4a16_workspace_size(1, 256, 4096, cfg)
+    assert small > 1024 + 256 * 4
+    assert awq.w4a16_workspace_size(4096, 4096, 4096, cfg) == 1024  # enough tiles: no split, error word only
+    assert awq.w4a16_workspace_size(16, 256, 4112, cfg) == 0      # d_in not a multiple of 32 / of g
+    assert awq.w4a16_workspace_size(16, 256, 4096, awq.make_cfg(5, 128, False, 1)) == 0
+    assert awq.w4a16_workspace_size(0, 256, 4096, cfg) == 0
+
+    def call(X=FAKE, q=FAKE, sc=FAKE, zr=FAKE, N=1, d_out=256, d_in=4096, cfg_=cfg, Y=FAKE, ws=FAKE, wsb=big):
+        return lib.awq_w4a16_gemm(X, q, sc, zr, N, d_out, d_in, ctypes.byref(cfg_), Y, ws, wsb, None)
+    assert call(d_in=4000) == 2
+    assert call(N=0) == 2
+    assert call(cfg_=awq.make_cfg(4, 96, False, 1)) == 1
+    assert call(X=None) == 1
+    assert call(Y=None) == 1
+    assert call(ws=None) == 1
+    assert call(X=ctypes.c_void_p(0x10008)) == 1   # activations must be 16-byte aligned (TMA)
+    assert call(wsb=small - 1) == 3
+    # fold
+    assert lib.awq_fold_inv_scales(None, 16, FAKE, 1, None) == 1
+    assert lib.awq_fold_inv_scales(FAKE, 0, FAKE, 1, None) == 2
+    assert lib.awq_fold_inv_scales(FAKE, 16, FAKE, 0, None) == 2

@@ -9,7 +9,7 @@ ROOT = os.path.dirname(PKG)
 LIB_DIR = os.path.join(PKG, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libawq_b200.so")
 SOURCES = [os.path.join(PKG, "csrc", "awq_api.cu")]
-DEPS = SOURCES + [os.path.join(PKG, "csrc", f) for f in ("ptx.cuh", "fq.cuh", "gemm_sm100.cuh", "gemm_pair_sm100.cuh", "awq_kernels.cuh")] + [
+DEPS = SOURCES + [os.path.join(PKG, "csrc", f) for f in ("ptx.cuh", "fq.cuh", "gemm_sm100.cuh", "gemm_pair_sm100.cuh", "awq_kernels.cuh", "w4a16_sm100.cuh")] + [
     os.path.join(ROOT, "include", "awq.h")]
 
 NVCC_FLAGS = [

@@ -26,7 +26,7 @@ EXPORTED = (
     "awq_step_scales", "awq_step_fake_quant", "awq_step_gram", "awq_step_contract", "awq_step_reduce",
     "awq_debug_copy_dw", "awq_act_stats_noalloc", "awq_search_scales_segmented", "awq_search_candidates",
     "awq_quantize_pack_clipped", "awq_group_clip_workspace_size", "awq_search_group_clip",
-    "awq_quantize_pack_group_clip",
+    "awq_quantize_pack_group_clip", "awq_fold_inv_scales", "awq_w4a16_workspace_size", "awq_w4a16_gemm",
 )
 
 
@@ -85,6 +85,10 @@ def lib() -> ctypes.CDLL:
                                                 cfgp, c_void_p, c_size_t, c_void_p, c_void_p, c_void_p]),
             "awq_quantize_pack_group_clip": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_int64,
                                                        c_int64, cfgp, c_void_p, c_void_p, c_void_p, c_void_p]),
+            "awq_fold_inv_scales": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_void_p]),
+            "awq_w4a16_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, cfgp]),
+            "awq_w4a16_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, cfgp,
+                                         c_void_p, c_void_p, c_size_t, c_void_p]),
             "awq_workspace_error": (c_int32, [c_void_p, c_void_p]),
             "awq_quantize_pack": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_void_p, c_void_p,
                                             c_void_p, c_void_p]),
@@ -311,6 +315,46 @@ def quantize_pack_group_clip(W, s, clips, best_clip, cfg: QCfg, outputs=None):
                                               _ptr(best_clip), d_out, d_in, ctypes.byref(cfg), _ptr(q), _ptr(sc),
                                               _ptr(zr), _stream()), "awq_quantize_pack_group_clip")
     return q, sc, zr
+
+
+# --------------------------------------------------------------------------- inference side
+def fold_inv_scales(s, p):
+    """In place: row i of p (bf16 [d_in] or [d_in, inner], CUDA) becomes p / s_i."""
+    torch = _torch()
+    _req(s, torch.float32, None, "s")
+    _req(p, torch.bfloat16, None, "p")
+    d_in = s.numel()
+    if p.shape[0] != d_in:
+        raise ValueError("p must have the channel (length of s) on its first axis")
+    inner = p.numel() // d_in if d_in else 0
+    _check(lib().awq_fold_inv_scales(_ptr(s), d_in, _ptr(p), inner, _stream()), "awq_fold_inv_scales")
+    return p
+
+
+def w4a16_workspace_size(N, d_out, d_in, cfg: QCfg) -> int:
+    return int(lib().awq_w4a16_workspace_size(N, d_out, d_in, ctypes.byref(cfg)))
+
+
+def w4a16_gemm(Xp, qweight, scales, zeros, cfg: QCfg, ws=None, out=None):
+    """Y bf16 [N, d_out] = X' (bf16 [N, d_in]) times the dequantised packed weights."""
+    torch = _torch()
+    _req(Xp, torch.bfloat16, None, "X")
+    N, d_in = Xp.shape
+    _req(qweight, torch.int32, None, "qweight")
+    d_out = qweight.shape[0]
+    if qweight.shape != (d_out, d_in // 8):
+        raise ValueError("qweight must be [d_out, d_in/8]")
+    ng = d_in // cfg.group if cfg.group > 0 else 0
+    _req(scales, torch.float16, (d_out, ng), "scales")
+    _req(zeros, torch.float16, (d_out, ng), "zeros")
+    if ws is None:
+        ws = workspace(max(w4a16_workspace_size(N, d_out, d_in, cfg), 256))
+    if out is None:
+        out = torch.empty((N, d_out), dtype=torch.bfloat16, device=Xp.device)
+    _req(out, torch.bfloat16, (N, d_out), "out")
+    _check(lib().awq_w4a16_gemm(_ptr(Xp), _ptr(qweight), _ptr(scales), _ptr(zeros), N, d_out, d_in,
+                                ctypes.byref(cfg), _ptr(out), _ptr(ws), ws.numel(), _stream()), "awq_w4a16_gemm")
+    return out
 
 
 def workspace_error(ws):

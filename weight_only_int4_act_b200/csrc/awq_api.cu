@@ -13,6 +13,7 @@
 #include "awq_kernels.cuh"
 #include "gemm_pair_sm100.cuh"
 #include "gemm_sm100.cuh"
+#include "w4a16_sm100.cuh"
 
 using namespace awq;
 
@@ -197,6 +198,22 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2-D uint32 map over the packed codes [rows, words] (no swizzle), box of
+// box_words x box_rows.
+bool make_map_u32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t words, uint32_t box_words,
+                  uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {words, rows};
+  cuuint64_t strides[1] = {words * 4};
+  cuuint32_t box[2] = {box_words, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -787,5 +804,148 @@ extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t d_
       static_cast<const __nv_bfloat16*>(X), N, (int)d_in, L.rows_per_chunk, part);
   if ((st = launch_status()) != AWQ_OK) return st;
   act_absmean_final<<<(unsigned)cdiv(d_in, 256), 256, 0, s>>>(part, L.n_chunks, N, (int)d_in, a);
+  return launch_status();
+}
+
+// ===================================================================== inference side
+namespace {
+constexpr int kW4TargetCtas = 148;  // split K until the tiles cover this many CTAs
+
+struct W4Plan {
+  int bn, n_mb, n_nb, n_kb, splits, kb_per_split;
+  int as, xs, rs;  // ring depths
+  long long tiles, p_stride;
+  int smem;
+  size_t ws;
+};
+
+W4Plan w4_plan(int64_t N, int64_t d_out, int64_t d_in) {
+  W4Plan p{};
+  p.bn = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+  // ring depths: deep packed-code rings for narrow (weight-streaming) tiles
+  if (p.bn <= 32) { p.as = 4; p.xs = 8; p.rs = 24; }
+  else if (p.bn == 64) { p.as = 4; p.xs = 6; p.rs = 16; }
+  else if (p.bn == 128) { p.as = 4; p.xs = 4; p.rs = 16; }
+  else { p.as = 3; p.xs = 4; p.rs = 8; }
+  p.smem = w4_smem_bytes(p.as, p.xs, p.rs, p.bn);
+  p.n_mb = (int)cdiv(d_out, W4_BM);
+  p.n_nb = (int)cdiv(N, p.bn);
+  p.n_kb = (int)cdiv(d_in, W4_BK);
+  const long long mn = (long long)p.n_mb * p.n_nb;
+  int splits = 1;
+  if (mn < kW4TargetCtas) {
+    const long long want = cdiv(kW4TargetCtas, mn);
+    const int most = p.n_kb / 4 > 1 ? p.n_kb / 4 : 1;  // at least 4 K steps per split
+    splits = (int)(want < most ? want : most);
+  }
+  p.kb_per_split = (int)cdiv(p.n_kb, splits);
+  p.splits = (int)cdiv(p.n_kb, p.kb_per_split);
+  p.tiles = mn * p.splits;
+  p.p_stride = (N * d_out + 3) / 4 * 4;
+  p.ws = kAlign + (p.splits > 1 ? align_up((size_t)p.splits * p.p_stride * sizeof(float)) : 0);
+  return p;
+}
+
+awq_status check_w4(int64_t N, int64_t d_out, int64_t d_in, const awq_qcfg* cfg) {
+  if (!cfg) return AWQ_ERR_INVALID_ARG;
+  if (cfg->bits < 2 || cfg->bits > 4) return AWQ_ERR_INVALID_ARG;
+  const int g = cfg->group;
+  if (g < 8 || g > 256 || (g & (g - 1)) != 0) return AWQ_ERR_INVALID_ARG;
+  if (N < 1 || d_out < 1 || d_in < 32) return AWQ_ERR_SHAPE;
+  if (d_in % 32 != 0 || d_in % g != 0) return AWQ_ERR_SHAPE;  // packed rows: a multiple of 16 bytes
+  if (d_in > (1 << 20) || d_out > (1 << 24) || N > (1 << 24)) return AWQ_ERR_SHAPE;
+  if ((long long)N * d_out > (long long)INT32_MAX * 4) return AWQ_ERR_SHAPE;
+  if (w4_plan(N, d_out, d_in).tiles > INT32_MAX) return AWQ_ERR_SHAPE;
+  return AWQ_OK;
+}
+}  // namespace
+
+extern "C" size_t awq_w4a16_workspace_size(int64_t N, int64_t d_out, int64_t d_in, const awq_qcfg* cfg) {
+  if (check_w4(N, d_out, d_in, cfg) != AWQ_OK) return 0;
+  return w4_plan(N, d_out, d_in).ws;
+}
+
+extern "C" awq_status awq_w4a16_gemm(const void* X, const uint32_t* qweight, const void* scales, const void* zeros, int64_t N,
+                          int64_t d_out, int64_t d_in, const awq_qcfg* cfg, void* Y, void* ws, size_t ws_bytes,
+                          awq_stream_t stream) {
+  awq_status st = check_w4(N, d_out, d_in, cfg);
+  if (st != AWQ_OK) return st;
+  if (!X || !qweight || !scales || !zeros || !Y || !ws) return AWQ_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 2) || !aligned(zeros, 2) || !aligned(Y, 16) ||
+      !aligned(ws, 256))
+    return AWQ_ERR_INVALID_ARG;
+  const W4Plan p = w4_plan(N, d_out, d_in);
+  if (ws_bytes < p.ws) return AWQ_ERR_WORKSPACE;
+  int sms = 0;
+  if ((st = check_device(&sms)) != AWQ_OK) return st;
+  cudaStream_t cs = as_stream(stream);
+  CUtensorMap tx, tw;
+  if (!make_map(&tx, X, N, d_in, d_in, p.bn)) return AWQ_ERR_CUDA;
+  if (!make_map_u32(&tw, qweight, d_out, d_in / 8, W4_BK / 8, W4_BM)) return AWQ_ERR_CUDA;
+  W4Args a{};
+  a.N = (int)N;
+  a.d_out = (int)d_out;
+  a.d_in = (int)d_in;
+  a.bn = p.bn;
+  a.n_mb = p.n_mb;
+  a.n_nb = p.n_nb;
+  a.splits = p.splits;
+  a.kb_per_split = p.kb_per_split;
+  a.n_kb = p.n_kb;
+  a.num_tiles = (int)p.tiles;
+  a.ng = (int)(d_in / cfg->group);
+  int sh = 0;
+  while ((1 << sh) < cfg->group) ++sh;
+  a.group_shift = sh;
+  a.as = p.as;
+  a.xs = p.xs;
+  a.rs = p.rs;
+  if (p.smem > W4_SMEM_LIMIT) return AWQ_ERR_UNSUPPORTED;
+  a.scales = static_cast<const __half*>(scales);
+  a.zeros = static_cast<const __half*>(zeros);
+  a.Y = static_cast<__nv_bfloat16*>(Y);
+  a.P = p.splits > 1 ? at<float>(ws, kAlign) : nullptr;
+  a.p_stride = p.p_stride;
+  a.err = at<int>(ws, 0);
+  if (cudaMemsetAsync(ws, 0, sizeof(int), cs) != cudaSuccess) return AWQ_ERR_CUDA;
+  const int grid = (int)(p.tiles < sms ? p.tiles : sms);
+  auto launch = [&](auto kernel) -> awq_status {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem) != cudaSuccess)
+      return AWQ_ERR_CUDA;
+    kernel<<<grid, W4_THREADS, p.smem, cs>>>(tx, tw, a);
+    return launch_status();
+  };
+  switch (cfg->group) {
+    case 8: st = launch(w4a16_gemm_tcgen05<4>); break;
+    case 16: st = launch(w4a16_gemm_tcgen05<2>); break;
+    default: st = launch(w4a16_gemm_tcgen05<1>); break;
+  }
+  if (st != AWQ_OK) return st;
+  if (p.splits > 1) {
+    const long long n = N * d_out;
+    const long long blocks = cdiv(n / 4 > 0 ? n / 4 : 1, 256);
+    w4a16_split_reduce<<<(unsigned)(blocks < 4 * sms ? blocks : 4 * sms), 256, 0, cs>>>(a.P, p.splits, n,
+                                                                                       p.p_stride, a.Y);
+    return launch_status();
+  }
+  return AWQ_OK;
+}
+
+extern "C" awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p, int64_t inner, awq_stream_t stream) {
+  if (!s || !p) return AWQ_ERR_INVALID_ARG;
+  if (d_in < 1 || inner < 1 || d_in > (1 << 24) || inner > (1 << 24)) return AWQ_ERR_SHAPE;
+  if (!aligned(p, 2) || !aligned(s, 4)) return AWQ_ERR_INVALID_ARG;
+  int sms = 0;
+  awq_status st = check_device(&sms);
+  if (st != AWQ_OK) return st;
+  cudaStream_t cs = as_stream(stream);
+  const bool vec = inner % 8 == 0 && aligned(p, 16);
+  const long long units = d_in * inner / (vec ? 8 : 1);
+  const long long blocks = cdiv(units, 256);
+  const unsigned grid = (unsigned)(blocks < 8LL * sms ? blocks : 8LL * sms);
+  if (vec)
+    fold_inv_scales_kernel<8><<<grid, 256, 0, cs>>>(s, d_in, inner, static_cast<__nv_bfloat16*>(p));
+  else
+    fold_inv_scales_kernel<1><<<grid, 256, 0, cs>>>(s, d_in, inner, static_cast<__nv_bfloat16*>(p));
   return launch_status();
 }
