@@ -348,16 +348,19 @@ def run_ours(args, rank, world, local_rank):
         hbm_ = peaks_.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         tc_ = peaks_.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         w4 = {}
-        for label, n_tok in (("decode_16", 16), ("prefill_N", N)):
-            Xp = Xp_all[:n_tok].contiguous()
+        W16 = W.to(torch.float16)
+        for label, n_tok, dt in (("decode_16_f16", 16, torch.float16), ("prefill_N_f16", N, torch.float16),
+                                 ("decode_16_bf16", 16, torch.bfloat16), ("prefill_N_bf16", N, torch.bfloat16)):
+            Xp = Xp_all[:n_tok].to(dt).contiguous()
+            Wd = W16 if dt == torch.float16 else W
             wsw = awq.workspace(awq.w4a16_workspace_size(n_tok, d_out, d_in, cfg))
-            Yw = torch.empty((n_tok, d_out), dtype=torch.bfloat16, device=dev)
+            Yw = torch.empty((n_tok, d_out), dtype=dt, device=dev)
 
             def run_w4():
                 awq.w4a16_gemm(Xp, *pk, cfg, ws=wsw, out=Yw)
 
             def run_dense():
-                torch.matmul(Xp, W.t(), out=Yw)
+                torch.matmul(Xp, Wd.t(), out=Yw)
 
             res = {}
             for nm, fn in (("w4a16", run_w4), ("bf16_dense_cublas", run_dense)):
@@ -378,8 +381,9 @@ def run_ours(args, rank, world, local_rank):
             byts = d_out * d_in // 2 + 4 * d_out * ng + n_tok * d_in * 2 + n_tok * d_out * 2
             flops = 2.0 * n_tok * d_out * d_in
             ms = res["w4a16"]
-            entry = {"tokens": n_tok, "ms": round(ms, 4), "bf16_dense_cublas_ms": round(res["bf16_dense_cublas"], 4),
-                     "speedup_vs_bf16_dense": round(res["bf16_dense_cublas"] / ms, 3),
+            entry = {"tokens": n_tok, "activations": "fp16" if dt == torch.float16 else "bf16", "ms": round(ms, 4),
+                     "dense_cublas_ms": round(res["bf16_dense_cublas"], 4),
+                     "speedup_vs_dense": round(res["bf16_dense_cublas"] / ms, 3),
                      "gbs": round(byts / (ms * 1e-3) / 1e9, 1), "hbm_frac": round(byts / (ms * 1e-3) / 1e9 / hbm_, 4),
                      "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
                      "tensor_frac": round(flops / (ms * 1e-3) / 1e12 / tc_, 4),
@@ -388,9 +392,9 @@ def run_ours(args, rank, world, local_rank):
             w4[label] = entry
             del wsw, Yw, Xp
         w4["note"] = ("awq_w4a16_gemm on this layer's packed weights (s_best), activations folded by "
-                      "awq_fold_inv_scales; " + str(KB) + " runs each, L2 flushed; cuBLAS bf16 dense on the "
-                      "unquantised W for context")
-        del Xp_all, pk
+                      "awq_fold_inv_scales; " + str(KB) + " runs each, L2 flushed; cuBLAS dense GEMM of the "
+                      "same activation type on the unquantised W for context")
+        del Xp_all, pk, W16
 
     peaks = load_peaks()
     n_a = wl.n_alpha
@@ -469,10 +473,12 @@ def run_w4a16_only(args):
                               wl.outlier_factor)
     W = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).to(dev)
     X = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).to(dev)
+    if args.dtype == "f16":
+        X = X.to(torch.float16)
     cfg = awq.make_cfg(wl.bits, wl.group, wl.symmetric, 1)
     pk = awq.quantize_pack(W, torch.ones(wl.d_in, dtype=torch.float32, device=dev), cfg)
     ws = awq.workspace(awq.w4a16_workspace_size(args.tokens, wl.d_out, wl.d_in, cfg))
-    Y = torch.empty((args.tokens, wl.d_out), dtype=torch.bfloat16, device=dev)
+    Y = torch.empty((args.tokens, wl.d_out), dtype=X.dtype, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         awq.w4a16_gemm(X, *pk, cfg, ws=ws, out=Y)
@@ -492,7 +498,7 @@ def run_w4a16_only(args):
     return {"metric": "W4A16 product (awq_w4a16_gemm)", "value": round(t, 4), "unit": "ms",
             "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
             "config": {"workload": f"{wl.key} layer {wl.d_out}x{wl.d_in}, {args.tokens} tokens",
-                       "bits": wl.bits, "group": wl.group, "l2": "flushed between runs"},
+                       "bits": wl.bits, "group": wl.group, "activations": args.dtype, "l2": "flushed between runs"},
             "gbs": round(byts / (t * 1e-3) / 1e9, 1),
             "tflops": round(2.0 * args.tokens * wl.d_out * wl.d_in / (t * 1e-3) / 1e12, 2)}
 
@@ -578,6 +584,7 @@ def main():
     ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 inference-side timing")
     ap.add_argument("--only", default=None, choices=["w4a16"], help="time one component alone (its own JSON line)")
     ap.add_argument("--tokens", type=int, default=16, help="tokens for --only w4a16")
+    ap.add_argument("--dtype", default="f16", choices=["f16", "bf16"], help="activations for --only w4a16")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -237,38 +237,45 @@ awq_status awq_quantize_pack_group_clip(const void* W_bf16, const float* s, cons
 /* ---------------------------------------------------------------------------
  * Inference side: the quantised layer as it runs after calibration.
  * ------------------------------------------------------------------------- */
+/* 16-bit floating-point types of the inference-side calls. */
+typedef enum awq_dtype { AWQ_DTYPE_BF16 = 0, AWQ_DTYPE_F16 = 1 } awq_dtype;
+
 /* Fold S^-1 into the operation that produces X ("AWQ" (scholia-log) §4.3: a
  * diagonal S^-1 is absorbed by the adjacent LayerNorm or Linear, so the
  * layer computes Q(W S)(S^-1 X) at no extra cost). p is that operation's bf16
  * parameter block with the channel on the first axis, DEVICE [d_in, inner]
- * row-major, updated in place: p[i, j] <- bf16(p[i, j] / s[i]), the quotient
- * in fp32 (correctly rounded) and rounded to nearest even. inner = 1 for a
+ * row-major, bf16 or fp16 (dtype), updated in place: p[i, j] <- p[i, j] /
+ * s[i], the quotient in fp32 (correctly rounded) and rounded to nearest even
+ * in the same type. inner = 1 for a
  * norm's weight or bias, d_prev for the previous linear layer's weight
  * [d_in, d_prev]. s is DEVICE float [d_in]; a non-positive or non-finite s_i
  * gives the IEEE quotient (no check). Asynchronous. */
-awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p_bf16, int64_t inner, awq_stream_t stream);
+awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p, awq_dtype dtype, int64_t inner,
+                               awq_stream_t stream);
 
 /* W4A16 product reading the packed format ("AWQ量化技术解析" (kwkr.cn) §1.2,
  * §4.2: weights dequantised on the fly as W_int4 x scale_fp16, fused with the
- * GEMM; ewbang.com AWQ 二.3):
+ * GEMM; ewbang.com AWQ 二.3: dequantised to FP16 for the product):
  *   Y[t, o] = sum_i X'[t, i] * (code[o, i] - z[o, i/g]) * Delta[o, i/g]
- * X'      DEVICE bf16 [N, d_in] row-major, 16-byte aligned: activations that
- *         already carry S^-1 (awq_fold_inv_scales on their producer).
+ * X'      DEVICE [N, d_in] row-major, fp16 or bf16 (dtype), 16-byte aligned:
+ *         activations that already carry S^-1 (awq_fold_inv_scales on their
+ *         producer).
  * qweight, scales, zeros: the output of awq_quantize_pack* for this layer
  *         (DEVICE uint32 [d_out, d_in/8], fp16 [d_out, d_in/g] twice);
  *         cfg->bits and cfg->group describe them (cfg->n_alpha, form, eps_a
  *         and alphas are ignored; symmetric codes carry their zero point).
- * Y       DEVICE bf16 [N, d_out] row-major, 16-byte aligned.
- * The dequantised weights enter the tensor cores as bf16 ((code - z) Delta
- * is exact in fp32 and rounded once); accumulation is fp32; Y is rounded
- * once to bf16. Requires d_in a multiple of 32 and of g (AWQ_ERR_SHAPE).
+ * Y       DEVICE [N, d_out] row-major in the same type, 16-byte aligned.
+ * The dequantised weights enter the tensor cores in that type: fp16 rounds
+ * (code - z) * Delta once; bf16 rounds Delta to bf16 and then the product.
+ * Accumulation is fp32; Y is rounded once. Requires d_in a multiple of 32
+ * and of g (AWQ_ERR_SHAPE).
  * Workspace: awq_w4a16_workspace_size (error word, split-K partials when
  * there are fewer output tiles than SMs); AWQ_ERR_WORKSPACE if smaller.
  * Asynchronous; device-side errors land in the workspace (awq_workspace_error). */
 size_t awq_w4a16_workspace_size(int64_t N, int64_t d_out, int64_t d_in, const awq_qcfg* cfg);
-awq_status awq_w4a16_gemm(const void* X_bf16, const uint32_t* qweight, const void* scales_f16,
+awq_status awq_w4a16_gemm(const void* X, awq_dtype dtype, const uint32_t* qweight, const void* scales_f16,
                           const void* zeros_f16, int64_t N, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
-                          void* Y_bf16, void* ws, size_t ws_bytes, awq_stream_t stream);
+                          void* Y, void* ws, size_t ws_bytes, awq_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * The search, one step at a time (awq_search_scales is exactly these calls

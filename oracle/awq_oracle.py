@@ -401,23 +401,42 @@ def to_bf16_bits(x32: np.ndarray) -> np.ndarray:
     return out
 
 
-def fold_inv_scales(p_bits: np.ndarray, s: np.ndarray) -> np.ndarray:
+def widen_f16(bits: np.ndarray) -> np.ndarray:
+    """IEEE binary16 bit patterns (uint16) -> exact float64 values."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def to_f16_bits(x32: np.ndarray) -> np.ndarray:
+    """float32 -> binary16 bit patterns, round to nearest even (beyond the
+    fp16 range: infinity)."""
+    with np.errstate(over="ignore"):
+        return np.asarray(x32, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
+def widen(bits: np.ndarray, dtype: str) -> np.ndarray:
+    """16-bit patterns of type ``dtype`` ("bf16" or "f16") -> float64."""
+    return widen_bf16(bits) if dtype == "bf16" else widen_f16(bits)
+
+
+def fold_inv_scales(p_bits: np.ndarray, s: np.ndarray, dtype: str = "bf16") -> np.ndarray:
     """Absorb S^-1 into the operation that produces X.
 
     [P5] §4.3 (why S is diagonal): S^-1 x is a per-channel scaling that can be
     folded into the adjacent LayerNorm or Linear, so X' = X S^-1 costs nothing
     at run time; [P3] AWQ 二.1: the layer then computes Q(W s)(X / s).
-    p_bits holds that producer's bf16 parameters with the channel on the
-    first axis: a norm's weight or bias [d_in], or the previous linear
-    layer's weight [d_in, d_prev] / bias [d_in]. Entry (i, ...) becomes
-    p / s_i, rounded to bf16. Reading: the quotient is taken in float32 (the
-    kernel's precision; float32 division is correctly rounded on both sides),
-    so the bf16 rounding decides the same value on both sides.
+    p_bits holds that producer's parameters (bf16 or fp16 bit patterns, per
+    ``dtype``) with the channel on the first axis: a norm's weight or bias
+    [d_in], or the previous linear layer's weight [d_in, d_prev] / bias
+    [d_in]. Entry (i, ...) becomes p / s_i, rounded to the same type.
+    Reading: the quotient is taken in float32 (the kernel's precision;
+    float32 division is correctly rounded on both sides), so the final
+    rounding decides the same value on both sides.
     """
-    p = widen_bf16(p_bits).astype(np.float32)
+    p = widen(p_bits, dtype).astype(np.float32)
     s32 = np.asarray(s, dtype=np.float32)
     shape = (-1,) + (1,) * (p.ndim - 1)
-    return to_bf16_bits(p / s32.reshape(shape))
+    q = p / s32.reshape(shape)
+    return to_bf16_bits(q) if dtype == "bf16" else to_f16_bits(q)
 
 
 def unpack_codes(qweight: np.ndarray, d_in: int) -> np.ndarray:
@@ -447,11 +466,12 @@ def dequant_packed(qweight: np.ndarray, scales_f16: np.ndarray, zeros_f16: np.nd
 
 
 def w4a16_matmul(Xp_bits: np.ndarray, qweight: np.ndarray, scales_f16: np.ndarray, zeros_f16: np.ndarray,
-                 group: int) -> np.ndarray:
+                 group: int, dtype: str = "bf16") -> np.ndarray:
     """Y[t, o] = sum_i X'[t, i] W_hat[o, i]: the quantised layer applied to
     activations that already carry S^-1 ([P5] §2.1 W X = (W S)(S^-1 X);
-    [P3] AWQ 二.3: weights stored in INT4, dequantised for the product).
-    Float64, exact products of the bf16 activations and the dequantised weights."""
-    Xp = widen_bf16(Xp_bits)
+    [P3] AWQ 二.3: weights stored in INT4, dequantised to FP16 for the
+    product). Float64, exact products of the 16-bit activations (bf16 or fp16
+    per ``dtype``) and the dequantised weights."""
+    Xp = widen(Xp_bits, dtype)
     W_hat = dequant_packed(qweight, scales_f16, zeros_f16, group, Xp.shape[1])
     return Xp @ W_hat.T

@@ -184,8 +184,8 @@ def test_w4a16_and_fold_validation():
     assert awq.w4a16_workspace_size(16, 256, 4096, awq.make_cfg(5, 128, False, 1)) == 0
     assert awq.w4a16_workspace_size(0, 256, 4096, cfg) == 0
 
-    def call(X=FAKE, q=FAKE, sc=FAKE, zr=FAKE, N=1, d_out=256, d_in=4096, cfg_=cfg, Y=FAKE, ws=FAKE, wsb=big):
-        return lib.awq_w4a16_gemm(X, q, sc, zr, N, d_out, d_in, ctypes.byref(cfg_), Y, ws, wsb, None)
+    def call(X=FAKE, q=FAKE, sc=FAKE, zr=FAKE, N=1, d_out=256, d_in=4096, cfg_=cfg, Y=FAKE, ws=FAKE, wsb=big, dt=0):
+        return lib.awq_w4a16_gemm(X, dt, q, sc, zr, N, d_out, d_in, ctypes.byref(cfg_), Y, ws, wsb, None)
     assert call(d_in=4000) == 2
     assert call(N=0) == 2
     assert call(cfg_=awq.make_cfg(4, 96, False, 1)) == 1
@@ -194,7 +194,10 @@ def test_w4a16_and_fold_validation():
     assert call(ws=None) == 1
     assert call(X=ctypes.c_void_p(0x10008)) == 1   # activations must be 16-byte aligned (TMA)
     assert call(wsb=small - 1) == 3
+    assert call(dt=2) == 1                          # activation type: 0 bf16, 1 fp16
+    assert call(dt=1, wsb=small - 1) == 3
     # fold
-    assert lib.awq_fold_inv_scales(None, 16, FAKE, 1, None) == 1
-    assert lib.awq_fold_inv_scales(FAKE, 0, FAKE, 1, None) == 2
-    assert lib.awq_fold_inv_scales(FAKE, 16, FAKE, 0, None) == 2
+    assert lib.awq_fold_inv_scales(None, 16, FAKE, 0, 1, None) == 1
+    assert lib.awq_fold_inv_scales(FAKE, 16, FAKE, 2, 1, None) == 1
+    assert lib.awq_fold_inv_scales(FAKE, 0, FAKE, 1, 1, None) == 2
+    assert lib.awq_fold_inv_scales(FAKE, 16, FAKE, 0, 0, None) == 2

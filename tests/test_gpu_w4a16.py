@@ -2,11 +2,13 @@
 fold (bit-exact: both sides round the same fp32 quotient to bf16), and
 awq_w4a16_gemm against the oracle's W4A16 product on packed weights.
 
-Tolerance of the product: the kernel rounds each dequantised weight to bf16
-(exact (code - z) Delta, one rounding: relative u = 2^-8), accumulates in
-fp32 and rounds Y to bf16 (u again). So |Y_gpu - Y| <= u |Y| + (u + d_in
-2^-23) sum_i |X'_ti| |W_hat_oi| to first order (the second term also covers
-fp32 accumulation of d_in products); the test allows 1.1 times that."""
+Tolerance of the product, with u the unit roundoff of the activation type
+(fp16 2^-11, bf16 2^-8): the kernel rounds each dequantised weight once in
+fp16 ((code - z) Delta) and twice in bf16 (Delta, then the product), so the
+weight carries a relative error e_w <= u (fp16) or 2u (bf16); it accumulates
+in fp32 and rounds Y once more. So |Y_gpu - Y| <= u |Y| + (e_w + d_in 2^-23)
+sum_i |X'_ti| |W_hat_oi| to first order (the last term also covers fp32
+accumulation of d_in products); the test allows 1.1 times that."""
 import zlib
 
 import numpy as np
@@ -17,6 +19,10 @@ from oracle import awq_oracle as O
 
 from gpu_util import to_device
 
+
+def to_device_f16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.float16).cuda()
+
 pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
@@ -25,7 +31,9 @@ if not torch.cuda.is_available():  # pragma: no cover
 
 import weight_only_int4_act_b200 as awq  # noqa: E402
 
-U = 2.0 ** -8
+UNIT = {"bf16": 2.0 ** -8, "f16": 2.0 ** -11}
+W_ERR = {"bf16": 2, "f16": 1}   # roundings of the dequantised weight, in units of u
+DTYPES = ["bf16", "f16"]
 
 CASES = [
     # name, N, d_out, d_in, bits, group, symmetric
@@ -40,35 +48,45 @@ CASES = [
 ]
 
 
-def _scaled_layer(N, d_out, d_in, bits, group, symmetric, seed):
+def _scaled_layer(N, d_out, d_in, bits, group, symmetric, seed, dtype="bf16"):
+    """W, X (bf16 bits), X' = X S^-1 in `dtype` (bits), s (fp32)."""
     wl = custom(d_out, d_in, N, bits=bits, symmetric=symmetric, group=group, seed=seed)
     Wb, Xb = make_inputs(wl)
     s32 = O.candidate_scales(O.act_stats(Xb), 0.5).astype(np.float32)
-    Xp = np.ascontiguousarray(O.fold_inv_scales(np.ascontiguousarray(Xb.T), s32).T)  # X S^-1, bf16
+    X16 = Xb if dtype == "bf16" else O.to_f16_bits(O.widen_bf16(Xb).astype(np.float32))
+    Xp = np.ascontiguousarray(O.fold_inv_scales(np.ascontiguousarray(X16.T), s32, dtype).T)
     return Wb, Xb, Xp, s32
 
 
-def _check_product(Y, Xp, qw, sc, zr, group):
-    ref = O.w4a16_matmul(Xp, qw, sc, zr, group)
+def _dev(bits, dtype):
+    return to_device(bits) if dtype == "bf16" else to_device_f16(bits)
+
+
+def _check_product(Y, Xp, qw, sc, zr, group, dtype="bf16"):
+    ref = O.w4a16_matmul(Xp, qw, sc, zr, group, dtype)
     What = O.dequant_packed(qw, sc, zr, group, Xp.shape[1])
-    form = np.abs(O.widen_bf16(Xp)) @ np.abs(What).T
-    tol = 1.1 * (U * np.abs(ref) + (U + Xp.shape[1] * 2.0 ** -23) * form) + 1e-30
+    form = np.abs(O.widen(Xp, dtype)) @ np.abs(What).T
+    u = UNIT[dtype]
+    tol = 1.1 * (u * np.abs(ref) + (W_ERR[dtype] * u + Xp.shape[1] * 2.0 ** -23) * form) + 1e-30
     got = Y.float().cpu().numpy().astype(np.float64)
     bad = np.abs(got - ref) > tol
     assert not bad.any(), (np.argwhere(bad)[:5], got[bad][:5], ref[bad][:5])
     return np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30)
 
 
+@pytest.mark.parametrize("dtype", DTYPES)
 @pytest.mark.parametrize("name,N,d_out,d_in,bits,group,symmetric", CASES)
-def test_w4a16_against_oracle(name, N, d_out, d_in, bits, group, symmetric):
-    Wb, _, Xp, s32 = _scaled_layer(N, d_out, d_in, bits, group, symmetric, seed=zlib.crc32(name.encode()) % 1000)
+def test_w4a16_against_oracle(name, N, d_out, d_in, bits, group, symmetric, dtype):
+    Wb, _, Xp, s32 = _scaled_layer(N, d_out, d_in, bits, group, symmetric, seed=zlib.crc32(name.encode()) % 1000,
+                                   dtype=dtype)
     qw, sc, zr, _, _, _ = O.pack(Wb, s32.astype(np.float64), bits, group, symmetric)
     cfg = awq.make_cfg(bits, group, symmetric, 1)
-    Y = awq.w4a16_gemm(to_device(Xp), torch.from_numpy(qw.view(np.int32)).cuda(),
+    Y = awq.w4a16_gemm(_dev(Xp, dtype), torch.from_numpy(qw.view(np.int32)).cuda(),
                        torch.from_numpy(sc).cuda(), torch.from_numpy(zr).cuda(), cfg)
     torch.cuda.synchronize()
-    rel = _check_product(Y, Xp, qw, sc, zr, group)
-    print(name, "max |err| / max |Y| =", rel)
+    assert Y.dtype == (torch.bfloat16 if dtype == "bf16" else torch.float16)
+    rel = _check_product(Y, Xp, qw, sc, zr, group, dtype)
+    print(name, dtype, "max |err| / max |Y| =", rel)
 
 
 def test_w4a16_deterministic_and_workspace_error_clear():
@@ -112,13 +130,15 @@ def test_pack_then_product_on_the_gpu():
     assert not ((O.unpack_codes(qw_h, d_in) != codes_ref) & ~near).any()
 
 
+@pytest.mark.parametrize("dtype", DTYPES)
 @pytest.mark.parametrize("shape", [(512,), (512, 24), (384, 5), (256, 1)])
-def test_fold_bit_exact(shape):
+def test_fold_bit_exact(shape, dtype):
     rng = np.random.default_rng(40 + len(shape))
-    p = gen.f64_to_bf16_bits(rng.standard_normal(shape) * 3)
+    x = (rng.standard_normal(shape) * 3).astype(np.float32)
+    p = gen.f64_to_bf16_bits(x.astype(np.float64)) if dtype == "bf16" else O.to_f16_bits(x)
     s = np.exp(rng.standard_normal(shape[0]) * 1.5).astype(np.float32)
-    dev = to_device(p)
+    dev = _dev(p, dtype)
     awq.fold_inv_scales(torch.from_numpy(s).cuda(), dev)
     torch.cuda.synchronize()
     got = dev.view(torch.int16).cpu().numpy().view(np.uint16)
-    assert np.array_equal(got, O.fold_inv_scales(p, s))
+    assert np.array_equal(got, O.fold_inv_scales(p, s, dtype))

@@ -655,3 +655,35 @@ def test_p5_worked_example_through_the_inference_path():
         assert O.widen_bf16(xp)[0, 1] == pytest.approx(ex["x_i"] / s_i)
         y = float(O.w4a16_matmul(xp, qw, sc, zr, d_in)[0, 0])
         assert y - y_true == pytest.approx(dy, abs=tol)
+
+
+def test_f16_rounding_and_fold_match_torch():
+    """float32 -> fp16 round to nearest even equals torch's conversion, and the
+    fp16 fold equals torch's float32 division rounded to fp16."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(36)
+    x = (rng.standard_normal(20000) * np.exp(rng.standard_normal(20000) * 3)).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.to_f16_bits(x), ref)
+    p = O.to_f16_bits(rng.standard_normal((48, 16)).astype(np.float32))
+    s = np.exp(rng.standard_normal(48)).astype(np.float32)
+    want = (torch.from_numpy(O.widen_f16(p).astype(np.float32)) / torch.from_numpy(s)[:, None]).to(torch.float16)
+    assert np.array_equal(O.fold_inv_scales(p, s, "f16"), want.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_w4a16_f16_activations_brute_force():
+    """The fp16-activation product (the pages' FP16 inference) equals a
+    triple loop over fp16 inputs and the stored codes."""
+    rng = np.random.default_rng(37)
+    rows, d_in, g, N = 3, 32, 16, 2
+    Wb = gen.f64_to_bf16_bits(rng.standard_normal((rows, d_in)) * 0.1)
+    qw, sc, zr, _, _, _ = O.pack(Wb, np.ones(d_in), 4, g, True)
+    Xh = O.to_f16_bits(rng.standard_normal((N, d_in)).astype(np.float32))
+    Y = O.w4a16_matmul(Xh, qw, sc, zr, g, "f16")
+    X = Xh.view(np.float16).astype(np.float64)
+    words = qw.view(np.uint32)
+    for t in range(N):
+        for o in range(rows):
+            acc = sum(X[t, i] * (((int(words[o, i // 8]) >> (4 * (i % 8))) & 0xF) - float(zr[o, i // g]))
+                      * float(sc[o, i // g]) for i in range(d_in))
+            assert Y[t, o] == pytest.approx(acc, rel=1e-12, abs=1e-14)

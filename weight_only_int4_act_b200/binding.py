@@ -18,6 +18,7 @@ STATUS_NAMES = {
     4: "AWQ_ERR_NONFINITE", 5: "AWQ_ERR_CUDA", 6: "AWQ_ERR_DEVICE", 7: "AWQ_ERR_UNSUPPORTED",
 }
 FORMS = {"auto": 0, "direct": 1, "gram": 2}
+AWQ_DTYPE_BF16, AWQ_DTYPE_F16 = 0, 1
 
 # every symbol include/awq.h declares
 EXPORTED = (
@@ -85,10 +86,10 @@ def lib() -> ctypes.CDLL:
                                                 cfgp, c_void_p, c_size_t, c_void_p, c_void_p, c_void_p]),
             "awq_quantize_pack_group_clip": (c_int32, [c_void_p, c_void_p, c_void_p, c_int32, c_void_p, c_int64,
                                                        c_int64, cfgp, c_void_p, c_void_p, c_void_p, c_void_p]),
-            "awq_fold_inv_scales": (c_int32, [c_void_p, c_int64, c_void_p, c_int64, c_void_p]),
+            "awq_fold_inv_scales": (c_int32, [c_void_p, c_int64, c_void_p, c_int32, c_int64, c_void_p]),
             "awq_w4a16_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, cfgp]),
-            "awq_w4a16_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64, cfgp,
-                                         c_void_p, c_void_p, c_size_t, c_void_p]),
+            "awq_w4a16_gemm": (c_int32, [c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64,
+                                         cfgp, c_void_p, c_void_p, c_size_t, c_void_p]),
             "awq_workspace_error": (c_int32, [c_void_p, c_void_p]),
             "awq_quantize_pack": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_void_p, c_void_p,
                                             c_void_p, c_void_p]),
@@ -318,16 +319,26 @@ def quantize_pack_group_clip(W, s, clips, best_clip, cfg: QCfg, outputs=None):
 
 
 # --------------------------------------------------------------------------- inference side
+def _dtype_code(t, name):
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return AWQ_DTYPE_BF16
+    if t.dtype == torch.float16:
+        return AWQ_DTYPE_F16
+    raise ValueError(f"{name} must be bfloat16 or float16, got {t.dtype}")
+
+
 def fold_inv_scales(s, p):
-    """In place: row i of p (bf16 [d_in] or [d_in, inner], CUDA) becomes p / s_i."""
+    """In place: row i of p (bf16 or fp16 [d_in] or [d_in, inner], CUDA) becomes p / s_i."""
     torch = _torch()
     _req(s, torch.float32, None, "s")
-    _req(p, torch.bfloat16, None, "p")
+    dt = _dtype_code(p, "p")
+    _req(p, p.dtype, None, "p")
     d_in = s.numel()
     if p.shape[0] != d_in:
         raise ValueError("p must have the channel (length of s) on its first axis")
     inner = p.numel() // d_in if d_in else 0
-    _check(lib().awq_fold_inv_scales(_ptr(s), d_in, _ptr(p), inner, _stream()), "awq_fold_inv_scales")
+    _check(lib().awq_fold_inv_scales(_ptr(s), d_in, _ptr(p), dt, inner, _stream()), "awq_fold_inv_scales")
     return p
 
 
@@ -336,9 +347,11 @@ def w4a16_workspace_size(N, d_out, d_in, cfg: QCfg) -> int:
 
 
 def w4a16_gemm(Xp, qweight, scales, zeros, cfg: QCfg, ws=None, out=None):
-    """Y bf16 [N, d_out] = X' (bf16 [N, d_in]) times the dequantised packed weights."""
+    """Y [N, d_out] = X' ([N, d_in], fp16 or bf16) times the dequantised packed
+    weights, in the activations' type."""
     torch = _torch()
-    _req(Xp, torch.bfloat16, None, "X")
+    dt = _dtype_code(Xp, "X")
+    _req(Xp, Xp.dtype, None, "X")
     N, d_in = Xp.shape
     _req(qweight, torch.int32, None, "qweight")
     d_out = qweight.shape[0]
@@ -350,9 +363,9 @@ def w4a16_gemm(Xp, qweight, scales, zeros, cfg: QCfg, ws=None, out=None):
     if ws is None:
         ws = workspace(max(w4a16_workspace_size(N, d_out, d_in, cfg), 256))
     if out is None:
-        out = torch.empty((N, d_out), dtype=torch.bfloat16, device=Xp.device)
-    _req(out, torch.bfloat16, (N, d_out), "out")
-    _check(lib().awq_w4a16_gemm(_ptr(Xp), _ptr(qweight), _ptr(scales), _ptr(zeros), N, d_out, d_in,
+        out = torch.empty((N, d_out), dtype=Xp.dtype, device=Xp.device)
+    _req(out, Xp.dtype, (N, d_out), "out")
+    _check(lib().awq_w4a16_gemm(_ptr(Xp), dt, _ptr(qweight), _ptr(scales), _ptr(zeros), N, d_out, d_in,
                                 ctypes.byref(cfg), _ptr(out), _ptr(ws), ws.numel(), _stream()), "awq_w4a16_gemm")
     return out
 

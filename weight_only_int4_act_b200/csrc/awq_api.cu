@@ -187,25 +187,27 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over a row-major [rows, cols] matrix with leading dimension ld
-// (elements), box = box_rows x 64 columns, 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+// 2-D map of 16-bit elements (bf16 unless given) over a row-major [rows, cols]
+// matrix with leading dimension ld (elements), box = box_rows x 64 columns,
+// 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {ld * 2};
   cuuint32_t box[2] = {(cuuint32_t)GEMM_BK, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-// 2-D uint32 map over the packed codes [rows, words] (no swizzle), box of
-// box_words x box_rows.
+// 2-D uint32 map over the packed codes [rows, words], box of box_words x
+// box_rows (128-byte swizzle: box_words = 32).
 bool make_map_u32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t words, uint32_t box_words,
-                  uint32_t box_rows) {
+                  uint32_t box_rows, CUtensorMapSwizzle swz) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {words, rows};
@@ -213,7 +215,7 @@ bool make_map_u32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t word
   cuuint32_t box[2] = {box_words, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -823,10 +825,12 @@ W4Plan w4_plan(int64_t N, int64_t d_out, int64_t d_in) {
   W4Plan p{};
   p.bn = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
   // ring depths: deep packed-code rings for narrow (weight-streaming) tiles
-  if (p.bn <= 32) { p.as = 4; p.xs = 8; p.rs = 24; }
-  else if (p.bn == 64) { p.as = 4; p.xs = 6; p.rs = 16; }
-  else if (p.bn == 128) { p.as = 4; p.xs = 4; p.rs = 16; }
-  else { p.as = 3; p.xs = 4; p.rs = 8; }
+  // Ring depths within the shared memory (an MMA's commit lands about a
+  // microsecond after issue and holds its weight and activation stages).
+  if (p.bn <= 32) { p.as = 3; p.xs = 6; p.rs = 3; }
+  else if (p.bn == 64) { p.as = 3; p.xs = 4; p.rs = 2; }
+  else if (p.bn == 128) { p.as = 3; p.xs = 3; p.rs = 2; }
+  else { p.as = 2; p.xs = 2; p.rs = 1; }
   p.smem = w4_smem_bytes(p.as, p.xs, p.rs, p.bn);
   p.n_mb = (int)cdiv(d_out, W4_BM);
   p.n_nb = (int)cdiv(N, p.bn);
@@ -865,11 +869,13 @@ extern "C" size_t awq_w4a16_workspace_size(int64_t N, int64_t d_out, int64_t d_i
   return w4_plan(N, d_out, d_in).ws;
 }
 
-extern "C" awq_status awq_w4a16_gemm(const void* X, const uint32_t* qweight, const void* scales, const void* zeros, int64_t N,
-                          int64_t d_out, int64_t d_in, const awq_qcfg* cfg, void* Y, void* ws, size_t ws_bytes,
-                          awq_stream_t stream) {
+extern "C" awq_status awq_w4a16_gemm(const void* X, awq_dtype dtype, const uint32_t* qweight, const void* scales,
+                                     const void* zeros, int64_t N, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
+                                     void* Y, void* ws, size_t ws_bytes, awq_stream_t stream) {
   awq_status st = check_w4(N, d_out, d_in, cfg);
   if (st != AWQ_OK) return st;
+  if (dtype != AWQ_DTYPE_BF16 && dtype != AWQ_DTYPE_F16) return AWQ_ERR_INVALID_ARG;
+  const bool f16 = dtype == AWQ_DTYPE_F16;
   if (!X || !qweight || !scales || !zeros || !Y || !ws) return AWQ_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 2) || !aligned(zeros, 2) || !aligned(Y, 16) ||
       !aligned(ws, 256))
@@ -880,8 +886,10 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, const uint32_t* qweight, con
   if ((st = check_device(&sms)) != AWQ_OK) return st;
   cudaStream_t cs = as_stream(stream);
   CUtensorMap tx, tw;
-  if (!make_map(&tx, X, N, d_in, d_in, p.bn)) return AWQ_ERR_CUDA;
-  if (!make_map_u32(&tw, qweight, d_out, d_in / 8, W4_BK / 8, W4_BM)) return AWQ_ERR_CUDA;
+  if (!make_map(&tx, X, N, d_in, d_in, p.bn, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+    return AWQ_ERR_CUDA;
+  if (!make_map_u32(&tw, qweight, d_out, d_in / 8, 32, W4_BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return AWQ_ERR_CUDA;
   W4Args a{};
   a.N = (int)N;
   a.d_out = (int)d_out;
@@ -903,7 +911,7 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, const uint32_t* qweight, con
   if (p.smem > W4_SMEM_LIMIT) return AWQ_ERR_UNSUPPORTED;
   a.scales = static_cast<const __half*>(scales);
   a.zeros = static_cast<const __half*>(zeros);
-  a.Y = static_cast<__nv_bfloat16*>(Y);
+  a.Y = Y;
   a.P = p.splits > 1 ? at<float>(ws, kAlign) : nullptr;
   a.p_stride = p.p_stride;
   a.err = at<int>(ws, 0);
@@ -915,24 +923,40 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, const uint32_t* qweight, con
     kernel<<<grid, W4_THREADS, p.smem, cs>>>(tx, tw, a);
     return launch_status();
   };
-  switch (cfg->group) {
-    case 8: st = launch(w4a16_gemm_tcgen05<4>); break;
-    case 16: st = launch(w4a16_gemm_tcgen05<2>); break;
-    default: st = launch(w4a16_gemm_tcgen05<1>); break;
+  // template argument: quantisation groups per 64 channels
+  if (f16) {
+    switch (cfg->group) {
+      case 8: st = launch(w4a16_gemm_tcgen05<8, true>); break;
+      case 16: st = launch(w4a16_gemm_tcgen05<4, true>); break;
+      case 32: st = launch(w4a16_gemm_tcgen05<2, true>); break;
+      default: st = launch(w4a16_gemm_tcgen05<1, true>); break;
+    }
+  } else {
+    switch (cfg->group) {
+      case 8: st = launch(w4a16_gemm_tcgen05<8, false>); break;
+      case 16: st = launch(w4a16_gemm_tcgen05<4, false>); break;
+      case 32: st = launch(w4a16_gemm_tcgen05<2, false>); break;
+      default: st = launch(w4a16_gemm_tcgen05<1, false>); break;
+    }
   }
   if (st != AWQ_OK) return st;
   if (p.splits > 1) {
     const long long n = N * d_out;
     const long long blocks = cdiv(n / 4 > 0 ? n / 4 : 1, 256);
-    w4a16_split_reduce<<<(unsigned)(blocks < 4 * sms ? blocks : 4 * sms), 256, 0, cs>>>(a.P, p.splits, n,
-                                                                                       p.p_stride, a.Y);
+    const unsigned rgrid = (unsigned)(blocks < 4 * sms ? blocks : 4 * sms);
+    if (f16)
+      w4a16_split_reduce<true><<<rgrid, 256, 0, cs>>>(a.P, p.splits, n, p.p_stride, Y);
+    else
+      w4a16_split_reduce<false><<<rgrid, 256, 0, cs>>>(a.P, p.splits, n, p.p_stride, Y);
     return launch_status();
   }
   return AWQ_OK;
 }
 
-extern "C" awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p, int64_t inner, awq_stream_t stream) {
+extern "C" awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p, awq_dtype dtype, int64_t inner,
+                                          awq_stream_t stream) {
   if (!s || !p) return AWQ_ERR_INVALID_ARG;
+  if (dtype != AWQ_DTYPE_BF16 && dtype != AWQ_DTYPE_F16) return AWQ_ERR_INVALID_ARG;
   if (d_in < 1 || inner < 1 || d_in > (1 << 24) || inner > (1 << 24)) return AWQ_ERR_SHAPE;
   if (!aligned(p, 2) || !aligned(s, 4)) return AWQ_ERR_INVALID_ARG;
   int sms = 0;
@@ -943,9 +967,14 @@ extern "C" awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p,
   const long long units = d_in * inner / (vec ? 8 : 1);
   const long long blocks = cdiv(units, 256);
   const unsigned grid = (unsigned)(blocks < 8LL * sms ? blocks : 8LL * sms);
-  if (vec)
-    fold_inv_scales_kernel<8><<<grid, 256, 0, cs>>>(s, d_in, inner, static_cast<__nv_bfloat16*>(p));
+  const bool f16 = dtype == AWQ_DTYPE_F16;
+  if (vec && f16)
+    fold_inv_scales_kernel<8, true><<<grid, 256, 0, cs>>>(s, d_in, inner, p);
+  else if (vec)
+    fold_inv_scales_kernel<8, false><<<grid, 256, 0, cs>>>(s, d_in, inner, p);
+  else if (f16)
+    fold_inv_scales_kernel<1, true><<<grid, 256, 0, cs>>>(s, d_in, inner, p);
   else
-    fold_inv_scales_kernel<1><<<grid, 256, 0, cs>>>(s, d_in, inner, static_cast<__nv_bfloat16*>(p));
+    fold_inv_scales_kernel<1, false><<<grid, 256, 0, cs>>>(s, d_in, inner, p);
   return launch_status();
 }

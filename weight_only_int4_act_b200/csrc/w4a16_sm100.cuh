@@ -1,8 +1,11 @@
 // W4A16 product on sm_100a: Y[t, o] = sum_i X'[t, i] W_hat[o, i], where
 // W_hat[o, i] = (code - z) * Delta is dequantised from the packed format
 // (8 codes per uint32 word, lowest channel in the lowest nibble; fp16 step
-// and zero point per (row, group)) inside the kernel, and X' is the bf16
-// activation that already carries S^-1 (folded into its producer).
+// and zero point per (row, group)) inside the kernel, and X' is the fp16 or
+// bf16 activation that already carries S^-1 (folded into its producer). The
+// dequantised weight enters the tensor cores in the activation type: in fp16
+// (code - z) * Delta is rounded once; in bf16 Delta is first rounded to bf16,
+// then the product.
 //
 // Pages: "AWQ量化技术解析：激活感知的权重量化革命" (kwkr.cn) §1.2 (weights
 // dequantised on the fly as W_int4 x scale_fp16) and §4.2 (dequantisation
@@ -16,18 +19,21 @@
 // the N operand, so a decode batch of a few tokens still fills a tile. One
 // K step is 64 channels. Three shared-memory rings, each with its own
 // full/empty mbarriers, so that each stream runs ahead as far as its ring
-// allows: packed codes (4 KB a step, up to 24 steps deep: the weight bytes in
-// flight that hide HBM latency), activations (BN x 64 bf16, 128-byte swizzle)
-// and dequantised weights (128 x 64 bf16, 128-byte swizzle). Depths depend on
-// BN (host plan). Warp roles (480 threads, one CTA per SM):
-//   warp 0       TMA of the packed codes (128 rows x 8 words, no swizzle);
+// allows: packed codes (4 K steps per stage: 128 rows x 128 B with the
+// 128-byte swizzle, up to 6 stages deep: the weight bytes in flight that hide
+// HBM latency; a box row of a single step's 32 B moved only ~7 GB/s per SM),
+// activations (BN x 64, 128-byte swizzle) and dequantised weights (128 x 64,
+// 128-byte swizzle). Depths depend on BN (host plan). Warp roles (480
+// threads, one CTA per SM):
+//   warp 0       TMA of the packed codes;
 //   warp 1       allocates 512 TMEM columns (two accumulators at columns 0
 //                and 256) and one thread issues the MMAs;
 //   warp 2       TMA of the activation tiles;
 //   warps 3..10  dequantise: thread (h, r) expands words 4h..4h+3 of row r
-//                ((code - z) * Delta in fp32, exact, then one rounding to
-//                bf16) into the K-major swizzled layout the MMA descriptor
-//                reads; a proxy fence and one arrive per warp publish it;
+//                into the activation type, two codes per packed subtract and
+//                multiply (dequant_word), and stores them in the K-major
+//                swizzled layout the MMA descriptor reads; a proxy fence and
+//                one arrive per warp publish the stage;
 //   warps 11..14 epilogue: tcgen05.ld of the accumulator (TMEM lane = output
 //                channel, column = token), bf16 stores of Y (or fp32 split-K
 //                partials), then release of the accumulator.
@@ -46,12 +52,15 @@
 namespace awq {
 
 constexpr int W4_BM = 128;
-constexpr int W4_BK = 64;
+constexpr int W4_BK = 128;                      // channels per K step: two 64-wide swizzled sub-tiles
+constexpr int W4_SUB = 64;
 constexpr int W4_MAX_BN = 256;
 constexpr int W4_THREADS = 480;
-constexpr int W4_A_STAGE = W4_BM * W4_BK * 2;  // dequantised weights, 16 KB
-constexpr int W4_R_STAGE = W4_BM * W4_BK / 2;  // packed codes, 4 KB
-constexpr int W4_MAX_RS = 32, W4_MAX_XS = 8, W4_MAX_AS = 4;
+constexpr int W4_RK = 2;                        // K steps of packed codes per TMA box (128 rows x 128 B)
+constexpr int W4_R_STAGE = W4_BM * 128;         // packed codes, 16 KB
+constexpr int W4_A_SUB = W4_BM * W4_SUB * 2;    // one 128 x 64 sub-tile of dequantised weights, 16 KB
+constexpr int W4_A_STAGE = 2 * W4_A_SUB;        // 32 KB
+constexpr int W4_MAX_RS = 32, W4_MAX_XS = 8, W4_MAX_AS = 8;
 constexpr int W4_NBARS = 2 * (W4_MAX_RS + W4_MAX_XS + W4_MAX_AS) + 5;
 constexpr int W4_TMEM_COLS = 512;
 constexpr int W4_SMEM_LIMIT = 232448;
@@ -77,7 +86,7 @@ struct W4Args {
   int as, xs, rs;    // ring depths: dequantised weights, activations, packed codes
   const __half* scales;  // [d_out, ng]
   const __half* zeros;   // [d_out, ng]
-  __nv_bfloat16* Y;      // [N, d_out] (splits == 1)
+  void* Y;               // [N, d_out] in the activation type (splits == 1)
   float* P;              // [splits][p_stride] with [N, d_out] in each slab (splits > 1)
   long long p_stride;    // N * d_out rounded up to a multiple of 4
   int* err;
@@ -99,17 +108,60 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
-// (code - z) * Delta for the 8 codes of one word, as 8 bf16 in a uint4.
-// 2^23 + code is built by OR-ing the code into the mantissa of 2^23, so
-// subtracting 2^23 + z leaves code - z exactly; the product with the fp16
-// step is exact in fp32 (at most 4 + 11 significant bits) and is rounded
-// once, to nearest even, to bf16.
-__device__ __forceinline__ uint4 dequant_word(uint32_t w, float zoff, float delta) {
-  float f[8];
+// The 16-bit activation type: bf16 (F16 = false) or fp16 (F16 = true).
+// kMagic: two copies of a value whose unit in the last place is 1 (128 in
+// bf16, 1024 in fp16), so OR-ing a 4-bit code into its mantissa gives
+// magic + code exactly.
+template <bool F16>
+struct W4Type {
+  using T = __nv_bfloat16;
+  using T2 = __nv_bfloat162;
+  static constexpr uint32_t kMagic = 0x43004300u;
+  static constexpr float kMagicF = 128.0f;
+  static __device__ __forceinline__ T from_float(float x) { return __float2bfloat16_rn(x); }
+  static __device__ __forceinline__ float to_float(T x) { return __bfloat162float(x); }
+};
+template <>
+struct W4Type<true> {
+  using T = __half;
+  using T2 = __half2;
+  static constexpr uint32_t kMagic = 0x64006400u;
+  static constexpr float kMagicF = 1024.0f;
+  static __device__ __forceinline__ T from_float(float x) { return __float2half_rn(x); }
+  static __device__ __forceinline__ float to_float(T x) { return __half2float(x); }
+};
+
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  using Ty = W4Type<F16>;
+  typename Ty::T2 p;
+  p.x = Ty::from_float(lo);
+  p.y = Ty::from_float(hi);
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// (code - z) * Delta for the 8 codes of one word, as 8 values of the
+// activation type in a uint4 (channel order). Per pair of codes (byte i of
+// the word): a byte permute puts code 2i in the low and code 2i+1 (from the
+// word shifted by 4) in the high 16-bit half; masking and OR-ing the magic
+// constant gives magic + code in each half, exactly; a packed subtract of
+// magic + z leaves code - z exactly; a packed multiply by Delta rounds once.
+// zz = (magic + z, magic + z) and dd = (Delta, Delta) in the activation type.
+template <bool F16>
+__device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t zz, uint32_t dd) {
+  using T2 = typename W4Type<F16>::T2;
+  const uint32_t w4 = w >> 4;
+  uint32_t out[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) f[j] = (__uint_as_float(((w >> (4 * j)) & 0xFu) | 0x4B000000u) - zoff) * delta;
-  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                    pack_bf16x2(f[6], f[7]));
+  for (int i = 0; i < 4; ++i) {
+    uint32_t t = __byte_perm(w, w4, (uint32_t)(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12)));
+    t = (t & 0x000F000Fu) | W4Type<F16>::kMagic;
+    T2 h = *reinterpret_cast<const T2*>(&t);
+    h = __hsub2(h, *reinterpret_cast<const T2*>(&zz));
+    h = __hmul2(h, *reinterpret_cast<const T2*>(&dd));
+    out[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 // A ring position: stage index and the parity of its current phase.
@@ -124,8 +176,9 @@ struct Ring {
   }
 };
 
-// GPH = quantisation groups per half K step of 32 channels (1 for g >= 32).
-template <int GPH>
+// GPH = quantisation groups per 64 channels (one dequantising thread's share
+// of a K step; 1 for g >= 64); F16: fp16 activations and output (else bf16).
+template <int GPH, bool F16>
 __global__ void __launch_bounds__(W4_THREADS, 1)
     w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                        const W4Args args) {
@@ -133,10 +186,11 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int bn = args.bn;
   const int AS = args.as, XS = args.xs, RS = args.rs;
-  const uint32_t x_stage = (uint32_t)bn * W4_BK * 2;  // a multiple of 1024 (bn >= 16 in steps of 16)
-  uint8_t* sA = smem;                        // [AS][128 rows][128 B], swizzled
-  uint8_t* sX = sA + AS * W4_A_STAGE;        // [XS][BN rows][128 B], swizzled
-  uint8_t* sR = sX + XS * x_stage;           // [RS][128 rows][32 B]
+  const uint32_t x_sub = (uint32_t)bn * W4_SUB * 2;  // one BN x 64 sub-tile; a multiple of 1024
+  const uint32_t x_stage = 2 * x_sub;
+  uint8_t* sA = smem;                        // [AS][2][128 rows][128 B], swizzled
+  uint8_t* sX = sA + AS * W4_A_STAGE;        // [XS][2][BN rows][128 B], swizzled
+  uint8_t* sR = sX + XS * x_stage;           // [RS][128 rows][128 B], swizzled
   uint64_t* bars = reinterpret_cast<uint64_t*>(sR + RS * W4_R_STAGE);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + W4_NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -189,7 +243,8 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
 
   if (warp == 0 || warp == 2) {
     if (lane == 0) {
-      // ---------------- TMA producers: packed codes (warp 0) or activations (warp 2)
+      // ---------------- TMA producers: packed codes (warp 0, one box per W4_RK
+      // steps) or activations (warp 2, two 64-wide boxes per step)
       const bool codes = warp == 0;
       const int depth = codes ? RS : XS;
       Ring ring;
@@ -200,7 +255,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         w4_tile_coords(t, args, mb, nb, split);
         const int kb0 = split * args.kb_per_split;
         const int kb1 = min(args.n_kb, kb0 + args.kb_per_split);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += codes ? W4_RK : 1) {
           const uint32_t full = codes ? rfull(ring.stage) : xfull(ring.stage);
           const uint32_t empty = codes ? rempty(ring.stage) : xempty(ring.stage);
           if (!mbar_wait(empty, ring.phase ^ 1u, abort_flag, args.err, codes ? ERR_W4_REMPTY : ERR_W4_XEMPTY)) {
@@ -212,7 +267,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
             tma_load_2d(smem_u32(sR + ring.stage * W4_R_STAGE), &tmW, full, kb * (W4_BK / 8), mb * W4_BM);
           } else {
             mbar_arrive_expect_tx(full, x_stage);
-            tma_load_2d(smem_u32(sX + ring.stage * x_stage), &tmX, full, kb * W4_BK, nb * bn);
+            uint8_t* dst = sX + ring.stage * x_stage;
+            tma_load_2d(smem_u32(dst), &tmX, full, kb * W4_BK, nb * bn);
+            tma_load_2d(smem_u32(dst + x_sub), &tmX, full, kb * W4_BK + W4_SUB, nb * bn);
           }
           issued |= 1u << ring.stage;
           last_parity = (last_parity & ~(1u << ring.stage)) | (ring.phase << ring.stage);
@@ -224,8 +281,14 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer
-      const uint32_t idesc = idesc_bf16_f32(W4_BM, bn);
+      // ---------------- MMA issuer: 8 MMAs (K = 16 each) per step
+      // kind::f16 with both operands fp16 (format 0) or both bf16 (format 1)
+      const uint32_t idesc = F16 ? ((1u << 4) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(W4_BM >> 4) << 24))
+                                 : idesc_bf16_f32(W4_BM, bn);
+      // descriptors of stage 0; a stage, a sub-tile and a K offset only move the
+      // start-address field (address >> 4; all shared addresses are below 256 KB)
+      const uint64_t da0 = desc_kmajor_sw128(smem_u32(sA));
+      const uint64_t dx0 = desc_kmajor_sw128(smem_u32(sX));
       Ring xr, ar;
       bool ok = true;
       int local = 0;
@@ -245,12 +308,14 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + ar.stage * W4_A_STAGE);
-          const uint32_t x_base = smem_u32(sX + xr.stage * x_stage);
+          const uint64_t da = da0 + ((uint64_t)(ar.stage * W4_A_STAGE) >> 4);
+          const uint64_t dx = dx0 + ((uint64_t)(xr.stage * x_stage) >> 4);
 #pragma unroll
-          for (int k = 0; k < W4_BK / 16; ++k)
-            mma_bf16(d_tmem, desc_kmajor_sw128(a_base + k * 32), desc_kmajor_sw128(x_base + k * 32), idesc,
+          for (int k = 0; k < W4_BK / 16; ++k) {
+            const uint32_t sub = (uint32_t)(k >> 2), kq = (uint32_t)(k & 3);
+            mma_bf16(d_tmem, da + ((sub * W4_A_SUB + kq * 32) >> 4), dx + ((sub * x_sub + kq * 32) >> 4), idesc,
                      (kb != kb0) || (k != 0));
+          }
           mma_commit(xempty(xr.stage));
           mma_commit(aempty(ar.stage));
           xr.next(XS);
@@ -262,11 +327,12 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       mbar_wait_drain(drain_bar, 0);
     }
   } else if (warp < 11) {
-    // ---------------- dequantisation: thread (h, r) takes words 4h..4h+3 of row r
+    // ---------------- dequantisation: thread (h, r) takes channels 64h .. 64h+63
+    // of each step for row r (8 words), i.e. row r of A sub-tile h
     const int d = threadIdx.x - 3 * 32;
     const int r = d & (W4_BM - 1);
     const int h = d >> 7;
-    const uint32_t a_row_off = (uint32_t)r * 128;
+    const uint32_t a_row_off = (uint32_t)(h * W4_A_SUB + r * 128);
     const int sw = r & 7;
     Ring rr, ar;
     bool ok = true;
@@ -279,47 +345,64 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       const bool valid = row < args.d_out;
       const __half* srow = args.scales + (long long)(valid ? row : 0) * args.ng;
       const __half* zrow = args.zeros + (long long)(valid ? row : 0) * args.ng;
-      // step and zero point of the GPH groups of this thread's 32 channels, loaded one step ahead
-      auto load_params = [&](int kb, float (&dq)[GPH], float (&zq)[GPH]) {
+      // step and zero point of the GPH groups of this thread's 64 channels. The
+      // raw fp16 values of step kb + 2 are loaded while step kb is processed
+      // and converted only when their step comes, so the loads stay in flight.
+      using Ty = W4Type<F16>;
+      auto load_params = [&](int kb, __half (&dq)[GPH], __half (&zq)[GPH]) {
 #pragma unroll
         for (int q = 0; q < GPH; ++q) {
-          const int ch = kb * W4_BK + h * 32 + q * (32 / GPH);
+          const int ch = kb * W4_BK + h * W4_SUB + q * (W4_SUB / GPH);
           const int gi = min(ch >> args.group_shift, args.ng - 1);
-          dq[q] = valid ? __half2float(srow[gi]) : 0.0f;
-          zq[q] = 8388608.0f + (valid ? __half2float(zrow[gi]) : 0.0f);
+          dq[q] = valid ? srow[gi] : __float2half_rn(0.0f);
+          zq[q] = valid ? zrow[gi] : __float2half_rn(0.0f);
         }
       };
-      float dn[GPH], zn[GPH];
-      load_params(kb0, dn, zn);
+      __half d0[GPH], z0[GPH], d1[GPH], z1[GPH], d2[GPH], z2[GPH];  // steps kb, kb + 1, kb + 2
+      load_params(kb0, d0, z0);
+      if (kb0 + 1 < kb1) load_params(kb0 + 1, d1, z1);
       for (int kb = kb0; kb < kb1; ++kb) {
-        float dc[GPH], zc[GPH];
+        if (kb + 2 < kb1) load_params(kb + 2, d2, z2);
+        uint32_t dc[GPH], zc[GPH];
 #pragma unroll
         for (int q = 0; q < GPH; ++q) {
-          dc[q] = dn[q];
-          zc[q] = zn[q];
+          const float dv = __half2float(d0[q]), zv = __half2float(z0[q]);
+          dc[q] = pack2<F16>(dv, dv);                              // fp16 step: exact in fp16, rounded in bf16
+          zc[q] = pack2<F16>(Ty::kMagicF + zv, Ty::kMagicF + zv);  // integer z <= 15: exact
+          d0[q] = d1[q];
+          z0[q] = z1[q];
+          d1[q] = d2[q];
+          z1[q] = z2[q];
         }
-        if (kb + 1 < kb1) load_params(kb + 1, dn, zn);
-        bool have = mbar_wait(rfull(rr.stage), rr.phase, abort_flag, args.err, ERR_W4_RFULL);
+        // step kk of the code box: 16-byte chunks 4 kk + 2h and 4 kk + 2h + 1 of row r, swizzled
+        const int kk = (kb - kb0) & (W4_RK - 1);
+        bool have = true;
+        if (kk == 0) have = mbar_wait(rfull(rr.stage), rr.phase, abort_flag, args.err, ERR_W4_RFULL);
         if (!__all_sync(0xffffffffu, have)) {
           ok = false;
           break;
         }
-        const uint4 w = *reinterpret_cast<const uint4*>(sR + rr.stage * W4_R_STAGE + r * 32 + h * 16);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(rempty(rr.stage));
-        rr.next(RS);
+        const uint8_t* rrow = sR + rr.stage * W4_R_STAGE + r * 128;
+        const int c0 = 4 * kk + 2 * h;
+        const uint4 w0 = *reinterpret_cast<const uint4*>(rrow + ((c0 ^ sw) << 4));
+        const uint4 w1 = *reinterpret_cast<const uint4*>(rrow + (((c0 + 1) ^ sw) << 4));
+        if (kk == W4_RK - 1 || kb == kb1 - 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(rempty(rr.stage));
+          rr.next(RS);
+        }
         have = mbar_wait(aempty(ar.stage), ar.phase ^ 1u, abort_flag, args.err, ERR_W4_AEMPTY);
         if (!__all_sync(0xffffffffu, have)) {
           ok = false;
           break;
         }
-        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         uint8_t* arow = sA + ar.stage * W4_A_STAGE + a_row_off;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          constexpr int WPG = 4 / GPH;  // words per group inside the half step
-          const uint4 v = dequant_word(words[c], zc[c / WPG], dc[c / WPG]);
-          *reinterpret_cast<uint4*>(arow + (((4 * h + c) ^ sw) << 4)) = v;
+        for (int c = 0; c < 8; ++c) {
+          constexpr int WPG = 8 / GPH;  // words per group inside the thread's 64 channels
+          const uint4 v = dequant_word<F16>(words[c], zc[c / WPG], dc[c / WPG]);
+          *reinterpret_cast<uint4*>(arow + ((c ^ sw) << 4)) = v;
         }
         fence_proxy_async_shared();
         __syncwarp();
@@ -336,7 +419,8 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       int mb, nb, split;
       w4_tile_coords(t, args, mb, nb, split);
       const int acc = local & 1;
-      const bool ready = mbar_wait(tfull(acc), (local >> 1) & 1, abort_flag, args.err, ERR_W4_TFULL);
+      // the accumulator takes a whole tile: wait without spinning
+      const bool ready = mbar_wait_sleep(tfull(acc), (local >> 1) & 1, abort_flag, args.err, ERR_W4_TFULL, 256);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
       const int o = mb * W4_BM + r;
@@ -351,10 +435,10 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         if (o < args.d_out) {
           const long long e0 = (long long)(t0 + c * 32) * args.d_out + o;
           if (args.splits == 1) {
-            __nv_bfloat16* y = args.Y + e0;
+            typename W4Type<F16>::T* y = static_cast<typename W4Type<F16>::T*>(args.Y) + e0;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < jn) y[(long long)j * args.d_out] = __float2bfloat16_rn(__uint_as_float(v[j]));
+              if (j < jn) y[(long long)j * args.d_out] = W4Type<F16>::from_float(__uint_as_float(v[j]));
           } else {
             float* P = args.P + (long long)split * args.p_stride + e0;
 #pragma unroll
@@ -377,10 +461,14 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   }
 }
 
-// Y = bf16(sum over splits of P[split]) in split order; 4 outputs per thread.
-// Slabs are `stride` floats apart (a multiple of 4, so every float4 is aligned).
+// Y = sum over splits of P[split] in split order, rounded to the activation
+// type; 4 outputs per thread. Slabs are `stride` floats apart (a multiple of
+// 4, so every float4 is aligned).
+template <bool F16>
 __global__ void w4a16_split_reduce(const float* __restrict__ P, int splits, long long n, long long stride,
-                                   __nv_bfloat16* __restrict__ Y) {
+                                   void* __restrict__ Yv) {
+  using T = typename W4Type<F16>::T;
+  T* Y = static_cast<T*>(Yv);
   const long long n4 = n >> 2;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
     float4 acc = reinterpret_cast<const float4*>(P)[i];
@@ -391,26 +479,25 @@ __global__ void w4a16_split_reduce(const float* __restrict__ P, int splits, long
       acc.z += p.z;
       acc.w += p.w;
     }
-    uint2 out = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-    reinterpret_cast<uint2*>(Y)[i] = out;
+    reinterpret_cast<uint2*>(Y)[i] = make_uint2(pack2<F16>(acc.x, acc.y), pack2<F16>(acc.z, acc.w));
   }
   // tail (n not a multiple of 4)
-  const long long tail0 = n4 << 2;
-  const long long i = tail0 + (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long i = (n4 << 2) + (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (blockIdx.x == 0 && i < n) {
     float acc = P[i];
     for (int s = 1; s < splits; ++s) acc += P[(long long)s * stride + i];
-    Y[i] = __float2bfloat16_rn(acc);
+    Y[i] = W4Type<F16>::from_float(acc);
   }
 }
 
-// Fold S^-1 into the producer of X: row i of p [d_in, inner] (bf16) becomes
-// p / s_i, the quotient in fp32 (correctly rounded division) rounded to
-// nearest even bf16. VEC = 8: eight elements of one row per thread (inner a
+// Fold S^-1 into the producer of X: row i of p [d_in, inner] (bf16 or fp16)
+// becomes p / s_i, the quotient in fp32 (correctly rounded division) rounded
+// to nearest even. VEC = 8: eight elements of one row per thread (inner a
 // multiple of 8, p 16-byte aligned); VEC = 1: one element per thread.
-template <int VEC>
-__global__ void fold_inv_scales_kernel(const float* __restrict__ s, long long d_in, long long inner,
-                                       __nv_bfloat16* __restrict__ p) {
+template <int VEC, bool F16>
+__global__ void fold_inv_scales_kernel(const float* __restrict__ s, long long d_in, long long inner, void* pv) {
+  using Ty = W4Type<F16>;
+  typename Ty::T* p = static_cast<typename Ty::T*>(pv);
   const long long units = d_in * inner / VEC;
   for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < units;
        u += (long long)gridDim.x * blockDim.x) {
@@ -418,13 +505,15 @@ __global__ void fold_inv_scales_kernel(const float* __restrict__ s, long long d_
     const float si = s[e / inner];
     if constexpr (VEC == 8) {
       uint4 w = reinterpret_cast<const uint4*>(p)[u];
-      uint32_t* h = reinterpret_cast<uint32_t*>(&w);
+      uint32_t* hw = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        h[q] = pack_bf16x2(__uint_as_float(h[q] << 16) / si, __uint_as_float(h[q] & 0xFFFF0000u) / si);
+      for (int q = 0; q < 4; ++q) {
+        const typename Ty::T2 v = *reinterpret_cast<const typename Ty::T2*>(&hw[q]);
+        hw[q] = pack2<F16>(Ty::to_float(v.x) / si, Ty::to_float(v.y) / si);
+      }
       reinterpret_cast<uint4*>(p)[u] = w;
     } else {
-      p[e] = __float2bfloat16_rn(__bfloat162float(p[e]) / si);
+      p[e] = Ty::from_float(Ty::to_float(p[e]) / si);
     }
   }
 }
