@@ -825,13 +825,15 @@ W4Plan w4_plan(int64_t N, int64_t d_out, int64_t d_in) {
   W4Plan p{};
   p.bn = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
   // ring depths: deep packed-code rings for narrow (weight-streaming) tiles
-  // Ring depths within the shared memory (an MMA's commit lands about a
-  // microsecond after issue and holds its weight and activation stages).
-  if (p.bn <= 32) { p.as = 3; p.xs = 6; p.rs = 3; }
-  else if (p.bn == 64) { p.as = 3; p.xs = 4; p.rs = 2; }
-  else if (p.bn == 128) { p.as = 3; p.xs = 3; p.rs = 2; }
-  else { p.as = 2; p.xs = 2; p.rs = 1; }
-  p.smem = w4_smem_bytes(p.as, p.xs, p.rs, p.bn);
+  // Ring depths: codes and activations in shared memory, dequantised weights
+  // in the tensor-memory columns the accumulators leave (an MMA's commit lands
+  // about a microsecond after issue and holds its stages until then).
+  if (p.bn <= 32) { p.xs = 8; p.rs = 6; }
+  else if (p.bn == 64) { p.xs = 6; p.rs = 4; }
+  else if (p.bn == 128) { p.xs = 4; p.rs = 4; }
+  else { p.xs = 3; p.rs = 2; }
+  p.as = w4_max_as(p.bn) < W4_MAX_AS ? w4_max_as(p.bn) : W4_MAX_AS;
+  p.smem = w4_smem_bytes(p.xs, p.rs, p.bn);
   p.n_mb = (int)cdiv(d_out, W4_BM);
   p.n_nb = (int)cdiv(N, p.bn);
   p.n_kb = (int)cdiv(d_in, W4_BK);

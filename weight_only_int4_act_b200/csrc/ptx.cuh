@@ -74,26 +74,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// mbar_wait for long waits: sleeps `ns` between polls so that a waiting warp
-// leaves the issue slots to the warps that do the work.
-__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err,
-                                                int code, uint32_t ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(ns);
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > AWQ_WAIT_LIMIT_NS) {
-        *abort_flag = 1;
-        if (err) atomicCAS(err, 0, code);
-        return false;
-      }
-    }
-  }
-}
-
 // Same bound, for draining: ignores the abort flag.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();

@@ -16,27 +16,31 @@
 //
 // Tiles are 128 output channels x BN tokens (BN = 16 .. 256): the weights are
 // the M = 128 operand of tcgen05.mma.cta_group::1.kind::f16 and the tokens
-// the N operand, so a decode batch of a few tokens still fills a tile. One
-// K step is 64 channels. Three shared-memory rings, each with its own
-// full/empty mbarriers, so that each stream runs ahead as far as its ring
-// allows: packed codes (4 K steps per stage: 128 rows x 128 B with the
-// 128-byte swizzle, up to 6 stages deep: the weight bytes in flight that hide
-// HBM latency; a box row of a single step's 32 B moved only ~7 GB/s per SM),
-// activations (BN x 64, 128-byte swizzle) and dequantised weights (128 x 64,
-// 128-byte swizzle). Depths depend on BN (host plan). Warp roles (480
-// threads, one CTA per SM):
+// the N operand, so a decode batch of a few tokens still fills a tile. One K
+// step is 128 channels (8 MMAs of K = 16). The dequantised weights never touch
+// shared memory: the dequantising warps write them into tensor memory with
+// tcgen05.st and the MMAs read A from there (lane = output channel, 32-bit
+// column = two consecutive channels), so shared memory carries only the
+// packed codes and the activations. Rings, each with full/empty mbarriers:
+// packed codes in shared memory (two steps per TMA box, 128 rows x 128 B with
+// the 128-byte swizzle: narrow boxes of one step's 32 B per row moved only
+// ~7 GB/s per SM), activations in shared memory (BN x 128 as two 128-byte-
+// swizzled 64-wide boxes), and dequantised weights in tensor memory (64
+// columns a step, behind one or two accumulators). Depths depend on BN (host
+// plan). Warp roles (480 threads, one CTA per SM):
 //   warp 0       TMA of the packed codes;
-//   warp 1       allocates 512 TMEM columns (two accumulators at columns 0
-//                and 256) and one thread issues the MMAs;
+//   warp 1       allocates the 512 TMEM columns and one thread issues the MMAs;
 //   warp 2       TMA of the activation tiles;
-//   warps 3..10  dequantise: thread (h, r) expands words 4h..4h+3 of row r
-//                into the activation type, two codes per packed subtract and
-//                multiply (dequant_word), and stores them in the K-major
-//                swizzled layout the MMA descriptor reads; a proxy fence and
-//                one arrive per warp publish the stage;
+//   warps 3..10  dequantise: warp w, lane l takes output channel
+//                32 (w % 4) + l (its TMEM lane) and the half h = (w - 3) / 4 of
+//                each step's channels, two codes per packed subtract and
+//                multiply (dequant_word), 32 columns per tcgen05.st;
 //   warps 11..14 epilogue: tcgen05.ld of the accumulator (TMEM lane = output
-//                channel, column = token), bf16 stores of Y (or fp32 split-K
+//                channel, column = token), stores of Y (or fp32 split-K
 //                partials), then release of the accumulator.
+// The MMA issuer is the critical path: every other role waits with a short
+// sleep between polls, so that waiting warps leave the issue slots of their
+// scheduler (which the issuer shares with two dequantising warps) free.
 // K may be split across CTAs when there are fewer tiles than SMs; the
 // partials are then summed in split order by a second kernel.
 // Every wait is bounded; on a timeout the CTA records an error in *err,
@@ -51,6 +55,52 @@
 
 namespace awq {
 
+// mbar_wait for long waits: sleeps `ns` between polls so that a waiting warp
+// leaves the issue slots to the warps that do the work.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                                int code, uint32_t ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > AWQ_WAIT_LIMIT_NS) {
+        *abort_flag = 1;
+        if (err) atomicCAS(err, 0, code);
+        return false;
+      }
+    }
+  }
+}
+
+// Each thread of the warp writes 32 consecutive 32-bit columns of its TMEM lane.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16 (A in tensor memory: lane =
+// row of A, 32-bit column = two consecutive K elements).
+__device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 constexpr int W4_BM = 128;
 constexpr int W4_BK = 128;                      // channels per K step: two 64-wide swizzled sub-tiles
 constexpr int W4_SUB = 64;
@@ -58,16 +108,21 @@ constexpr int W4_MAX_BN = 256;
 constexpr int W4_THREADS = 480;
 constexpr int W4_RK = 2;                        // K steps of packed codes per TMA box (128 rows x 128 B)
 constexpr int W4_R_STAGE = W4_BM * 128;         // packed codes, 16 KB
-constexpr int W4_A_SUB = W4_BM * W4_SUB * 2;    // one 128 x 64 sub-tile of dequantised weights, 16 KB
-constexpr int W4_A_STAGE = 2 * W4_A_SUB;        // 32 KB
+constexpr int W4_A_COLS = W4_BK / 2;           // TMEM columns of one step of dequantised weights
 constexpr int W4_MAX_RS = 32, W4_MAX_XS = 8, W4_MAX_AS = 8;
 constexpr int W4_NBARS = 2 * (W4_MAX_RS + W4_MAX_XS + W4_MAX_AS) + 5;
 constexpr int W4_TMEM_COLS = 512;
 constexpr int W4_SMEM_LIMIT = 232448;
 
 // Shared-memory bytes for ring depths (as, xs, rs) at BN tokens.
-__host__ __device__ constexpr int w4_smem_bytes(int as, int xs, int rs, int bn) {
-  return 1024 + as * W4_A_STAGE + xs * bn * W4_BK * 2 + rs * W4_R_STAGE + W4_NBARS * 8 + 64;
+__host__ __device__ constexpr int w4_smem_bytes(int xs, int rs, int bn) {
+  return 1024 + xs * bn * W4_BK * 2 + rs * W4_R_STAGE + W4_NBARS * 8 + 64;
+}
+// TMEM columns: NACC accumulators of acc_stride columns, then the A ring.
+__host__ __device__ constexpr int w4_nacc(int bn) { return bn == 256 ? 1 : 2; }
+__host__ __device__ constexpr int w4_acc_stride(int bn) { return bn < 32 ? 32 : bn; }
+__host__ __device__ constexpr int w4_max_as(int bn) {
+  return (W4_TMEM_COLS - w4_nacc(bn) * w4_acc_stride(bn)) / W4_A_COLS;
 }
 
 constexpr int ERR_W4_RFULL = 0x301, ERR_W4_REMPTY = 0x302, ERR_W4_XFULL = 0x303, ERR_W4_XEMPTY = 0x304,
@@ -188,8 +243,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   const int AS = args.as, XS = args.xs, RS = args.rs;
   const uint32_t x_sub = (uint32_t)bn * W4_SUB * 2;  // one BN x 64 sub-tile; a multiple of 1024
   const uint32_t x_stage = 2 * x_sub;
-  uint8_t* sA = smem;                        // [AS][2][128 rows][128 B], swizzled
-  uint8_t* sX = sA + AS * W4_A_STAGE;        // [XS][2][BN rows][128 B], swizzled
+  uint8_t* sX = smem;                        // [XS][2][BN rows][128 B], swizzled
   uint8_t* sR = sX + XS * x_stage;           // [RS][128 rows][128 B], swizzled
   uint64_t* bars = reinterpret_cast<uint64_t*>(sR + RS * W4_R_STAGE);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + W4_NBARS);
@@ -240,6 +294,8 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int nacc = w4_nacc(bn), acc_stride = w4_acc_stride(bn);
+  const uint32_t a_col0 = (uint32_t)(nacc * acc_stride);  // first TMEM column of the A ring
 
   if (warp == 0 || warp == 2) {
     if (lane == 0) {
@@ -258,7 +314,8 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         for (int kb = kb0; kb < kb1; kb += codes ? W4_RK : 1) {
           const uint32_t full = codes ? rfull(ring.stage) : xfull(ring.stage);
           const uint32_t empty = codes ? rempty(ring.stage) : xempty(ring.stage);
-          if (!mbar_wait(empty, ring.phase ^ 1u, abort_flag, args.err, codes ? ERR_W4_REMPTY : ERR_W4_XEMPTY)) {
+          if (!mbar_wait_sleep(empty, ring.phase ^ 1u, abort_flag, args.err, codes ? ERR_W4_REMPTY : ERR_W4_XEMPTY,
+                               64)) {
             ok = false;
             break;
           }
@@ -285,9 +342,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       // kind::f16 with both operands fp16 (format 0) or both bf16 (format 1)
       const uint32_t idesc = F16 ? ((1u << 4) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(W4_BM >> 4) << 24))
                                  : idesc_bf16_f32(W4_BM, bn);
-      // descriptors of stage 0; a stage, a sub-tile and a K offset only move the
-      // start-address field (address >> 4; all shared addresses are below 256 KB)
-      const uint64_t da0 = desc_kmajor_sw128(smem_u32(sA));
+      // descriptor of activation stage 0; a stage, a sub-tile and a K offset
+      // only move the start-address field (address >> 4; shared addresses are
+      // below 256 KB)
       const uint64_t dx0 = desc_kmajor_sw128(smem_u32(sX));
       Ring xr, ar;
       bool ok = true;
@@ -297,10 +354,11 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         w4_tile_coords(t, args, mb, nb, split);
         const int kb0 = split * args.kb_per_split;
         const int kb1 = min(args.n_kb, kb0 + args.kb_per_split);
-        const int acc = local & 1;
-        if (!mbar_wait(tempty(acc), ((local >> 1) & 1) ^ 1u, abort_flag, args.err, ERR_W4_TEMPTY)) break;
+        const int acc = local % nacc;
+        const uint32_t use = (uint32_t)(local / nacc);
+        if (!mbar_wait(tempty(acc), (use & 1u) ^ 1u, abort_flag, args.err, ERR_W4_TEMPTY)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * 256;
+        const uint32_t d_tmem = tmem_base + acc * acc_stride;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(xfull(xr.stage), xr.phase, abort_flag, args.err, ERR_W4_XFULL) ||
               !mbar_wait(afull(ar.stage), ar.phase, abort_flag, args.err, ERR_W4_AFULL)) {
@@ -308,13 +366,13 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t da = da0 + ((uint64_t)(ar.stage * W4_A_STAGE) >> 4);
+          const uint32_t a_tmem = tmem_base + a_col0 + ar.stage * W4_A_COLS;
           const uint64_t dx = dx0 + ((uint64_t)(xr.stage * x_stage) >> 4);
 #pragma unroll
           for (int k = 0; k < W4_BK / 16; ++k) {
             const uint32_t sub = (uint32_t)(k >> 2), kq = (uint32_t)(k & 3);
-            mma_bf16(d_tmem, da + ((sub * W4_A_SUB + kq * 32) >> 4), dx + ((sub * x_sub + kq * 32) >> 4), idesc,
-                     (kb != kb0) || (k != 0));
+            mma_f16_tmem_a(d_tmem, a_tmem + k * 8, dx + ((sub * x_sub + kq * 32) >> 4), idesc,
+                           (kb != kb0) || (k != 0));
           }
           mma_commit(xempty(xr.stage));
           mma_commit(aempty(ar.stage));
@@ -327,12 +385,12 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       mbar_wait_drain(drain_bar, 0);
     }
   } else if (warp < 11) {
-    // ---------------- dequantisation: thread (h, r) takes channels 64h .. 64h+63
-    // of each step for row r (8 words), i.e. row r of A sub-tile h
-    const int d = threadIdx.x - 3 * 32;
-    const int r = d & (W4_BM - 1);
-    const int h = d >> 7;
-    const uint32_t a_row_off = (uint32_t)(h * W4_A_SUB + r * 128);
+    // ---------------- dequantisation: warp w, lane l takes output channel
+    // r = 32 (w % 4) + l (its TMEM lane) and channels 64h .. 64h+63 of each step
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int h = (warp - 3) >> 2;
+    const uint32_t a_lane = tmem_base + ((uint32_t)(quad * 32) << 16) + a_col0 + (uint32_t)(h * 32);
     const int sw = r & 7;
     Ring rr, ar;
     bool ok = true;
@@ -377,7 +435,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         // step kk of the code box: 16-byte chunks 4 kk + 2h and 4 kk + 2h + 1 of row r, swizzled
         const int kk = (kb - kb0) & (W4_RK - 1);
         bool have = true;
-        if (kk == 0) have = mbar_wait(rfull(rr.stage), rr.phase, abort_flag, args.err, ERR_W4_RFULL);
+        if (kk == 0) have = mbar_wait_sleep(rfull(rr.stage), rr.phase, abort_flag, args.err, ERR_W4_RFULL, 32);
         if (!__all_sync(0xffffffffu, have)) {
           ok = false;
           break;
@@ -391,20 +449,26 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           if (lane == 0) mbar_arrive(rempty(rr.stage));
           rr.next(RS);
         }
-        have = mbar_wait(aempty(ar.stage), ar.phase ^ 1u, abort_flag, args.err, ERR_W4_AEMPTY);
+        have = mbar_wait_sleep(aempty(ar.stage), ar.phase ^ 1u, abort_flag, args.err, ERR_W4_AEMPTY, 32);
         if (!__all_sync(0xffffffffu, have)) {
           ok = false;
           break;
         }
+        tc_fence_after();  // the MMAs that read this A stage have completed
         const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        uint8_t* arow = sA + ar.stage * W4_A_STAGE + a_row_off;
+        uint32_t cols[32];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           constexpr int WPG = 8 / GPH;  // words per group inside the thread's 64 channels
           const uint4 v = dequant_word<F16>(words[c], zc[c / WPG], dc[c / WPG]);
-          *reinterpret_cast<uint4*>(arow + ((c ^ sw) << 4)) = v;
+          cols[4 * c] = v.x;
+          cols[4 * c + 1] = v.y;
+          cols[4 * c + 2] = v.z;
+          cols[4 * c + 3] = v.w;
         }
-        fence_proxy_async_shared();
+        tmem_st_32x32b_x32(a_lane + ar.stage * W4_A_COLS, cols);
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(afull(ar.stage));
         ar.next(AS);
@@ -418,14 +482,15 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x, ++local) {
       int mb, nb, split;
       w4_tile_coords(t, args, mb, nb, split);
-      const int acc = local & 1;
+      const int acc = local % nacc;
+      const uint32_t use = (uint32_t)(local / nacc);
       // the accumulator takes a whole tile: wait without spinning
-      const bool ready = mbar_wait_sleep(tfull(acc), (local >> 1) & 1, abort_flag, args.err, ERR_W4_TFULL, 256);
+      const bool ready = mbar_wait_sleep(tfull(acc), use & 1u, abort_flag, args.err, ERR_W4_TFULL, 256);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
       const int o = mb * W4_BM + r;
       const int t0 = nb * bn;
-      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * 256;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * acc_stride;
       for (int c = 0; c * 32 < bn; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + c * 32, v);
