@@ -262,41 +262,73 @@ def run_ours(args, rank, world, local_rank):
     step_split = {"stats": round(float(api_mean[0]), 4), "search": round(float(api_mean[1]), 4),
                   "pack": round(float(api_mean[2]), 4)}
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers. Every step copies
+    # its inputs (W, X) from pinned host memory and all its results back; the
+    # inputs of step k+1 are copied on a second stream while step k computes
+    # (two device slots for inputs and results, ordered by events).
     Wh = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).pin_memory()
     Xh = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).pin_memory()
-    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in
-                (outs["losses"], outs["best"], outs["s_best"], *packed)]
-    Wd = torch.empty_like(W)
-    Xd = torch.empty_like(X)
+    dev_in = [(torch.empty_like(W), torch.empty_like(X)) for _ in range(2)]
+    dev_out = [dict(losses=torch.empty_like(outs["losses"]), best=torch.empty_like(outs["best"]),
+                    s_best=torch.empty_like(outs["s_best"]), row_losses=None) for _ in range(2)]
+    dev_pack = [tuple(torch.empty_like(t) for t in packed) for _ in range(2)]
+    host_out = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in
+                 (outs["losses"], outs["best"], outs["s_best"], *packed)] for _ in range(2)]
+    comp = torch.cuda.current_stream()
+    cstream = torch.cuda.Stream()
 
-    def e2e_step():
-        Wd.copy_(Wh, non_blocking=True)
-        Xd.copy_(Xh, non_blocking=True)
-        aa = awq.act_stats(Xd, ws_stats, out=a)
-        r = awq.search_scales(Wd, Xd, aa, cfg, ws=ws, outputs=outs)
-        p = awq.quantize_pack(Wd, r["s_best"], cfg, outputs=packed)
-        for h, d in zip(host_out, (r["losses"], r["best"], r["s_best"], *p)):
-            h.copy_(d, non_blocking=True)
+    def e2e_run(n):
+        """n pipelined steps; returns their total device time in ms."""
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        in_ready, done, copied = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(comp)
+        cstream.wait_event(t0)
+        with torch.cuda.stream(cstream):
+            dev_in[0][0].copy_(Wh, non_blocking=True)
+            dev_in[0][1].copy_(Xh, non_blocking=True)
+            in_ready[0].record(cstream)
+        for k in range(n):
+            sl = k % 2
+            comp.wait_event(in_ready[sl])
+            if k >= 2:
+                comp.wait_event(copied[sl])  # step k-2's results have left this slot
+            Wd, Xd = dev_in[sl]
+            aa = awq.act_stats(Xd, ws_stats, out=a)
+            r = awq.search_scales(Wd, Xd, aa, cfg, ws=ws, outputs=dev_out[sl])
+            pk = awq.quantize_pack(Wd, r["s_best"], cfg, outputs=dev_pack[sl])
+            done[sl].record(comp)
+            with torch.cuda.stream(cstream):
+                if k + 1 < n:
+                    nx = (k + 1) % 2
+                    if k >= 1:
+                        cstream.wait_event(done[nx])  # step k-1 no longer reads that slot
+                    dev_in[nx][0].copy_(Wh, non_blocking=True)
+                    dev_in[nx][1].copy_(Xh, non_blocking=True)
+                    in_ready[nx].record(cstream)
+                cstream.wait_event(done[sl])
+                for h, d in zip(host_out[sl], (r["losses"], r["best"], r["s_best"], *pk)):
+                    h.copy_(d, non_blocking=True)
+                copied[sl].record(cstream)
+        comp.wait_event(copied[(n - 1) % 2])
+        if n >= 2:
+            comp.wait_event(copied[(n - 2) % 2])
+        t1.record(comp)
+        t1.synchronize()
+        return t0.elapsed_time(t1)
 
-    for _ in range(2):
-        e2e_step()
+    e2e_run(2)
     torch.cuda.synchronize()
-    e_ms = []
-    for k in range(K):
-        flush.fill_(k & 0xFF)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        e2e_step()
-        e1.record()
-        e1.synchronize()
-        e_ms.append(e0.elapsed_time(e1))
-    e2e_total = float(sum(e_ms))
+    e2e_total = e2e_run(K)
     if world > 1:
         e2e_total = max_over_ranks([e2e_total], dev)[0]
     awq.workspace_error(ws)
+    # the pipelined steps returned what the device-resident steps computed (deterministic kernels)
+    last = host_out[(K - 1) % 2]
+    if not (torch.equal(last[0], outs["losses"].cpu()) and torch.equal(last[1], outs["best"].cpu())):
+        raise RuntimeError("end-to-end results differ from the device-resident run")
     h2d = Wb.nbytes + Xb.nbytes
-    d2h = sum(h.numel() * h.element_size() for h in host_out)
+    d2h = sum(h.numel() * h.element_size() for h in host_out[0])
 
     # ---- per-group clipping with the chosen scales (a follow-on pass, timed apart from the step)
     gclip = None
@@ -450,6 +482,9 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "group_clip": gclip,
         "w4a16": w4,
+        "e2e_note": "each step: H2D of W and X from pinned memory, the search and pack, D2H of every result; "
+                    "step k+1's inputs are copied on a second stream while step k computes; working set "
+                    "(the candidate stack) larger than L2, no flush",
         "gpu_launches": launches_per_step(form, n_a) * K,
         "clocks": clk,
         "wall_s_timed_region": round(t_wall, 3),

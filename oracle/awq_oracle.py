@@ -127,8 +127,15 @@ def quantize_groups(V: np.ndarray, bits: int, group: int, symmetric: bool,
     the step is taken — max|v| -> c max|v| (symmetric), max v -> c max v and
     min v -> c min v (asymmetric) — and values outside the shrunk range clip to
     the extreme codes. c = 1 is the plain quantiser.
+
+    group = 0 is per-tensor quantisation ([P1] 量化基础: one step s = max|W|
+    / (2^(b-1) - 1) for the whole matrix): the flattened matrix is one group,
+    and delta / zero are [1, 1].
     """
     V = np.asarray(V, dtype=np.float64)
+    if group == 0:
+        Vh, codes, delta, zero = quantize_groups(V.reshape(1, -1), bits, V.size, symmetric, eps_delta, clip)
+        return Vh.reshape(V.shape), codes.reshape(V.shape), delta, zero
     rows, d_in = V.shape
     if d_in % group:
         raise ValueError("d_in must be a multiple of the group size")
@@ -370,6 +377,10 @@ def boundary_mask(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symm
     computation may round those either way; everything else must match."""
     W = widen_bf16(W_bits)
     V = W * np.asarray(s, dtype=np.float64)[None, :]
+    if group == 0:  # per tensor: one group of all elements
+        flat = W_bits.reshape(1, -1)
+        s_flat = np.tile(np.asarray(s, dtype=np.float64), W_bits.shape[0])
+        return boundary_mask(flat, s_flat, bits, flat.shape[1], symmetric, band, clip).reshape(W_bits.shape)
     rows, d_in = V.shape
     G = V.reshape(rows, d_in // group, group)
     if symmetric:

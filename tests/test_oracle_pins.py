@@ -687,3 +687,63 @@ def test_w4a16_f16_activations_brute_force():
             acc = sum(X[t, i] * (((int(words[o, i // 8]) >> (4 * (i % 8))) & 0xF) - float(zr[o, i // g]))
                       * float(sc[o, i // g]) for i in range(d_in))
             assert Y[t, o] == pytest.approx(acc, rel=1e-12, abs=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# per-tensor quantisation (group = 0)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("symmetric,bits", [(True, 4), (False, 4), (True, 3), (False, 2)])
+def test_per_tensor_quantiser_brute_force(symmetric, bits):
+    """group = 0: one step for the whole matrix ([P1] 量化基础 for the
+    symmetric case), checked element by element against the textbook formula
+    written with Python scalars."""
+    rng = np.random.default_rng(50 + bits)
+    V = rng.standard_normal((3, 16)) * np.linspace(0.2, 2.0, 16)
+    Vh, codes, delta, zero = O.quantize_groups(V, bits, 0, symmetric)
+    assert delta.shape == (1, 1) and zero.shape == (1, 1)
+    flat = [float(x) for x in V.ravel()]
+    if symmetric:
+        qmax = 2 ** (bits - 1) - 1
+        d = max(abs(x) for x in flat) / qmax
+        for x, vh, c in zip(flat, Vh.ravel(), codes.ravel()):
+            q = min(max(round(x / d), -qmax - 1), qmax)   # Python round: half to even
+            assert vh == pytest.approx(q * d, rel=1e-15, abs=1e-15)
+            assert c == q + qmax + 1
+    else:
+        levels = 2 ** bits - 1
+        d = (max(flat) - min(flat)) / levels
+        z = min(max(round(-min(flat) / d), 0), levels)
+        for x, vh, c in zip(flat, Vh.ravel(), codes.ravel()):
+            q = min(max(round(x / d) + z, 0), levels)
+            assert vh == pytest.approx((q - z) * d, rel=1e-15, abs=1e-15)
+            assert c == q
+
+
+def test_per_tensor_worked_example():
+    """AWQ (scholia-log) §3.1: w_max = 1 anywhere in the tensor gives the INT4
+    step 1/7, and w_i = 0.05 rounds to 0 (output error -0.5 with x_i = 10)."""
+    ex = GOLD["int4_group_example"]
+    W = np.zeros((2, 8))
+    W[1, 3] = ex["w_max"]
+    W[0, 1] = ex["w_i"]
+    Vh, codes, delta, _ = O.quantize_groups(W, 4, 0, True)
+    assert delta[0, 0] == pytest.approx(ex["delta"], rel=1e-15)
+    assert Vh[0, 1] == 0.0
+    assert (Vh[0, 1] - W[0, 1]) * ex["x_i"] == pytest.approx(ex["unscaled_dy"])
+
+
+def test_per_tensor_pack_and_search_shapes():
+    """The search and the pack take group = 0: one fp16 step / zero for the
+    layer; alpha = 0 of the search is plain per-tensor RTN."""
+    rng = np.random.default_rng(53)
+    Wb = gen.f64_to_bf16_bits(rng.standard_normal((4, 32)) * 0.05)
+    Xb = gen.f64_to_bf16_bits(rng.standard_normal((6, 32)))
+    a = O.act_stats(Xb)
+    res = O.search(Wb, Xb, a, 4, 0, True, 4)
+    W = O.widen_bf16(Wb)
+    rtn = O.quantize_groups(W, 4, 0, True)[0]
+    assert res["losses"][0] == pytest.approx(float(((rtn - W) @ O.widen_bf16(Xb).T) ** 2 @ np.ones(6) @ np.ones(4)),
+                                             rel=1e-12)
+    qw, sc, zr, codes, delta, zero = O.pack(Wb, res["s_best"], 4, 0, True)
+    assert sc.shape == (1, 1) and zr.shape == (1, 1) and qw.shape == (4, 4)
+    assert O.boundary_mask(Wb, res["s_best"], 4, 0, True).shape == (4, 32)
