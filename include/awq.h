@@ -56,7 +56,10 @@ typedef enum { AWQ_FORM_AUTO = 0, AWQ_FORM_DIRECT = 1, AWQ_FORM_GRAM = 2 } awq_f
  * zero_point). */
 typedef struct {
   int32_t bits;         /* 2, 3 or 4; codes are stored one per 4-bit nibble */
-  int32_t group;        /* g in {8, 16, 32, 64, 128, 256}; d_in % g == 0 */
+  int32_t group;        /* g in {8, 16, 32, 64, 128, 256}, d_in % g == 0; or 0: per tensor
+                           (one step for the whole layer, as in [P1] 量化基础; d_in % 16
+                           == 0; not for the segmented or group-clip searches nor the
+                           W4A16 product, and the pack needs awq_quantize_pack_ws) */
   int32_t symmetric;    /* 0: min/max affine with zero point; 1: symmetric */
   int32_t n_alpha;      /* grid size, 1..64 */
   int32_t form;         /* awq_form: how the loss contraction is evaluated */
@@ -180,6 +183,16 @@ awq_status awq_quantize_pack(const void* W_bf16, const float* s, int64_t d_out, 
 awq_status awq_quantize_pack_clipped(const void* W_bf16, const float* s, int64_t d_out, int64_t d_in,
                                      const awq_qcfg* cfg, float clip, uint32_t* qweight, void* scales_f16,
                                      void* zeros_f16, awq_stream_t stream);
+
+/* The clipped pack with a workspace (DEVICE, 256-byte aligned, at least
+ * awq_pack_workspace_size bytes): any cfg->group, including 0 (per tensor:
+ * the layer-wide max and min of W S are taken first, and scales / zeros are
+ * [1] each). awq_quantize_pack* without a workspace return AWQ_ERR_WORKSPACE
+ * for group 0. */
+size_t awq_pack_workspace_size(int64_t d_out, int64_t d_in, const awq_qcfg* cfg);
+awq_status awq_quantize_pack_ws(const void* W_bf16, const float* s, int64_t d_out, int64_t d_in,
+                                const awq_qcfg* cfg, float clip, void* ws, size_t ws_bytes, uint32_t* qweight,
+                                void* scales_f16, void* zeros_f16, awq_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * The search over caller-given candidates instead of the a^alpha grid

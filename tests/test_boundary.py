@@ -201,3 +201,23 @@ def test_w4a16_and_fold_validation():
     assert lib.awq_fold_inv_scales(FAKE, 16, FAKE, 2, 1, None) == 1
     assert lib.awq_fold_inv_scales(FAKE, 0, FAKE, 1, 1, None) == 2
     assert lib.awq_fold_inv_scales(FAKE, 16, FAKE, 0, 0, None) == 2
+
+
+def test_per_tensor_validation():
+    lib = awq.lib()
+    big = 1 << 40
+    cfg = awq.make_cfg(4, 0, True, 20)
+    assert awq.search_workspace_size(256, 512, 256, cfg) > 0
+    assert awq.search_workspace_size(256, 520, 256, cfg) == 0          # d_in % 16 for one step per layer
+    assert awq.pack_workspace_size(256, 512, cfg) >= 2 * 512 * 4
+    c = ctypes.byref(cfg)
+    # the pack without a workspace cannot take the layer-wide extremes
+    assert lib.awq_quantize_pack(FAKE, FAKE, 256, 512, c, FAKE, FAKE, FAKE, None) == 3
+    need = awq.pack_workspace_size(256, 512, cfg)
+    assert lib.awq_quantize_pack_ws(FAKE, FAKE, 256, 512, c, 1.0, FAKE, need - 1, FAKE, FAKE, FAKE, None) == 3
+    # one step per layer does not apply to concatenated layers, per-group clipping or the W4A16 product
+    arr = (ctypes.c_int64 * 2)(128, 128)
+    assert lib.awq_search_scales_segmented(FAKE, FAKE, FAKE, 256, 512, 256, c, 2, ctypes.cast(arr, ctypes.c_void_p),
+                                           FAKE, big, FAKE, FAKE, FAKE, None, None) == 7
+    assert awq.group_clip_workspace_size(256, 512, 256, cfg) == 0
+    assert awq.w4a16_workspace_size(16, 256, 512, cfg) == 0

@@ -28,6 +28,7 @@ EXPORTED = (
     "awq_debug_copy_dw", "awq_act_stats_noalloc", "awq_search_scales_segmented", "awq_search_candidates",
     "awq_quantize_pack_clipped", "awq_group_clip_workspace_size", "awq_search_group_clip",
     "awq_quantize_pack_group_clip", "awq_fold_inv_scales", "awq_w4a16_workspace_size", "awq_w4a16_gemm",
+    "awq_pack_workspace_size", "awq_quantize_pack_ws",
 )
 
 
@@ -90,6 +91,9 @@ def lib() -> ctypes.CDLL:
             "awq_w4a16_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, cfgp]),
             "awq_w4a16_gemm": (c_int32, [c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_int64,
                                          cfgp, c_void_p, c_void_p, c_size_t, c_void_p]),
+            "awq_pack_workspace_size": (c_size_t, [c_int64, c_int64, cfgp]),
+            "awq_quantize_pack_ws": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_float, c_void_p,
+                                               c_size_t, c_void_p, c_void_p, c_void_p, c_void_p]),
             "awq_workspace_error": (c_int32, [c_void_p, c_void_p]),
             "awq_quantize_pack": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_void_p, c_void_p,
                                             c_void_p, c_void_p]),
@@ -391,19 +395,29 @@ def debug_dw(ws, d_out, d_in, N, cfg, k):
 
 
 # --------------------------------------------------------------------------- a7
-def quantize_pack(W, s, cfg: QCfg, outputs=None, clip=1.0):
-    """(qweight int32 view of uint32 [d_out, d_in/8], scales fp16 [d_out, d_in/g], zeros fp16 [d_out, d_in/g])."""
+def pack_workspace_size(d_out, d_in, cfg: QCfg) -> int:
+    return int(lib().awq_pack_workspace_size(d_out, d_in, ctypes.byref(cfg)))
+
+
+def quantize_pack(W, s, cfg: QCfg, outputs=None, clip=1.0, ws=None):
+    """(qweight int32 view of uint32 [d_out, d_in/8], scales fp16 [d_out, d_in/g], zeros fp16 [d_out, d_in/g]);
+    per tensor (cfg.group == 0): scales and zeros are [1, 1] and a workspace is used."""
     torch = _torch()
     _req(W, torch.bfloat16, None, "W")
     d_out, d_in = W.shape
     _req(s, torch.float32, (d_in,), "s")
     if outputs is None:
-        ng = d_in // cfg.group if cfg.group > 0 else 0
+        shape = (d_out, d_in // cfg.group) if cfg.group > 0 else (1, 1)
         outputs = (torch.empty((d_out, d_in // 8), dtype=torch.int32, device=W.device),
-                   torch.empty((d_out, ng), dtype=torch.float16, device=W.device),
-                   torch.empty((d_out, ng), dtype=torch.float16, device=W.device))
+                   torch.empty(shape, dtype=torch.float16, device=W.device),
+                   torch.empty(shape, dtype=torch.float16, device=W.device))
     q, sc, zr = outputs
-    if clip == 1.0:
+    if cfg.group == 0 or ws is not None:
+        if ws is None:
+            ws = workspace(pack_workspace_size(d_out, d_in, cfg))
+        _check(lib().awq_quantize_pack_ws(_ptr(W), _ptr(s), d_out, d_in, ctypes.byref(cfg), float(clip), _ptr(ws),
+                                          ws.numel(), _ptr(q), _ptr(sc), _ptr(zr), _stream()), "awq_quantize_pack_ws")
+    elif clip == 1.0:
         _check(lib().awq_quantize_pack(_ptr(W), _ptr(s), d_out, d_in, ctypes.byref(cfg), _ptr(q), _ptr(sc), _ptr(zr),
                                        _stream()), "awq_quantize_pack")
     else:

@@ -35,8 +35,8 @@ inline cudaStream_t as_stream(awq_stream_t s) { return reinterpret_cast<cudaStre
 awq_status check_cfg(const awq_qcfg* cfg) {
   if (!cfg) return AWQ_ERR_INVALID_ARG;
   if (cfg->bits < 2 || cfg->bits > 4) return AWQ_ERR_INVALID_ARG;
-  const int g = cfg->group;
-  if (g < 8 || g > 256 || (g & (g - 1)) != 0) return AWQ_ERR_INVALID_ARG;
+  const int g = cfg->group;  // 0: one step for the whole layer (per tensor)
+  if (g != 0 && (g < 8 || g > 256 || (g & (g - 1)) != 0)) return AWQ_ERR_INVALID_ARG;
   if (cfg->symmetric != 0 && cfg->symmetric != 1) return AWQ_ERR_INVALID_ARG;
   if (cfg->n_alpha < 1 || cfg->n_alpha > MAX_ALPHA) return AWQ_ERR_INVALID_ARG;
   if (cfg->form < AWQ_FORM_AUTO || cfg->form > AWQ_FORM_GRAM) return AWQ_ERR_INVALID_ARG;
@@ -52,7 +52,7 @@ awq_status check_cfg(const awq_qcfg* cfg) {
 // keep every index of the kernels and TMA coordinates inside int32.
 awq_status check_layer_shape(int64_t d_out, int64_t d_in, const awq_qcfg* cfg) {
   if (d_out < 1 || d_in < 8 || d_in % 8 != 0) return AWQ_ERR_SHAPE;
-  if (d_in % cfg->group != 0) return AWQ_ERR_SHAPE;
+  if (cfg->group == 0 ? d_in % FQ_CPT != 0 : d_in % cfg->group != 0) return AWQ_ERR_SHAPE;
   if (d_in > (1 << 20) || d_out > (1 << 24)) return AWQ_ERR_SHAPE;
   const long long M = (long long)cfg->n_alpha * cdiv(d_out, GEMM_BM) * GEMM_BM;
   if (M > (long long)INT32_MAX / 2) return AWQ_ERR_SHAPE;
@@ -113,7 +113,7 @@ struct SearchLayout {
   long long M;      // rows of the dW stack
   int n_blocks_n;   // column tiles of the contraction
   int n_red_chunks; // blocks per alpha in the row reduction
-  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_seg, off_g, total;
+  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_seg, off_ext, off_g, total;
 };
 
 // sum over 256-wide column blocks J of width(J) * min(d_in, 256 (J + 1)): the
@@ -136,6 +136,12 @@ int choose_form(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg) {
   return direct <= gram ? AWQ_FORM_DIRECT : AWQ_FORM_GRAM;
 }
 
+// Per-tensor scratch: keys of the column max and min of W [d_in] each, then
+// the extremes (max, min) of every candidate [MAX_ALPHA][2].
+size_t ext_bytes(int64_t d_in) {
+  return align_up((size_t)2 * d_in * sizeof(uint32_t)) + align_up((size_t)2 * MAX_ALPHA * sizeof(float));
+}
+
 SearchLayout search_layout(int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg) {
   SearchLayout L{};
   L.form = choose_form(d_out, d_in, N, cfg);
@@ -152,6 +158,7 @@ SearchLayout search_layout(int64_t d_out, int64_t d_in, int64_t N, const awq_qcf
   L.off_blk = off;    off += align_up((size_t)L.n_alpha * L.n_red_chunks * sizeof(double));
   L.off_loss64 = off; off += align_up((size_t)L.n_alpha * sizeof(double));
   L.off_seg = off;    off += align_up((size_t)MAX_ALPHA * MAX_SEG * sizeof(double));
+  L.off_ext = off;    off += ext_bytes(d_in);  // per tensor: column extremes and candidate extremes
   if (L.form == AWQ_FORM_GRAM) {
     L.off_g = off;    off += align_up((size_t)d_in * d_in * 2);
   }
@@ -369,6 +376,32 @@ awq_status awq_step_scales(const float* a, int64_t d_out, int64_t d_in, int64_t 
   return launch_status();
 }
 
+// Per-tensor extremes into the scratch at `ext_ws` (ext_bytes(d_in)): column
+// max / min of W, then (max, min) of v = w s for each of the n scale vectors
+// s_all[n][d_in], at ext_table(ext_ws, d_in).
+float* ext_table(void* ext_ws, int64_t d_in) {
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(ext_ws) + align_up((size_t)2 * d_in * sizeof(uint32_t)));
+}
+
+awq_status launch_tensor_extremes(const void* W, int64_t d_out, int64_t d_in, const float* s_all, int n,
+                                  void* ext_ws, int sms, cudaStream_t st) {
+  uint32_t* kmax = static_cast<uint32_t*>(ext_ws);
+  uint32_t* kmin = kmax + d_in;
+  if (cudaMemsetAsync(kmax, 0, (size_t)d_in * sizeof(uint32_t), st) != cudaSuccess ||
+      cudaMemsetAsync(kmin, 0xFF, (size_t)d_in * sizeof(uint32_t), st) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  const int xb = (int)cdiv(d_in / 8, 256);
+  long long yb = (4LL * sms + xb - 1) / xb;
+  if (yb > d_out) yb = d_out;
+  if (yb < 1) yb = 1;
+  const int rows_per_block = (int)cdiv(d_out, yb);
+  yb = cdiv(d_out, rows_per_block);
+  col_minmax<<<dim3(xb, (unsigned)yb), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in,
+                                                     rows_per_block, kmax, kmin);
+  tensor_extremes<<<n, 256, 0, st>>>(kmax, kmin, s_all, (int)d_in, ext_table(ext_ws, d_in));
+  return launch_status();
+}
+
 // Fake quantisation of grid points [k0, k1) into their slices of the dW stack.
 // max_per_sm > 0 caps the grid at that many blocks per SM.
 awq_status launch_fake_quant(const void* W, int64_t d_out, int64_t d_in, const awq_qcfg* cfg, const SearchLayout& L,
@@ -379,6 +412,14 @@ awq_status launch_fake_quant(const void* W, int64_t d_out, int64_t d_in, const a
   if (clip_table)
     for (int k = k0; k < k1; ++k) clips.c[k - k0] = clip_table->c[k];
   const long long slice = (long long)L.d_out_pad * d_in;
+  float* ext = nullptr;
+  if (cfg->group == 0) {
+    // per tensor: the layer-wide extremes of every candidate first
+    awq_status es = launch_tensor_extremes(W, d_out, d_in, at<float>(ws, L.off_s) + (long long)k0 * d_in, k1 - k0,
+                                           at<void>(ws, L.off_ext), sms, st);
+    if (es != AWQ_OK) return es;
+    ext = ext_table(at<void>(ws, L.off_ext), d_in);
+  }
   auto launch = [&](auto kernel, int cpt) {
     const long long units = (long long)(L.d_out_pad / FQ_ROWS) * (d_in / cpt);
     int grid = elementwise_grid(kernel, units, sms);
@@ -386,10 +427,11 @@ awq_status launch_fake_quant(const void* W, int64_t d_out, int64_t d_in, const a
     kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), (int)d_out, (int)d_in, L.d_out_pad,
                                  at<float>(ws, L.off_s) + (long long)k0 * d_in,
                                  at<float>(ws, L.off_inv) + (long long)k0 * d_in, k1 - k0, cfg->bits,
-                                 cfg->symmetric, at<__nv_bfloat16>(ws, L.off_dw) + k0 * slice, clips);
+                                 cfg->symmetric, at<__nv_bfloat16>(ws, L.off_dw) + k0 * slice, clips, ext);
   };
   constexpr int C = FQ_CPT;
   switch (cfg->group) {
+    case 0: launch(fake_quant_delta<C, FQ_ROWS, 1, true>, C); break;
     case 8: launch(fake_quant_delta<8, FQ_ROWS, 1>, 8); break;
     case 16: launch(fake_quant_delta<(C < 16 ? C : 16), FQ_ROWS, 16 / (C < 16 ? C : 16)>, (C < 16 ? C : 16)); break;
     case 32: launch(fake_quant_delta<(C < 32 ? C : 32), FQ_ROWS, 32 / (C < 32 ? C : 32)>, (C < 32 ? C : 32)); break;
@@ -506,6 +548,7 @@ awq_status awq_search_scales_segmented(const void* W, const void* X, const float
   if (!W || !X || !a || !losses || !best || !s_best || !seg_rows) return AWQ_ERR_INVALID_ARG;
   if (!aligned(W, 16) || !aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
   if (n_seg < 1 || n_seg > MAX_SEG) return AWQ_ERR_INVALID_ARG;
+  if (cfg->group == 0) return AWQ_ERR_UNSUPPORTED;  // one step per layer would span the segments
   SegTable seg{};
   int64_t acc = 0;
   for (int i = 0; i < n_seg; ++i) {
@@ -644,25 +687,36 @@ awq_status awq_workspace_error(void* ws, awq_stream_t stream) {
 
 awq_status pack_impl(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg, float clip,
                      const uint8_t* group_clip, const ClipTable& gtable, uint32_t* qweight, void* scales, void* zeros,
-                     awq_stream_t stream) {
+                     awq_stream_t stream, void* ws = nullptr, size_t ws_bytes = 0) {
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if ((st = check_layer_shape(d_out, d_in, cfg)) != AWQ_OK) return st;
+  if (cfg->group == 0) {  // per tensor: the extremes need scratch
+    if (!ws || !aligned(ws, 256)) return ws ? AWQ_ERR_INVALID_ARG : AWQ_ERR_WORKSPACE;
+    if (ws_bytes < ext_bytes(d_in)) return AWQ_ERR_WORKSPACE;
+    if (group_clip) return AWQ_ERR_UNSUPPORTED;
+  }
   if (!(clip > 0.f && clip <= 1.f)) return AWQ_ERR_INVALID_ARG;
   if (!W || !s || !qweight || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
   if (!aligned(W, 16) || !aligned(s, 16) || !aligned(qweight, 4) || !aligned(scales, 2) || !aligned(zeros, 2))
     return AWQ_ERR_INVALID_ARG;
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;
+  const float* ext = nullptr;
+  if (cfg->group == 0) {
+    if ((st = launch_tensor_extremes(W, d_out, d_in, s, 1, ws, sms, as_stream(stream))) != AWQ_OK) return st;
+    ext = ext_table(ws, d_in);
+  }
   auto launch = [&](auto kernel, int cpt) {
     const long long units = cdiv(d_out, PACK_ROWS) * (d_in / cpt);
     const int grid = elementwise_grid(kernel, units, sms);
     kernel<<<grid, 256, 0, as_stream(stream)>>>(static_cast<const __nv_bfloat16*>(W), s, (int)d_out, (int)d_in,
                                                 cfg->bits, cfg->symmetric, qweight, static_cast<__half*>(scales),
-                                                static_cast<__half*>(zeros), clip, group_clip, gtable);
+                                                static_cast<__half*>(zeros), clip, group_clip, gtable, ext);
   };
   constexpr int C = FQ_CPT;
   switch (cfg->group) {
+    case 0: launch(quantize_pack<C, 1, true>, C); break;
     case 8: launch(quantize_pack<8, 1>, 8); break;
     case 16: launch(quantize_pack<(C < 16 ? C : 16), 16 / (C < 16 ? C : 16)>, (C < 16 ? C : 16)); break;
     case 32: launch(quantize_pack<(C < 32 ? C : 32), 32 / (C < 32 ? C : 32)>, (C < 32 ? C : 32)); break;
@@ -683,6 +737,18 @@ awq_status awq_quantize_pack_clipped(const void* W, const float* s, int64_t d_ou
 awq_status awq_quantize_pack(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
                              uint32_t* qweight, void* scales, void* zeros, awq_stream_t stream) {
   return awq_quantize_pack_clipped(W, s, d_out, d_in, cfg, 1.0f, qweight, scales, zeros, stream);
+}
+
+size_t awq_pack_workspace_size(int64_t d_out, int64_t d_in, const awq_qcfg* cfg) {
+  if (check_cfg(cfg) != AWQ_OK || check_layer_shape(d_out, d_in, cfg) != AWQ_OK) return 0;
+  return cfg->group == 0 ? ext_bytes(d_in) : 256;
+}
+
+awq_status awq_quantize_pack_ws(const void* W, const float* s, int64_t d_out, int64_t d_in, const awq_qcfg* cfg,
+                                float clip, void* ws, size_t ws_bytes, uint32_t* qweight, void* scales, void* zeros,
+                                awq_stream_t stream) {
+  ClipTable none{};
+  return pack_impl(W, s, d_out, d_in, cfg, clip, nullptr, none, qweight, scales, zeros, stream, ws, ws_bytes);
 }
 
 awq_status awq_quantize_pack_group_clip(const void* W, const float* s, const float* clips, int32_t n_clips,

@@ -180,12 +180,14 @@ struct ClipTable {
   float c[MAX_ALPHA];  // clip ratio of each candidate (1: none)
 };
 
-template <int CPT, int ROWS, int GL>
+// PT (per tensor): every candidate's step comes from the layer-wide extremes
+// ext[2k] = max v, ext[2k+1] = min v (tensor_extremes) instead of a group.
+template <int CPT, int ROWS, int GL, bool PT = false>
 __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* __restrict__ W, int d_out, int d_in,
                                                            int d_out_pad, const float* __restrict__ s_all,
                                                            const float* __restrict__ inv_all, int n_alpha, int bits,
                                                            int symmetric, __nv_bfloat16* __restrict__ dW,
-                                                           ClipTable clips) {
+                                                           ClipTable clips, const float* __restrict__ ext) {
   const int chunks = d_in / CPT;
   const long long total = (long long)(d_out_pad / ROWS) * chunks;
   const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -224,7 +226,10 @@ __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* 
 #pragma unroll
         for (int j = 0; j < CPT; ++j) v[j] = w[r][j] * s[j];
         FqGroup<CPT> fr;
-        fq_group<CPT, GL>(v, bits, sym, fr, clips.c[k]);
+        if constexpr (PT)
+          fq_from_extremes<CPT>(v, bits, sym, fr, ext[2 * k], ext[2 * k + 1], clips.c[k]);
+        else
+          fq_group<CPT, GL>(v, bits, sym, fr, clips.c[k]);
 #pragma unroll
         for (int q = 0; q < CPT / 8; ++q) {
           uint32_t out[4];
@@ -399,6 +404,88 @@ __global__ void segment_argmin(const double* __restrict__ seg_sums, int n_seg, i
 }
 
 // ---------------------------------------------------------------------------
+// Per-tensor quantisation: the layer-wide extremes of v = w s for each
+// candidate. With every s_i > 0, max over (r, i) of fp32(w[r, i] s_i) is
+// max over i of fp32(colmax_i s_i) (fp32 rounding is monotone), so one pass
+// over W for column extremes serves every candidate.
+// ---------------------------------------------------------------------------
+// Order-preserving map of floats to unsigned keys (for atomicMax / atomicMin).
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord_val(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// kmax[i] / kmin[i]: keys of max / min over rows of column i (kmax zeroed,
+// kmin filled with 0xFF before the launch). Thread: 8 columns x a row block.
+__global__ void col_minmax(const __nv_bfloat16* __restrict__ W, int d_out, int d_in, int rows_per_block,
+                           uint32_t* __restrict__ kmax, uint32_t* __restrict__ kmin) {
+  const int c8 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (c8 >= d_in) return;
+  const int r0 = blockIdx.y * rows_per_block;
+  const int r1 = min(d_out, r0 + rows_per_block);
+  float mx[8], mn[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    mx[j] = -INFINITY;
+    mn[j] = INFINITY;
+  }
+  for (int r = r0; r < r1; ++r) {
+    float f[8];
+    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(W + (long long)r * d_in + c8)), f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      mx[j] = fmaxf(mx[j], f[j]);
+      mn[j] = fminf(mn[j], f[j]);
+    }
+  }
+  if (r0 >= r1) return;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    atomicMax(&kmax[c8 + j], ord_key(mx[j]));
+    atomicMin(&kmin[c8 + j], ord_key(mn[j]));
+  }
+}
+
+// ext[2k] = max_i fp32(colmax_i s_k[i]), ext[2k + 1] = min_i fp32(colmin_i s_k[i]);
+// one block per candidate.
+__global__ void tensor_extremes(const uint32_t* __restrict__ kmax, const uint32_t* __restrict__ kmin,
+                                const float* __restrict__ s_all, int d_in, float* __restrict__ ext) {
+  const float* s = s_all + (long long)blockIdx.x * d_in;
+  float mx = -INFINITY, mn = INFINITY;
+  for (int i = threadIdx.x; i < d_in; i += blockDim.x) {
+    mx = fmaxf(mx, ord_val(kmax[i]) * s[i]);
+    mn = fminf(mn, ord_val(kmin[i]) * s[i]);
+  }
+  __shared__ float smx[32], smn[32];
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    smx[warp] = mx;
+    smn[warp] = mn;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    mx = lane < nw ? smx[lane] : -INFINITY;
+    mn = lane < nw ? smn[lane] : INFINITY;
+    for (int o = 16; o > 0; o >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    if (lane == 0) {
+      ext[2 * blockIdx.x] = mx;
+      ext[2 * blockIdx.x + 1] = mn;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Per-group clipping search. s_all[k] = s, inv_all[k] = 1/s for k < n.
 // ---------------------------------------------------------------------------
 __global__ void repeat_scales(const float* __restrict__ s, int d_in, int n, float* __restrict__ s_all,
@@ -453,12 +540,15 @@ __global__ void group_clip_argmin(const float* __restrict__ part, long long part
 // in flight per thread). Each row yields CPT/8 consecutive words.
 constexpr int PACK_ROWS = 4;
 
-template <int CPT, int GL>
+// PT (per tensor): the step from the layer-wide extremes ext[0] = max v,
+// ext[1] = min v; one step and zero point (scales[0], zeros[0]).
+template <int CPT, int GL, bool PT = false>
 __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __restrict__ W, const float* __restrict__ s,
                                                      int d_out, int d_in, int bits, int symmetric,
                                                      uint32_t* __restrict__ qweight, __half* __restrict__ scales,
                                                      __half* __restrict__ zeros, float clip,
-                                                     const uint8_t* __restrict__ group_clip, ClipTable clips) {
+                                                     const uint8_t* __restrict__ group_clip, ClipTable clips,
+                                                     const float* __restrict__ ext) {
   const int chunks = d_in / CPT;
   const int row_groups = (d_out + PACK_ROWS - 1) / PACK_ROWS;
   const long long total = (long long)row_groups * chunks;
@@ -502,7 +592,10 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
         c = idx < MAX_ALPHA ? clips.c[idx] : 1.0f;
       }
       FqGroup<CPT> fr;
-      fq_group<CPT, GL>(v, bits, sym, fr, c);
+      if constexpr (PT)
+        fq_from_extremes<CPT>(v, bits, sym, fr, ext[0], ext[1], c);
+      else
+        fq_group<CPT, GL>(v, bits, sym, fr, c);
       if (active && row0 + r < d_out) {
         const int row = row0 + r;
         uint32_t* wp = qweight + (long long)row * words + c0 / 8;
@@ -513,8 +606,8 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
           for (int j = 0; j < 8; ++j) word |= (fq_code(fr, 8 * q + j) & 0xFu) << (4 * j);
           __stcs(wp + q, word);
         }
-        if ((chunk & (GL - 1)) == 0) {
-          const long long gidx = (long long)row * groups + chunk / GL;
+        if (PT ? (row == 0 && chunk == 0) : (chunk & (GL - 1)) == 0) {
+          const long long gidx = PT ? 0 : (long long)row * groups + chunk / GL;
           scales[gidx] = __float2half_rn(fr.delta);
           zeros[gidx] = __float2half_rn(fr.zero);
         }
