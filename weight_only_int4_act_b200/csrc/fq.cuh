@@ -96,32 +96,34 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   return d;
 }
 
+// Quantise this thread's CPT values of a group spread over GL lanes.
 // The clamp to the code range is done on the FMA pipe: with span = 2^b - 1
 // codes, y = sat((v / Delta + z) / span) is clamp(v / Delta + z, 0, span) / span,
 // and fma(y, span, 1.5*2^23) rounds y * span to the nearest integer (ties to
 // even) in magic form. This equals clamp(rne(v / Delta) + z, 0, span) except
 // where v / Delta lies within ~1e-6 of a rounding boundary.
-
-// Step, zero point and codes of CPT values from their group's clipped range:
-// symmetric: hi = max |v| (lo unused); asymmetric: [lo, hi] = [min v, max v].
-template <int CPT>
-__device__ __forceinline__ void fq_core(const float (&v)[CPT], int bits, bool symmetric, FqGroup<CPT>& r, float hi,
-                                        float lo) {
+// clip in (0, 1] shrinks the group's range before the step is taken (1: none).
+template <int CPT, int GL>
+__device__ __forceinline__ void fq_group(const float (&v)[CPT], int bits, bool symmetric, FqGroup<CPT>& r,
+                                         float clip = 1.0f) {
   const float span = (float)((1 << bits) - 1);
   const float inv_span = inv_levels(bits);
   float a, b;  // y = sat(v * a + b)
   if (symmetric) {
+    const float amax = clip * group_max<GL>(fmaxf(maxN(v), -minN(v)));
     const float half = (float)(1 << (bits - 1));  // -qmin
-    r.delta = fmaxf(hi, kEpsDelta) * inv_levels(bits - 1);
+    r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
     const float inv = __frcp_rn(r.delta);
     r.zero = half;
     r.off = kRoundMagic + half;
     a = inv * inv_span;
     b = half * inv_span;  // q - qmin = rne(v / Delta) + 2^(b-1)
   } else {
-    r.delta = fmaxf(hi - lo, kEpsDelta) * inv_span;
+    const float mx = clip * group_max<GL>(maxN(v));
+    const float mn = clip * group_min<GL>(minN(v));
+    r.delta = fmaxf(mx - mn, kEpsDelta) * inv_span;
     const float inv = __frcp_rn(r.delta);
-    r.zero = fminf(fmaxf(__fmaf_rn(-lo, inv, kRoundMagic) - kRoundMagic, 0.f), span);  // clamp(rne(-min / Delta))
+    r.zero = fminf(fmaxf(__fmaf_rn(-mn, inv, kRoundMagic) - kRoundMagic, 0.f), span);  // clamp(rne(-min / Delta))
     r.off = kRoundMagic + r.zero;
     a = inv * inv_span;
     b = r.zero * inv_span;
@@ -130,28 +132,37 @@ __device__ __forceinline__ void fq_core(const float (&v)[CPT], int bits, bool sy
   for (int j = 0; j < CPT; ++j) r.c[j] = __fmaf_rn(fma_sat(v[j], a, b), span, kRoundMagic);
 }
 
-// Quantise this thread's CPT values of a group spread over GL lanes (the
-// group's extremes by shuffles over those lanes); clip in (0, 1] shrinks the
-// range before the step is taken (1: none).
-template <int CPT, int GL>
-__device__ __forceinline__ void fq_group(const float (&v)[CPT], int bits, bool symmetric, FqGroup<CPT>& r,
-                                         float clip = 1.0f) {
-  float hi, lo = 0.f;
-  if (symmetric) {
-    hi = clip * group_max<GL>(fmaxf(maxN(v), -minN(v)));
-  } else {
-    hi = clip * group_max<GL>(maxN(v));
-    lo = clip * group_min<GL>(minN(v));
-  }
-  fq_core<CPT>(v, bits, symmetric, r, hi, lo);
-}
-
-// The same with the group's extremes given (mx = max v, mn = min v, e.g. of
-// the whole layer).
+// The same quantiser with the group's extremes given (mx = max v, mn = min v;
+// e.g. of the whole layer for per-tensor quantisation) instead of reduced over
+// lanes: the formulas of fq_group, kept apart so that fq_group's code (the
+// search's hot loop) stays as it is.
 template <int CPT>
 __device__ __forceinline__ void fq_from_extremes(const float (&v)[CPT], int bits, bool symmetric, FqGroup<CPT>& r,
                                                  float mx, float mn, float clip) {
-  fq_core<CPT>(v, bits, symmetric, r, clip * (symmetric ? fmaxf(mx, -mn) : mx), clip * mn);
+  const float span = (float)((1 << bits) - 1);
+  const float inv_span = inv_levels(bits);
+  float a, b;
+  if (symmetric) {
+    const float amax = clip * fmaxf(mx, -mn);
+    const float half = (float)(1 << (bits - 1));
+    r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
+    const float inv = __frcp_rn(r.delta);
+    r.zero = half;
+    r.off = kRoundMagic + half;
+    a = inv * inv_span;
+    b = half * inv_span;
+  } else {
+    mx *= clip;
+    mn *= clip;
+    r.delta = fmaxf(mx - mn, kEpsDelta) * inv_span;
+    const float inv = __frcp_rn(r.delta);
+    r.zero = fminf(fmaxf(__fmaf_rn(-mn, inv, kRoundMagic) - kRoundMagic, 0.f), span);
+    r.off = kRoundMagic + r.zero;
+    a = inv * inv_span;
+    b = r.zero * inv_span;
+  }
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) r.c[j] = __fmaf_rn(fma_sat(v[j], a, b), span, kRoundMagic);
 }
 
 // Dequantised value v_hat of element j ((q - z) Delta, or q Delta when symmetric).
