@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/awq.h"
 #include "awq_kernels.cuh"
@@ -880,29 +881,32 @@ namespace {
 constexpr int kW4TargetCtas = 148;  // split K until the tiles cover this many CTAs
 
 struct W4Plan {
-  int bn, n_mb, n_nb, n_kb, splits, kb_per_split;
+  int bn, bk, n_mb, n_nb, n_kb, splits, kb_per_split;
   int as, xs, rs;  // ring depths
   long long tiles, p_stride;
   int smem;
   size_t ws;
 };
 
-W4Plan w4_plan(int64_t N, int64_t d_out, int64_t d_in) {
+W4Plan w4_plan(int64_t N, int64_t d_out, int64_t d_in, int group) {
   W4Plan p{};
   p.bn = N <= 16 ? 16 : N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
   // ring depths: deep packed-code rings for narrow (weight-streaming) tiles
-  // Ring depths: codes and activations in shared memory, dequantised weights
-  // in the tensor-memory columns the accumulators leave (an MMA's commit lands
-  // about a microsecond after issue and holds its stages until then).
-  if (p.bn <= 32) { p.xs = 8; p.rs = 6; }
-  else if (p.bn == 64) { p.xs = 6; p.rs = 4; }
+  // K steps of 256 channels for decode-width tiles (16 MMAs per handshake),
+  // 128 otherwise (a 256-wide activation stage of 256 tokens would take
+  // 128 KB). Ring depths: codes and activations in shared memory, dequantised
+  // weights in the tensor-memory columns the accumulators leave (an MMA's
+  // commit lands about a microsecond after issue and holds its stages).
+  p.bk = p.bn <= 64 && group > 8 ? 256 : 128;  // g = 8 keeps 128 (sixteen groups a thread would spill)
+  if (p.bn <= 32) { p.xs = p.bn == 16 ? 8 : 6; p.rs = 6; }
+  else if (p.bn == 64) { p.xs = 4; p.rs = 4; }
   else if (p.bn == 128) { p.xs = 4; p.rs = 4; }
   else { p.xs = 3; p.rs = 2; }
-  p.as = w4_max_as(p.bn) < W4_MAX_AS ? w4_max_as(p.bn) : W4_MAX_AS;
-  p.smem = w4_smem_bytes(p.xs, p.rs, p.bn);
+  p.as = w4_max_as(p.bn, p.bk) < W4_MAX_AS ? w4_max_as(p.bn, p.bk) : W4_MAX_AS;
+  p.smem = w4_smem_bytes(p.xs, p.rs, p.bn, p.bk);
   p.n_mb = (int)cdiv(d_out, W4_BM);
   p.n_nb = (int)cdiv(N, p.bn);
-  p.n_kb = (int)cdiv(d_in, W4_BK);
+  p.n_kb = (int)cdiv(d_in, p.bk);
   const long long mn = (long long)p.n_mb * p.n_nb;
   int splits = 1;
   if (mn < kW4TargetCtas) {
@@ -927,14 +931,14 @@ awq_status check_w4(int64_t N, int64_t d_out, int64_t d_in, const awq_qcfg* cfg)
   if (d_in % 32 != 0 || d_in % g != 0) return AWQ_ERR_SHAPE;  // packed rows: a multiple of 16 bytes
   if (d_in > (1 << 20) || d_out > (1 << 24) || N > (1 << 24)) return AWQ_ERR_SHAPE;
   if ((long long)N * d_out > (long long)INT32_MAX * 4) return AWQ_ERR_SHAPE;
-  if (w4_plan(N, d_out, d_in).tiles > INT32_MAX) return AWQ_ERR_SHAPE;
+  if (w4_plan(N, d_out, d_in, cfg->group).tiles > INT32_MAX) return AWQ_ERR_SHAPE;
   return AWQ_OK;
 }
 }  // namespace
 
 extern "C" size_t awq_w4a16_workspace_size(int64_t N, int64_t d_out, int64_t d_in, const awq_qcfg* cfg) {
   if (check_w4(N, d_out, d_in, cfg) != AWQ_OK) return 0;
-  return w4_plan(N, d_out, d_in).ws;
+  return w4_plan(N, d_out, d_in, cfg->group).ws;
 }
 
 extern "C" awq_status awq_w4a16_gemm(const void* X, awq_dtype dtype, const uint32_t* qweight, const void* scales,
@@ -948,7 +952,7 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, awq_dtype dtype, const uint3
   if (!aligned(X, 16) || !aligned(qweight, 16) || !aligned(scales, 2) || !aligned(zeros, 2) || !aligned(Y, 16) ||
       !aligned(ws, 256))
     return AWQ_ERR_INVALID_ARG;
-  const W4Plan p = w4_plan(N, d_out, d_in);
+  const W4Plan p = w4_plan(N, d_out, d_in, cfg->group);
   if (ws_bytes < p.ws) return AWQ_ERR_WORKSPACE;
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;
@@ -991,22 +995,29 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, awq_dtype dtype, const uint3
     kernel<<<grid, W4_THREADS, p.smem, cs>>>(tx, tw, a);
     return launch_status();
   };
-  // template argument: quantisation groups per 64 channels
-  if (f16) {
+  // template arguments: quantisation groups per BK / 2 channels, activation type, K step
+  auto dispatch = [&](auto f16_tag, auto bk_tag) -> awq_status {
+    constexpr bool F = decltype(f16_tag)::value;
+    constexpr int K = decltype(bk_tag)::value;
+    constexpr int H = K / 2;  // channels per dequantising thread and step
     switch (cfg->group) {
-      case 8: st = launch(w4a16_gemm_tcgen05<8, true>); break;
-      case 16: st = launch(w4a16_gemm_tcgen05<4, true>); break;
-      case 32: st = launch(w4a16_gemm_tcgen05<2, true>); break;
-      default: st = launch(w4a16_gemm_tcgen05<1, true>); break;
+      case 8:
+        if constexpr (K == 128) return launch(w4a16_gemm_tcgen05<H / 8, F, K>);
+        return AWQ_ERR_UNSUPPORTED;  // the plan keeps g = 8 on 128-channel steps
+      case 16: return launch(w4a16_gemm_tcgen05<H / 16, F, K>);
+      case 32: return launch(w4a16_gemm_tcgen05<H / 32, F, K>);
+      case 64: return launch(w4a16_gemm_tcgen05<(H / 64 > 0 ? H / 64 : 1), F, K>);
+      default: return launch(w4a16_gemm_tcgen05<(H / 128 > 0 ? H / 128 : 1), F, K>);  // 128 and 256
     }
-  } else {
-    switch (cfg->group) {
-      case 8: st = launch(w4a16_gemm_tcgen05<8, false>); break;
-      case 16: st = launch(w4a16_gemm_tcgen05<4, false>); break;
-      case 32: st = launch(w4a16_gemm_tcgen05<2, false>); break;
-      default: st = launch(w4a16_gemm_tcgen05<1, false>); break;
-    }
-  }
+  };
+  using T = std::true_type;
+  using Fa = std::false_type;
+  using K128 = std::integral_constant<int, 128>;
+  using K256 = std::integral_constant<int, 256>;
+  if (f16)
+    st = p.bk == 256 ? dispatch(T{}, K256{}) : dispatch(T{}, K128{});
+  else
+    st = p.bk == 256 ? dispatch(Fa{}, K256{}) : dispatch(Fa{}, K128{});
   if (st != AWQ_OK) return st;
   if (p.splits > 1) {
     const long long n = N * d_out;

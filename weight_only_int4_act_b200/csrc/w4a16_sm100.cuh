@@ -102,27 +102,35 @@ __device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem,
 }
 
 constexpr int W4_BM = 128;
-constexpr int W4_BK = 128;                      // channels per K step: two 64-wide swizzled sub-tiles
-constexpr int W4_SUB = 64;
+constexpr int W4_SUB = 64;                      // channels per 128-byte-swizzled activation box
 constexpr int W4_MAX_BN = 256;
 constexpr int W4_THREADS = 480;
-constexpr int W4_RK = 2;                        // K steps of packed codes per TMA box (128 rows x 128 B)
-constexpr int W4_R_STAGE = W4_BM * 128;         // packed codes, 16 KB
-constexpr int W4_A_COLS = W4_BK / 2;           // TMEM columns of one step of dequantised weights
+constexpr int W4_R_STAGE = W4_BM * 128;         // packed codes: one TMA box of 128 rows x 128 B (256 channels)
+
+// A K step of BK channels (128 or 256): NSUB activation boxes, A_COLS TMEM
+// columns of dequantised weights, RK steps per code box; a dequantising
+// thread takes BK / 2 channels (CHUNKS 16-byte chunks of codes).
+template <int BK>
+struct W4Step {
+  static constexpr int NSUB = BK / W4_SUB;
+  static constexpr int A_COLS = BK / 2;
+  static constexpr int RK = 256 / BK;
+  static constexpr int CHUNKS = BK / 64;
+};
 constexpr int W4_MAX_RS = 32, W4_MAX_XS = 8, W4_MAX_AS = 8;
 constexpr int W4_NBARS = 2 * (W4_MAX_RS + W4_MAX_XS + W4_MAX_AS) + 5;
 constexpr int W4_TMEM_COLS = 512;
 constexpr int W4_SMEM_LIMIT = 232448;
 
 // Shared-memory bytes for ring depths (as, xs, rs) at BN tokens.
-__host__ __device__ constexpr int w4_smem_bytes(int xs, int rs, int bn) {
-  return 1024 + xs * bn * W4_BK * 2 + rs * W4_R_STAGE + W4_NBARS * 8 + 64;
+__host__ __device__ constexpr int w4_smem_bytes(int xs, int rs, int bn, int bk) {
+  return 1024 + xs * bn * bk * 2 + rs * W4_R_STAGE + W4_NBARS * 8 + 64;
 }
 // TMEM columns: NACC accumulators of acc_stride columns, then the A ring.
 __host__ __device__ constexpr int w4_nacc(int bn) { return bn == 256 ? 1 : 2; }
 __host__ __device__ constexpr int w4_acc_stride(int bn) { return bn < 32 ? 32 : bn; }
-__host__ __device__ constexpr int w4_max_as(int bn) {
-  return (W4_TMEM_COLS - w4_nacc(bn) * w4_acc_stride(bn)) / W4_A_COLS;
+__host__ __device__ constexpr int w4_max_as(int bn, int bk) {
+  return (W4_TMEM_COLS - w4_nacc(bn) * w4_acc_stride(bn)) / (bk / 2);
 }
 
 constexpr int ERR_W4_RFULL = 0x301, ERR_W4_REMPTY = 0x302, ERR_W4_XFULL = 0x303, ERR_W4_XEMPTY = 0x304,
@@ -231,9 +239,11 @@ struct Ring {
   }
 };
 
-// GPH = quantisation groups per 64 channels (one dequantising thread's share
-// of a K step; 1 for g >= 64); F16: fp16 activations and output (else bf16).
-template <int GPH, bool F16>
+// GPH = quantisation groups per BK / 2 channels (one dequantising thread's
+// share of a K step; 1 for g >= BK / 2); F16: fp16 activations and output
+// (else bf16); BK: channels per K step (256 for decode-width tiles, so that
+// each handshake carries 16 MMAs; 128 otherwise).
+template <int GPH, bool F16, int BK>
 __global__ void __launch_bounds__(W4_THREADS, 1)
     w4a16_gemm_tcgen05(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                        const W4Args args) {
@@ -241,8 +251,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int bn = args.bn;
   const int AS = args.as, XS = args.xs, RS = args.rs;
+  using St = W4Step<BK>;
   const uint32_t x_sub = (uint32_t)bn * W4_SUB * 2;  // one BN x 64 sub-tile; a multiple of 1024
-  const uint32_t x_stage = 2 * x_sub;
+  const uint32_t x_stage = St::NSUB * x_sub;
   uint8_t* sX = smem;                        // [XS][2][BN rows][128 B], swizzled
   uint8_t* sR = sX + XS * x_stage;           // [RS][128 rows][128 B], swizzled
   uint64_t* bars = reinterpret_cast<uint64_t*>(sR + RS * W4_R_STAGE);
@@ -299,8 +310,8 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
 
   if (warp == 0 || warp == 2) {
     if (lane == 0) {
-      // ---------------- TMA producers: packed codes (warp 0, one box per W4_RK
-      // steps) or activations (warp 2, two 64-wide boxes per step)
+      // ---------------- TMA producers: packed codes (warp 0, one box per RK
+      // steps) or activations (warp 2, NSUB 64-wide boxes per step)
       const bool codes = warp == 0;
       const int depth = codes ? RS : XS;
       Ring ring;
@@ -311,7 +322,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         w4_tile_coords(t, args, mb, nb, split);
         const int kb0 = split * args.kb_per_split;
         const int kb1 = min(args.n_kb, kb0 + args.kb_per_split);
-        for (int kb = kb0; kb < kb1; kb += codes ? W4_RK : 1) {
+        for (int kb = kb0; kb < kb1; kb += codes ? St::RK : 1) {
           const uint32_t full = codes ? rfull(ring.stage) : xfull(ring.stage);
           const uint32_t empty = codes ? rempty(ring.stage) : xempty(ring.stage);
           if (!mbar_wait_sleep(empty, ring.phase ^ 1u, abort_flag, args.err, codes ? ERR_W4_REMPTY : ERR_W4_XEMPTY,
@@ -321,12 +332,13 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           }
           if (codes) {
             mbar_arrive_expect_tx(full, W4_R_STAGE);
-            tma_load_2d(smem_u32(sR + ring.stage * W4_R_STAGE), &tmW, full, kb * (W4_BK / 8), mb * W4_BM);
+            tma_load_2d(smem_u32(sR + ring.stage * W4_R_STAGE), &tmW, full, kb * (BK / 8), mb * W4_BM);
           } else {
             mbar_arrive_expect_tx(full, x_stage);
             uint8_t* dst = sX + ring.stage * x_stage;
-            tma_load_2d(smem_u32(dst), &tmX, full, kb * W4_BK, nb * bn);
-            tma_load_2d(smem_u32(dst + x_sub), &tmX, full, kb * W4_BK + W4_SUB, nb * bn);
+#pragma unroll
+            for (int sb = 0; sb < St::NSUB; ++sb)
+              tma_load_2d(smem_u32(dst + sb * x_sub), &tmX, full, kb * BK + sb * W4_SUB, nb * bn);
           }
           issued |= 1u << ring.stage;
           last_parity = (last_parity & ~(1u << ring.stage)) | (ring.phase << ring.stage);
@@ -338,7 +350,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer: 8 MMAs (K = 16 each) per step
+      // ---------------- MMA issuer: BK / 16 MMAs (K = 16 each) per step
       // kind::f16 with both operands fp16 (format 0) or both bf16 (format 1)
       const uint32_t idesc = F16 ? ((1u << 4) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(W4_BM >> 4) << 24))
                                  : idesc_bf16_f32(W4_BM, bn);
@@ -366,10 +378,10 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + a_col0 + ar.stage * W4_A_COLS;
+          const uint32_t a_tmem = tmem_base + a_col0 + ar.stage * St::A_COLS;
           const uint64_t dx = dx0 + ((uint64_t)(xr.stage * x_stage) >> 4);
 #pragma unroll
-          for (int k = 0; k < W4_BK / 16; ++k) {
+          for (int k = 0; k < BK / 16; ++k) {
             const uint32_t sub = (uint32_t)(k >> 2), kq = (uint32_t)(k & 3);
             mma_f16_tmem_a(d_tmem, a_tmem + k * 8, dx + ((sub * x_sub + kq * 32) >> 4), idesc,
                            (kb != kb0) || (k != 0));
@@ -386,11 +398,11 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     }
   } else if (warp < 11) {
     // ---------------- dequantisation: warp w, lane l takes output channel
-    // r = 32 (w % 4) + l (its TMEM lane) and channels 64h .. 64h+63 of each step
+    // r = 32 (w % 4) + l (its TMEM lane) and channels h BK/2 .. (h+1) BK/2 - 1 of each step
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int h = (warp - 3) >> 2;
-    const uint32_t a_lane = tmem_base + ((uint32_t)(quad * 32) << 16) + a_col0 + (uint32_t)(h * 32);
+    const uint32_t a_lane = tmem_base + ((uint32_t)(quad * 32) << 16) + a_col0 + (uint32_t)(h * (BK / 4));
     const int sw = r & 7;
     Ring rr, ar;
     bool ok = true;
@@ -403,14 +415,14 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       const bool valid = row < args.d_out;
       const __half* srow = args.scales + (long long)(valid ? row : 0) * args.ng;
       const __half* zrow = args.zeros + (long long)(valid ? row : 0) * args.ng;
-      // step and zero point of the GPH groups of this thread's 64 channels. The
+      // step and zero point of the GPH groups of this thread's BK / 2 channels. The
       // raw fp16 values of step kb + 2 are loaded while step kb is processed
       // and converted only when their step comes, so the loads stay in flight.
       using Ty = W4Type<F16>;
       auto load_params = [&](int kb, __half (&dq)[GPH], __half (&zq)[GPH]) {
 #pragma unroll
         for (int q = 0; q < GPH; ++q) {
-          const int ch = kb * W4_BK + h * W4_SUB + q * (W4_SUB / GPH);
+          const int ch = kb * BK + h * (BK / 2) + q * ((BK / 2) / GPH);
           const int gi = min(ch >> args.group_shift, args.ng - 1);
           dq[q] = valid ? srow[gi] : __float2half_rn(0.0f);
           zq[q] = valid ? zrow[gi] : __float2half_rn(0.0f);
@@ -432,8 +444,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           d1[q] = d2[q];
           z1[q] = z2[q];
         }
-        // step kk of the code box: 16-byte chunks 4 kk + 2h and 4 kk + 2h + 1 of row r, swizzled
-        const int kk = (kb - kb0) & (W4_RK - 1);
+        // step kk of the code box: CHUNKS 16-byte chunks of row r from
+        // 2 CHUNKS kk + CHUNKS h, swizzled
+        const int kk = (kb - kb0) & (St::RK - 1);
         bool have = true;
         if (kk == 0) have = mbar_wait_sleep(rfull(rr.stage), rr.phase, abort_flag, args.err, ERR_W4_RFULL, 32);
         if (!__all_sync(0xffffffffu, have)) {
@@ -441,10 +454,17 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           break;
         }
         const uint8_t* rrow = sR + rr.stage * W4_R_STAGE + r * 128;
-        const int c0 = 4 * kk + 2 * h;
-        const uint4 w0 = *reinterpret_cast<const uint4*>(rrow + ((c0 ^ sw) << 4));
-        const uint4 w1 = *reinterpret_cast<const uint4*>(rrow + (((c0 + 1) ^ sw) << 4));
-        if (kk == W4_RK - 1 || kb == kb1 - 1) {
+        const int c0 = 2 * St::CHUNKS * kk + St::CHUNKS * h;
+        uint32_t words[4 * St::CHUNKS];
+#pragma unroll
+        for (int c = 0; c < St::CHUNKS; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(rrow + (((c0 + c) ^ sw) << 4));
+          words[4 * c] = w.x;
+          words[4 * c + 1] = w.y;
+          words[4 * c + 2] = w.z;
+          words[4 * c + 3] = w.w;
+        }
+        if (kk == St::RK - 1 || kb == kb1 - 1) {
           __syncwarp();
           if (lane == 0) mbar_arrive(rempty(rr.stage));
           rr.next(RS);
@@ -455,18 +475,22 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           break;
         }
         tc_fence_after();  // the MMAs that read this A stage have completed
-        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        uint32_t cols[32];
+        constexpr int NW = 4 * St::CHUNKS;  // words of the thread's BK / 2 channels
+        constexpr int WPG = NW / GPH;       // words per group among them
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          constexpr int WPG = 8 / GPH;  // words per group inside the thread's 64 channels
-          const uint4 v = dequant_word<F16>(words[c], zc[c / WPG], dc[c / WPG]);
-          cols[4 * c] = v.x;
-          cols[4 * c + 1] = v.y;
-          cols[4 * c + 2] = v.z;
-          cols[4 * c + 3] = v.w;
+        for (int half32 = 0; half32 < NW / 8; ++half32) {  // 32 TMEM columns per tcgen05.st
+          uint32_t cols[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int wi = 8 * half32 + c;
+            const uint4 v = dequant_word<F16>(words[wi], zc[wi / WPG], dc[wi / WPG]);
+            cols[4 * c] = v.x;
+            cols[4 * c + 1] = v.y;
+            cols[4 * c + 2] = v.z;
+            cols[4 * c + 3] = v.w;
+          }
+          tmem_st_32x32b_x32(a_lane + ar.stage * St::A_COLS + 32 * half32, cols);
         }
-        tmem_st_32x32b_x32(a_lane + ar.stage * W4_A_COLS, cols);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
