@@ -321,6 +321,14 @@ awq_status awq_step_reduce(int64_t d_out, int64_t d_in, int64_t N, const awq_qcf
 awq_status awq_debug_copy_dw(const void* ws, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg,
                              int32_t k, void* dst_bf16, awq_stream_t stream);
 
+/* Failure path of the bounded waits, for tests: one block waits on an
+ * mbarrier that nothing arrives at, through the wait every GEMM of this
+ * library uses; after the wall-clock limit (2 s) the wait gives up, sets the
+ * workspace error word and the kernel returns, so that awq_workspace_error
+ * then reports AWQ_ERR_DEVICE and the context stays usable. ws: DEVICE,
+ * 256-byte aligned, at least 256 bytes. Asynchronous. */
+awq_status awq_selftest_bounded_wait(void* ws, awq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -221,3 +221,19 @@ def test_gpu_rejects_bad_arguments():
         awq.search_scales(W, X, a, awq.make_cfg(4, 128, False, 20), ws=small_ws)
     with pytest.raises(awq.AwqError, match="INVALID_ARG"):
         awq.search_scales(W, X, a, awq.make_cfg(5, 128, False, 20))
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    """A wait that nothing satisfies ends after the wall-clock limit with an
+    error in the workspace (no trap, no hang), and the context keeps working."""
+    import time
+    ws = awq.workspace(256)
+    t0 = time.perf_counter()
+    awq.selftest_bounded_wait(ws)
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    assert 1.0 < waited < 30.0, waited
+    with pytest.raises(awq.AwqError, match="DEVICE"):
+        awq.workspace_error(ws)
+    awq.workspace_error(ws)  # the read cleared the word
+    run_case(SMALL["C1"], check_rows=False)

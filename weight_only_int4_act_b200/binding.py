@@ -28,7 +28,7 @@ EXPORTED = (
     "awq_debug_copy_dw", "awq_act_stats_noalloc", "awq_search_scales_segmented", "awq_search_candidates",
     "awq_quantize_pack_clipped", "awq_group_clip_workspace_size", "awq_search_group_clip",
     "awq_quantize_pack_group_clip", "awq_fold_inv_scales", "awq_w4a16_workspace_size", "awq_w4a16_gemm",
-    "awq_pack_workspace_size", "awq_quantize_pack_ws",
+    "awq_pack_workspace_size", "awq_quantize_pack_ws", "awq_selftest_bounded_wait",
 )
 
 
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
             "awq_pack_workspace_size": (c_size_t, [c_int64, c_int64, cfgp]),
             "awq_quantize_pack_ws": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_float, c_void_p,
                                                c_size_t, c_void_p, c_void_p, c_void_p, c_void_p]),
+            "awq_selftest_bounded_wait": (c_int32, [c_void_p, c_void_p]),
             "awq_workspace_error": (c_int32, [c_void_p, c_void_p]),
             "awq_quantize_pack": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_void_p, c_void_p,
                                             c_void_p, c_void_p]),
@@ -372,6 +373,11 @@ def w4a16_gemm(Xp, qweight, scales, zeros, cfg: QCfg, ws=None, out=None):
     _check(lib().awq_w4a16_gemm(_ptr(Xp), dt, _ptr(qweight), _ptr(scales), _ptr(zeros), N, d_out, d_in,
                                 ctypes.byref(cfg), _ptr(out), _ptr(ws), ws.numel(), _stream()), "awq_w4a16_gemm")
     return out
+
+
+def selftest_bounded_wait(ws):
+    """Launch the bounded-wait failure path (see include/awq.h); the error lands in ws."""
+    _check(lib().awq_selftest_bounded_wait(_ptr(ws), _stream()), "awq_selftest_bounded_wait")
 
 
 def workspace_error(ws):

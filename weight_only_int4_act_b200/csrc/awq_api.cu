@@ -1057,3 +1057,13 @@ extern "C" awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p,
     fold_inv_scales_kernel<1, false><<<grid, 256, 0, cs>>>(s, d_in, inner, p);
   return launch_status();
 }
+
+extern "C" awq_status awq_selftest_bounded_wait(void* ws, awq_stream_t stream) {
+  if (!ws || !aligned(ws, 256)) return AWQ_ERR_INVALID_ARG;
+  awq_status st = check_device(nullptr);
+  if (st != AWQ_OK) return st;
+  cudaStream_t cs = as_stream(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(int), cs) != cudaSuccess) return AWQ_ERR_CUDA;
+  bounded_wait_selftest<<<1, 32, 0, cs>>>(at<int>(ws, 0));
+  return launch_status();
+}

@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "fq.cuh"
+#include "ptx.cuh"
 
 namespace awq {
 
@@ -401,6 +402,25 @@ __global__ void segment_argmin(const double* __restrict__ seg_sums, int n_seg, i
   }
   for (int i = lane; i < d_in; i += 32)
     s_best[(long long)sg * d_in + i] = b >= 0 ? s_all[(long long)b * d_in + i] : __int_as_float(0x7fc00000);
+}
+
+// ---------------------------------------------------------------------------
+// Failure path of the bounded waits: one thread waits on an mbarrier that no
+// one arrives at, through the same mbar_wait the GEMMs use; it gives up after
+// AWQ_WAIT_LIMIT_NS and records ERR_WAIT_SELFTEST in *err.
+// ---------------------------------------------------------------------------
+constexpr int ERR_WAIT_SELFTEST = 0x401;
+
+__global__ void bounded_wait_selftest(int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, err, ERR_WAIT_SELFTEST);
 }
 
 // ---------------------------------------------------------------------------
