@@ -174,13 +174,17 @@ def run_ours(args, rank, world, local_rank):
 
     def step_api(ev):
         # the public calls, as a user makes them
-        ev[0].record()
+        if ev is not None:
+            ev[0].record()
         awq.act_stats(X, ws_stats, out=a)
-        ev[1].record()
+        if ev is not None:
+            ev[1].record()
         awq.search_scales(W, X, a, cfg, ws=ws, outputs=outs)
-        ev[2].record()
+        if ev is not None:
+            ev[2].record()
         awq.quantize_pack(W, outs["s_best"], cfg, outputs=packed)
-        ev[3].record()
+        if ev is not None:
+            ev[3].record()
 
     def step(ev=None):
         # the same path one step entry point at a time (no overlap), for the per-kernel breakdown
@@ -234,12 +238,60 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     t_wall = time.perf_counter() - t_wall0
-    clk = clocks.stop()
     awq.workspace_error(ws)
 
     api = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(3)] for k in range(K)])  # ms
     step_ms = api.sum(axis=1)
     total_ms = float(step_ms.sum())
+    eager_losses, eager_best = outs["losses"].clone(), outs["best"].clone()
+
+    # ---- the same public calls captured once in a CUDA graph and replayed: the
+    # calls are stream-ordered with no host synchronisation, so they capture, and
+    # the replay removes the host's launch time between the step's kernels
+    graph, graph_note = None, "eager public calls"
+    if not args.no_graph:
+        try:
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                step_api(None)
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                step_api(None)
+            torch.cuda.synchronize()
+            graph = g
+        except Exception as e:  # report it; the eager timing stands
+            graph_note = f"eager public calls (graph capture failed: {type(e).__name__})"
+    if graph is not None:
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        awq.workspace_error(ws)
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_wall0 = time.perf_counter()
+        for k in range(K):
+            flush.fill_(k & 0xFF)  # outside the replay's events
+            gev[k][0].record()
+            graph.replay()
+            gev[k][1].record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        t_wall = time.perf_counter() - t_wall0
+        awq.workspace_error(ws)
+        if not (torch.equal(outs["losses"], eager_losses) and torch.equal(outs["best"], eager_best)):
+            raise RuntimeError("graph replay results differ from the eager calls")
+        eager_total_ms = total_ms
+        total_ms = float(sum(e0.elapsed_time(e1) for e0, e1 in gev))
+        graph_note = "CUDA graph replay of the public calls (act_stats, search_scales, quantize_pack)"
+    else:
+        eager_total_ms = total_ms
+    clk = clocks.stop()
 
     # per-kernel breakdown: the same work one entry point at a time
     KB = min(K, 20)
@@ -254,6 +306,7 @@ def run_ours(args, rank, world, local_rank):
         seg = np.array(max_over_ranks(seg.ravel().tolist(), dev)).reshape(seg.shape)
     if world > 1:
         total_ms = max_over_ranks([total_ms], dev)[0]
+        eager_total_ms = max_over_ranks([eager_total_ms], dev)[0]
     ms_per_step = total_ms / K
     mean = seg.mean(axis=0)
     names = ["stats", "scales+fake_quant", "gram", "contraction", "reduce_argmin", "pack"]
@@ -453,6 +506,7 @@ def run_ours(args, rank, world, local_rank):
         "steps": K,
         "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4),
+        "ms_per_step_eager": round(eager_total_ms / K, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -461,6 +515,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": f"{wl.key}: {wl.title}", "d_out": d_out, "d_in": d_in, "N": N, "bits": wl.bits,
                    "group": wl.group, "symmetric": wl.symmetric, "n_alpha": n_a, "form": form,
                    "l2": "flushed: 256 MiB write between timed steps, outside the step events",
+                   "timing": graph_note,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"kernel": "gemm_pair_bf16_tcgen05 (CTA pairs, " + ("direct, sum-of-squares epilogue)" if form == "direct"
                                                                  else "block-triangular Gram, dot epilogue)"),
@@ -617,6 +672,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-group-clip", action="store_true", help="skip the per-group clipping pass")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 inference-side timing")
+    ap.add_argument("--no-graph", action="store_true", help="time the eager public calls only")
     ap.add_argument("--only", default=None, choices=["w4a16"], help="time one component alone (its own JSON line)")
     ap.add_argument("--tokens", type=int, default=16, help="tokens for --only w4a16")
     ap.add_argument("--dtype", default="f16", choices=["f16", "bf16"], help="activations for --only w4a16")
