@@ -47,7 +47,8 @@ typedef enum {
   AWQ_ERR_NONFINITE = 4,   /* a candidate loss was NaN or infinite (device-side) */
   AWQ_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
   AWQ_ERR_DEVICE = 6,      /* a kernel gave up a bounded wait (device-side) */
-  AWQ_ERR_UNSUPPORTED = 7  /* no sm_100 device, or a configuration not built */
+  AWQ_ERR_UNSUPPORTED = 7, /* no sm_100 device, or a configuration not built */
+  AWQ_ERR_BOUNDS = 8       /* debug build: an index check failed (awq_bounds_error) */
 } awq_status;
 
 typedef enum { AWQ_FORM_AUTO = 0, AWQ_FORM_DIRECT = 1, AWQ_FORM_GRAM = 2 } awq_form;
@@ -328,6 +329,34 @@ awq_status awq_debug_copy_dw(const void* ws, int64_t d_out, int64_t d_in, int64_
  * then reports AWQ_ERR_DEVICE and the context stays usable. ws: DEVICE,
  * 256-byte aligned, at least 256 bytes. Asynchronous. */
 awq_status awq_selftest_bounded_wait(void* ws, awq_stream_t stream);
+
+/* Debug build (compiled with -DAWQ_BOUNDS_CHECK). Every global load and store
+ * that a kernel addresses by hand (everything but the TMA tensor-map copies)
+ * first checks the span it touches against the extent the kernel's arguments
+ * give that buffer; a failed check skips the access (a load reads zero) and
+ * records the site in a device word of the library, the first failure kept.
+ * The GEMM launchers also check on the host that the furthest element their
+ * epilogue may store or read lies inside the buffer, and return
+ * AWQ_ERR_BOUNDS without launching if not. In the release build the checks
+ * compile to nothing. */
+
+/* 1 if this library was built with the index checks, else 0. */
+int32_t awq_bounds_checks_enabled(void);
+
+/* Read back (synchronising `stream`) and clear the device word of the index
+ * checks: AWQ_OK if no check failed since the last call, else AWQ_ERR_BOUNDS
+ * with *site (host, may be NULL) set to the failing access's site code (the
+ * low byte of the word; 0x7F: awq_selftest_bounds). Always AWQ_OK in the
+ * release build. */
+awq_status awq_bounds_error(int32_t* site, awq_stream_t stream);
+
+/* Failure path of the index checks, for tests: one thread stores to element n
+ * of an int buffer whose extent it declares as n; the check refuses the store
+ * and records site 0x7F. The buffer is ws, which holds n + 1 ints, so even the
+ * refused store would have stayed inside it. ws: DEVICE, 256-byte aligned, at
+ * least 256 bytes. Asynchronous. Returns AWQ_ERR_UNSUPPORTED (and launches
+ * nothing) in the release build. */
+awq_status awq_selftest_bounds(void* ws, size_t ws_bytes, awq_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,8 +19,18 @@ def declared_symbols():
     return sorted(set(re.findall(r"\b(awq_[a-z0-9_]+)\s*\(", text)))
 
 
-def test_header_declarations_match_exports():
-    lib = awq.lib()
+@pytest.fixture(params=["release", "check"])
+def build_lib(request):
+    """The ctypes library of one build; the binding's choice is restored after."""
+    prev = binding.select_library(request.param)
+    try:
+        yield request.param, awq.lib()
+    finally:
+        binding.select_library(prev)
+
+
+def test_header_declarations_match_exports(build_lib):
+    _, lib = build_lib
     names = declared_symbols()
     assert len(names) >= 14
     for n in names:
@@ -28,8 +38,23 @@ def test_header_declarations_match_exports():
     assert sorted(binding.EXPORTED) == names
 
 
+def test_bounds_entry_points_without_gpu(build_lib):
+    """Which build carries the index checks, and the checks' entry points up
+    to the point where they would need the device."""
+    variant, lib = build_lib
+    assert lib.awq_bounds_checks_enabled() == (1 if variant == "check" else 0)
+    assert lib.awq_selftest_bounds(None, 256, None) == 1  # AWQ_ERR_INVALID_ARG
+    assert lib.awq_selftest_bounds(ctypes.c_void_p(0x10010), 256, None) == 1  # not 256-byte aligned
+    assert lib.awq_selftest_bounds(FAKE, 64, None) == 3  # AWQ_ERR_WORKSPACE
+    if variant == "release":
+        # nothing to read back and no self-test to launch
+        site = ctypes.c_int32(5)
+        assert lib.awq_bounds_error(ctypes.byref(site), None) == 0 and site.value == 0
+        assert lib.awq_selftest_bounds(FAKE, 256, None) == 7  # AWQ_ERR_UNSUPPORTED, nothing launched
+
+
 def test_status_strings():
-    for s in range(8):
+    for s in range(9):
         txt = awq.status_str(s)
         assert txt.startswith(binding.STATUS_NAMES[s])
     assert awq.status_str(99) == "AWQ_ERR_UNKNOWN"

@@ -3,6 +3,11 @@
 Every computation runs in the CUDA library; PyTorch only provides device
 memory and the current stream. If the library is missing the calls raise:
 there is no fallback.
+
+Two builds of the library exist (see _build.py): "release" and "check", the
+debug build with index checks. The environment variable AWQ_B200_LIB
+(release | check) picks the one loaded at first use; select_library()
+switches later calls to the other.
 """
 from __future__ import annotations
 
@@ -10,13 +15,16 @@ import ctypes
 import os
 from ctypes import POINTER, c_char_p, c_float, c_int32, c_int64, c_size_t, c_void_p
 
-from ._build import LIB_PATH
+from ._build import VARIANTS, lib_path
 
 AWQ_OK = 0
 STATUS_NAMES = {
     0: "AWQ_OK", 1: "AWQ_ERR_INVALID_ARG", 2: "AWQ_ERR_SHAPE", 3: "AWQ_ERR_WORKSPACE",
     4: "AWQ_ERR_NONFINITE", 5: "AWQ_ERR_CUDA", 6: "AWQ_ERR_DEVICE", 7: "AWQ_ERR_UNSUPPORTED",
+    8: "AWQ_ERR_BOUNDS",
 }
+AWQ_ERR_BOUNDS = 8
+BOUNDS_SITE_SELFTEST = 0x7F
 FORMS = {"auto": 0, "direct": 1, "gram": 2}
 AWQ_DTYPE_BF16, AWQ_DTYPE_F16 = 0, 1
 
@@ -29,6 +37,7 @@ EXPORTED = (
     "awq_quantize_pack_clipped", "awq_group_clip_workspace_size", "awq_search_group_clip",
     "awq_quantize_pack_group_clip", "awq_fold_inv_scales", "awq_w4a16_workspace_size", "awq_w4a16_gemm",
     "awq_pack_workspace_size", "awq_quantize_pack_ws", "awq_selftest_bounded_wait",
+    "awq_bounds_checks_enabled", "awq_bounds_error", "awq_selftest_bounds",
 )
 
 
@@ -54,16 +63,29 @@ def make_cfg(bits=4, group=128, symmetric=False, n_alpha=20, form="auto", eps_a=
     return cfg
 
 
-_lib = None
+_libs = {}
+_active = os.environ.get("AWQ_B200_LIB", "release")
+
+
+def select_library(variant: str) -> str:
+    """Route later calls to the given build ("release" or "check"); returns
+    the previous choice."""
+    global _active
+    if variant not in VARIANTS:
+        raise ValueError(f"unknown library build {variant!r}; one of {sorted(VARIANTS)}")
+    prev, _active = _active, variant
+    return prev
 
 
 def lib() -> ctypes.CDLL:
-    """The loaded CUDA library (raises if it has not been built)."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"CUDA library {LIB_PATH} is missing; build it with __graft_entry__.build()")
-        L = ctypes.CDLL(LIB_PATH)
+    """The selected build of the CUDA library (raises if it has not been built)."""
+    if _active not in VARIANTS:
+        raise ValueError(f"AWQ_B200_LIB={_active!r}; one of {sorted(VARIANTS)}")
+    if _active not in _libs:
+        path = lib_path(_active)
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library {path} is missing; build it with __graft_entry__.build()")
+        L = ctypes.CDLL(path)
         cfgp = POINTER(QCfg)
         sig = {
             "awq_status_str": (c_char_p, [c_int32]),
@@ -95,6 +117,9 @@ def lib() -> ctypes.CDLL:
             "awq_quantize_pack_ws": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_float, c_void_p,
                                                c_size_t, c_void_p, c_void_p, c_void_p, c_void_p]),
             "awq_selftest_bounded_wait": (c_int32, [c_void_p, c_void_p]),
+            "awq_bounds_checks_enabled": (c_int32, []),
+            "awq_bounds_error": (c_int32, [POINTER(c_int32), c_void_p]),
+            "awq_selftest_bounds": (c_int32, [c_void_p, c_size_t, c_void_p]),
             "awq_workspace_error": (c_int32, [c_void_p, c_void_p]),
             "awq_quantize_pack": (c_int32, [c_void_p, c_void_p, c_int64, c_int64, cfgp, c_void_p, c_void_p,
                                             c_void_p, c_void_p]),
@@ -113,8 +138,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
-        _lib = L
-    return _lib
+        _libs[_active] = L
+    return _libs[_active]
 
 
 def status_str(status: int) -> str:
@@ -378,6 +403,26 @@ def w4a16_gemm(Xp, qweight, scales, zeros, cfg: QCfg, ws=None, out=None):
 def selftest_bounded_wait(ws):
     """Launch the bounded-wait failure path (see include/awq.h); the error lands in ws."""
     _check(lib().awq_selftest_bounded_wait(_ptr(ws), _stream()), "awq_selftest_bounded_wait")
+
+
+def bounds_checks_enabled() -> bool:
+    """True if the selected build carries the index checks."""
+    return bool(lib().awq_bounds_checks_enabled())
+
+
+def bounds_error():
+    """(status, site) of the index checks since the last call; reading clears
+    the device word (synchronises). Always (AWQ_OK, 0) in the release build."""
+    site = c_int32(0)
+    st = int(lib().awq_bounds_error(ctypes.byref(site), _stream()))
+    if st not in (AWQ_OK, AWQ_ERR_BOUNDS):
+        raise AwqError(st, "awq_bounds_error")
+    return st, int(site.value)
+
+
+def selftest_bounds(ws):
+    """Launch the index checks' failure path (see include/awq.h)."""
+    _check(lib().awq_selftest_bounds(_ptr(ws), ws.numel() * ws.element_size(), _stream()), "awq_selftest_bounds")
 
 
 def workspace_error(ws):

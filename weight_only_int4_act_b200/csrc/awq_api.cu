@@ -228,11 +228,40 @@ bool make_map_u32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t word
   return r == CUDA_SUCCESS;
 }
 
+// Elements from each epilogue pointer of GemmArgs to the end of the buffer it
+// points into (for the debug build's host-side index checks).
+struct GemmExtents {
+  long long part = 0, E = 0, C = 0;
+};
+
+// Debug build: does the furthest element the GEMM epilogue may touch lie inside
+// each buffer? Every epilogue access sits behind m < M and col < N; partials
+// take one row of part_ld per column tile (per 32-column chunk in EPI_DOT32),
+// E is read and C written 8 elements at a time (TRI_DIAG_STORE: columns
+// relative to the tile, at most bn of them).
+template <int MODE>
+bool gemm_extents_ok(const GemmArgs& a, int bn, const GemmExtents& x) {
+  if (!kBoundsCheck) return true;
+  const long long M = a.M, n8 = cdiv(a.N, 8) * 8;
+  if (MODE == EPI_SUMSQ || MODE == EPI_DOT || MODE == EPI_DOT32) {
+    const long long rows = MODE == EPI_DOT32 ? (long long)a.n_blocks_n * (bn / 32) : a.n_blocks_n;
+    if (a.part_ld < M || (rows - 1) * a.part_ld + M > x.part) return false;
+  }
+  if (MODE == EPI_DOT || MODE == EPI_DOT32) {
+    if (a.ldE < n8 || (M - 1) * a.ldE + n8 > x.E) return false;
+  }
+  if (MODE == EPI_STORE) {
+    const long long w = a.tri == TRI_DIAG_STORE ? (n8 < bn ? n8 : bn) : n8;
+    if (a.ldC < w || (M - 1) * a.ldC + w > x.C) return false;
+  }
+  return true;
+}
+
 // D = A[M, K] * B[Nr, K]^T with the given epilogue.
 // MN = true: A and B are row-major [K, M] / [K, Nr] matrices read transposed.
 template <int MODE, bool MN = false>
 awq_status run_gemm(const void* A, long long M, long long lda, const void* B, long long Nr, long long ldb, long long K,
-                    GemmArgs args, int tri, int num_sms, cudaStream_t st) {
+                    GemmArgs args, int tri, int num_sms, cudaStream_t st, const GemmExtents& ext) {
   CUtensorMap ta, tb;
   if (MN) {
     if (!make_map(&ta, A, K, M, lda, GEMM_BK)) return AWQ_ERR_CUDA;
@@ -254,6 +283,7 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
                                                   : (long long)args.n_blocks_m * args.n_blocks_n;
   if (tiles > INT32_MAX) return AWQ_ERR_SHAPE;
   args.num_tiles = (int)tiles;
+  if (!gemm_extents_ok<MODE>(args, GEMM_BN, ext)) return AWQ_ERR_BOUNDS;
   if (cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE, MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            GEMM_SMEM_BYTES) != cudaSuccess ||
       cudaFuncSetAttribute(gemm_bf16_tcgen05<MODE, MN>, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -268,7 +298,7 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
 // The contraction on CTA pairs (gemm_pair_sm100.cuh): 256 x 256 tiles.
 template <int MODE>
 awq_status run_gemm_pair(const void* A, long long M, long long lda, const void* B, long long Nr, long long ldb,
-                         long long K, GemmArgs args, int tri, int num_sms, cudaStream_t st) {
+                         long long K, GemmArgs args, int tri, int num_sms, cudaStream_t st, const GemmExtents& ext) {
   CUtensorMap ta, tb;
   if (!make_map(&ta, A, M, K, lda, 128)) return AWQ_ERR_CUDA;
   if (!make_map(&tb, B, Nr, K, ldb, 128)) return AWQ_ERR_CUDA;
@@ -282,6 +312,7 @@ awq_status run_gemm_pair(const void* A, long long M, long long lda, const void* 
   const long long tiles = (long long)args.n_blocks_m * args.n_blocks_n;
   if (tiles > INT32_MAX) return AWQ_ERR_SHAPE;
   args.num_tiles = (int)tiles;
+  if (!gemm_extents_ok<MODE>(args, PAIR_BN, ext)) return AWQ_ERR_BOUNDS;
   if (cudaFuncSetAttribute(gemm_pair_bf16_tcgen05<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            PAIR_SMEM_BYTES) != cudaSuccess)
     return AWQ_ERR_CUDA;
@@ -322,6 +353,7 @@ const char* awq_status_str(awq_status s) {
     case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA: CUDA runtime call or launch failed";
     case AWQ_ERR_DEVICE: return "AWQ_ERR_DEVICE: a kernel gave up a bounded wait";
     case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED: needs an sm_100 (B200) device";
+    case AWQ_ERR_BOUNDS: return "AWQ_ERR_BOUNDS: an index check of the debug build failed";
   }
   return "AWQ_ERR_UNKNOWN";
 }
@@ -456,15 +488,18 @@ awq_status launch_contract(const void* X, int64_t d_in, int64_t N, const SearchL
   ga.err = at<int>(ws, 0);
   ga.tile_counter = at<int>(ws, kTileCounterOffset);
   const __nv_bfloat16* dw = at<__nv_bfloat16>(ws, L.off_dw) + row0 * d_in;
+  GemmExtents ext;
+  ext.part = (long long)L.n_blocks_n * L.M - row0;
+  ext.E = (L.M - row0) * d_in;
   if (L.form == AWQ_FORM_DIRECT) {
-    if (AWQ_GEMM_PAIR) return run_gemm_pair<EPI_SUMSQ>(dw, rows, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, st);
-    return run_gemm<EPI_SUMSQ>(dw, rows, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, st);
+    if (AWQ_GEMM_PAIR) return run_gemm_pair<EPI_SUMSQ>(dw, rows, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, st, ext);
+    return run_gemm<EPI_SUMSQ>(dw, rows, d_in, X, N, d_in, d_in, ga, TRI_NONE, sms, st, ext);
   }
   ga.E = dw;
   ga.ldE = d_in;
   if (AWQ_GEMM_PAIR)
-    return run_gemm_pair<EPI_DOT>(dw, rows, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms, st);
-  return run_gemm<EPI_DOT>(dw, rows, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms, st);
+    return run_gemm_pair<EPI_DOT>(dw, rows, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms, st, ext);
+  return run_gemm<EPI_DOT>(dw, rows, d_in, at<void>(ws, L.off_g), d_in, d_in, d_in, ga, TRI_K, sms, st, ext);
 }
 
 awq_status awq_step_fake_quant(const void* W, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
@@ -492,8 +527,11 @@ awq_status awq_step_gram(const void* X, int64_t d_out, int64_t d_in, int64_t N, 
   ga.ldC = d_in;
   ga.err = at<int>(ws, 0);
   ga.tile_counter = at<int>(ws, kTileCounterOffset);
+  GemmExtents ext;
+  ext.C = (long long)d_in * d_in;
   // G = X^T X with both operands read transposed from X [N, d_in] (MN-major)
-  return run_gemm<EPI_STORE, true>(X, d_in, d_in, X, d_in, d_in, N, ga, TRI_LOWER_STORE, sms, as_stream(stream));
+  return run_gemm<EPI_STORE, true>(X, d_in, d_in, X, d_in, d_in, N, ga, TRI_LOWER_STORE, sms, as_stream(stream),
+                                   ext);
 }
 
 awq_status awq_step_contract(const void* X, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,
@@ -653,7 +691,10 @@ awq_status awq_search_group_clip(const void* W, const void* X, const float* s, c
   gs.group = cfg->group;
   // entries outside the stored diagonal (columns past d_in) must read as 0
   if (cudaMemsetAsync(gs.C, 0, (size_t)d_in * GEMM_BN * 2, cs) != cudaSuccess) return AWQ_ERR_CUDA;
-  if ((st = run_gemm<EPI_STORE, true>(X, d_in, d_in, X, d_in, d_in, N, gs, TRI_DIAG_STORE, sms, cs)) != AWQ_OK)
+  GemmExtents gext;
+  gext.C = (long long)d_in * GEMM_BN;
+  if ((st = run_gemm<EPI_STORE, true>(X, d_in, d_in, X, d_in, d_in, N, gs, TRI_DIAG_STORE, sms, cs, gext)) !=
+      AWQ_OK)
     return st;
   // per (row, 32-column chunk) errors of every candidate: dW[:, J] G_J dW[:, J]^T restricted to the groups
   GemmArgs ga{};
@@ -663,8 +704,11 @@ awq_status awq_search_group_clip(const void* W, const void* X, const float* s, c
   ga.tile_counter = at<int>(ws, kTileCounterOffset);
   ga.E = at<__nv_bfloat16>(ws, L.off_dw);
   ga.ldE = d_in;
+  GemmExtents cext;
+  cext.part = (long long)L.n_chunks * L.M;
+  cext.E = L.M * d_in;
   if ((st = run_gemm<EPI_DOT32>(at<void>(ws, L.off_dw), L.M, d_in, at<void>(ws, L.off_g), d_in, GEMM_BN, d_in, ga,
-                                TRI_DIAG, sms, cs)) != AWQ_OK)
+                                TRI_DIAG, sms, cs, cext)) != AWQ_OK)
     return st;
   const int ng = (int)(d_in / cfg->group);
   const long long units = (long long)ng * d_out;
@@ -1065,5 +1109,35 @@ extern "C" awq_status awq_selftest_bounded_wait(void* ws, awq_stream_t stream) {
   cudaStream_t cs = as_stream(stream);
   if (cudaMemsetAsync(ws, 0, sizeof(int), cs) != cudaSuccess) return AWQ_ERR_CUDA;
   bounded_wait_selftest<<<1, 32, 0, cs>>>(at<int>(ws, 0));
+  return launch_status();
+}
+
+extern "C" int32_t awq_bounds_checks_enabled(void) { return kBoundsCheck ? 1 : 0; }
+
+extern "C" awq_status awq_bounds_error(int32_t* site, awq_stream_t stream) {
+  if (site) *site = 0;
+  if (!kBoundsCheck) return AWQ_OK;
+  cudaStream_t cs = as_stream(stream);
+  int word = 0;
+  if (cudaMemcpyFromSymbolAsync(&word, g_bounds_err, sizeof(int), 0, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (word == 0) return AWQ_OK;
+  const int zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_bounds_err, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+    return AWQ_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return AWQ_ERR_CUDA;
+  if (site) *site = word & 0xFF;
+  return AWQ_ERR_BOUNDS;
+}
+
+extern "C" awq_status awq_selftest_bounds(void* ws, size_t ws_bytes, awq_stream_t stream) {
+  if (!ws || !aligned(ws, 256)) return AWQ_ERR_INVALID_ARG;
+  if (ws_bytes < 256) return AWQ_ERR_WORKSPACE;
+  if (!kBoundsCheck) return AWQ_ERR_UNSUPPORTED;
+  awq_status st = check_device(nullptr);
+  if (st != AWQ_OK) return st;
+  // ws holds 64 ints; the kernel declares an extent of 63 and stores to element 63
+  bounds_selftest<<<1, 32, 0, as_stream(stream)>>>(at<int>(ws, 0), 63);
   return launch_status();
 }

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "check.cuh"
 #include "fq.cuh"
 #include "ptx.cuh"
 
@@ -55,7 +56,9 @@ __global__ void __launch_bounds__(STATS_THREADS) act_absmean_partial(const __nv_
 #pragma unroll
       for (int k = 0; k < STATS_UNROLL; ++k) {
         const long long rr = r + 8 * k;
-        u[k] = rr < r1 ? __ldcs(reinterpret_cast<const uint4*>(base + rr * d_in)) : make_uint4(0, 0, 0, 0);
+        u[k] = (rr < r1 && AWQ_SPAN_OK(rr * d_in + col, 8, N * d_in, BS_STATS_X))
+                   ? __ldcs(reinterpret_cast<const uint4*>(base + rr * d_in))
+                   : make_uint4(0, 0, 0, 0);
       }
       float s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
@@ -77,7 +80,8 @@ __global__ void __launch_bounds__(STATS_THREADS) act_absmean_partial(const __nv_
     double t = 0.0;
 #pragma unroll
     for (int w = 0; w < STATS_THREADS / 32; ++w) t += red[w][threadIdx.x];
-    part[(long long)blockIdx.y * d_in + c] = t;
+    if (AWQ_IDX_OK((long long)blockIdx.y * d_in + c, (long long)gridDim.y * d_in, BS_STATS_PART))
+      part[(long long)blockIdx.y * d_in + c] = t;
   }
 }
 
@@ -209,8 +213,10 @@ __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* 
 #pragma unroll
       for (int q = 0; q < CPT / 8; ++q) {
         float f[8];
-        unpack_bf16x8(real ? __ldg(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0) + q)
-                           : make_uint4(0, 0, 0, 0),
+        const bool ld = real && AWQ_SPAN_OK((long long)(row0 + r) * d_in + c0 + 8 * q, 8, (long long)d_out * d_in,
+                                            BS_FQ_W);
+        unpack_bf16x8(ld ? __ldg(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0) + q)
+                         : make_uint4(0, 0, 0, 0),
                       f);
 #pragma unroll
         for (int j = 0; j < 8; ++j) w[r][8 * q + j] = f[j];
@@ -219,8 +225,13 @@ __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* 
     __nv_bfloat16* out_base = dW + (long long)row0 * d_in + c0;
     for (int k = 0; k < n_alpha; ++k) {
       float s[CPT], is[CPT];
-      load_f32<CPT>(s_all + (long long)k * d_in + c0, s);
-      load_f32<CPT>(inv_all + (long long)k * d_in + c0, is);
+      if (AWQ_SPAN_OK((long long)k * d_in + c0, CPT, (long long)n_alpha * d_in, BS_FQ_S)) {
+        load_f32<CPT>(s_all + (long long)k * d_in + c0, s);
+        load_f32<CPT>(inv_all + (long long)k * d_in + c0, is);
+      } else {
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) s[j] = is[j] = 0.f;
+      }
 #pragma unroll
       for (int r = 0; r < ROWS; ++r) {
         float v[CPT];
@@ -241,7 +252,8 @@ __global__ void __launch_bounds__(256, 2) fake_quant_delta(const __nv_bfloat16* 
                                                      fq_dequant(fr, j + 1) * is[j + 1] - w[r][j + 1]);
             out[h] = *reinterpret_cast<uint32_t*>(&p);
           }
-          if (active)
+          if (active && AWQ_SPAN_OK((long long)(row0 + r) * d_in + c0 + 8 * q + k * slice, 8, n_alpha * slice,
+                                    BS_FQ_DW))
             __stcs(reinterpret_cast<uint4*>(out_base + k * slice + (long long)r * d_in) + q,
                    make_uint4(out[0], out[1], out[2], out[3]));
         }
@@ -268,8 +280,11 @@ __global__ void __launch_bounds__(REDUCE_THREADS) row_loss_reduce(const float* _
   double s = 0.0;
   if (r < d_out) {
     const long long m = (long long)k * d_out_pad + r;
-    for (int nb = 0; nb < n_blocks_n; ++nb) s += (double)part[(long long)nb * M + m];
-    if (row_losses) row_losses[(long long)k * d_out + r] = (float)s;
+    for (int nb = 0; nb < n_blocks_n; ++nb)
+      if (AWQ_IDX_OK((long long)nb * M + m, (long long)n_blocks_n * M, BS_LOSS_PART))
+        s += (double)part[(long long)nb * M + m];
+    if (row_losses && AWQ_IDX_OK((long long)k * d_out + r, (long long)gridDim.y * d_out, BS_LOSS_ROW))
+      row_losses[(long long)k * d_out + r] = (float)s;
   }
   red[threadIdx.x] = s;
   __syncthreads();
@@ -330,7 +345,9 @@ __global__ void loss_argmin(const double* __restrict__ block_sums, int n_chunks,
   __syncthreads();
   const int b = best_sh;
   for (int i = threadIdx.x; i < d_in; i += blockDim.x)
-    s_best[i] = b >= 0 ? s_all[(long long)b * d_in + i] : __int_as_float(0x7fc00000);
+    s_best[i] = (b >= 0 && AWQ_IDX_OK((long long)b * d_in + i, (long long)n_alpha * d_in, BS_ARGMIN_S))
+                    ? s_all[(long long)b * d_in + i]
+                    : __int_as_float(0x7fc00000);
 }
 
 // ---------------------------------------------------------------------------
@@ -354,8 +371,11 @@ __global__ void __launch_bounds__(REDUCE_THREADS) segment_loss_reduce(const floa
   for (int r = seg.start[sg] + threadIdx.x; r < seg.start[sg + 1]; r += REDUCE_THREADS) {
     const long long m = (long long)k * d_out_pad + r;
     double s = 0.0;
-    for (int nb = 0; nb < n_blocks_n; ++nb) s += (double)part[(long long)nb * M + m];
-    if (row_losses) row_losses[(long long)k * d_out + r] = (float)s;
+    for (int nb = 0; nb < n_blocks_n; ++nb)
+      if (AWQ_IDX_OK((long long)nb * M + m, (long long)n_blocks_n * M, BS_LOSS_PART))
+        s += (double)part[(long long)nb * M + m];
+    if (row_losses && AWQ_IDX_OK((long long)k * d_out + r, (long long)gridDim.y * d_out, BS_LOSS_ROW))
+      row_losses[(long long)k * d_out + r] = (float)s;
     acc += s;
   }
   red[threadIdx.x] = acc;
@@ -401,7 +421,10 @@ __global__ void segment_argmin(const double* __restrict__ seg_sums, int n_seg, i
     if (!finite && err) atomicCAS(err, 0, ERR_NONFINITE);
   }
   for (int i = lane; i < d_in; i += 32)
-    s_best[(long long)sg * d_in + i] = b >= 0 ? s_all[(long long)b * d_in + i] : __int_as_float(0x7fc00000);
+    s_best[(long long)sg * d_in + i] =
+        (b >= 0 && AWQ_IDX_OK((long long)b * d_in + i, (long long)n_alpha * d_in, BS_ARGMIN_S))
+            ? s_all[(long long)b * d_in + i]
+            : __int_as_float(0x7fc00000);
 }
 
 // ---------------------------------------------------------------------------
@@ -443,7 +466,7 @@ __device__ __forceinline__ float ord_val(uint32_t k) {
 __global__ void col_minmax(const __nv_bfloat16* __restrict__ W, int d_out, int d_in, int rows_per_block,
                            uint32_t* __restrict__ kmax, uint32_t* __restrict__ kmin) {
   const int c8 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
-  if (c8 >= d_in) return;
+  if (c8 >= d_in || !AWQ_SPAN_OK(c8, 8, d_in, BS_MINMAX_KEY)) return;
   const int r0 = blockIdx.y * rows_per_block;
   const int r1 = min(d_out, r0 + rows_per_block);
   float mx[8], mn[8];
@@ -454,6 +477,7 @@ __global__ void col_minmax(const __nv_bfloat16* __restrict__ W, int d_out, int d
   }
   for (int r = r0; r < r1; ++r) {
     float f[8];
+    if (!AWQ_SPAN_OK((long long)r * d_in + c8, 8, (long long)d_out * d_in, BS_MINMAX_W)) continue;
     unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(W + (long long)r * d_in + c8)), f);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -537,16 +561,21 @@ __global__ void group_clip_argmin(const float* __restrict__ part, long long part
     for (int c = 0; c < n_clip; ++c) {
       double e = 0.0;
       for (int u = 0; u < chunks_per_group; ++u)
-        e += (double)part[(long long)(j * chunks_per_group + u) * part_ld + (long long)c * d_out_pad + r];
+        if (AWQ_IDX_OK((long long)c * d_out_pad + r, part_ld, BS_CLIP_PART) &&
+            AWQ_IDX_OK(j * chunks_per_group + u, (long long)n_groups * chunks_per_group, BS_CLIP_PART))
+          e += (double)part[(long long)(j * chunks_per_group + u) * part_ld + (long long)c * d_out_pad + r];
       if (!isfinite(e)) finite = false;
-      if (group_err) group_err[((long long)c * d_out + r) * n_groups + j] = (float)e;
+      if (group_err && AWQ_IDX_OK(((long long)c * d_out + r) * n_groups + j, (long long)n_clip * d_out * n_groups,
+                                  BS_CLIP_OUT))
+        group_err[((long long)c * d_out + r) * n_groups + j] = (float)e;
       if (e < bv) {
         bv = e;
         bi = c;
       }
     }
     if (!finite) atomicCAS(err, 0, ERR_NONFINITE);
-    best[(long long)r * n_groups + j] = (uint8_t)bi;
+    if (AWQ_IDX_OK((long long)r * n_groups + j, (long long)d_out * n_groups, BS_CLIP_OUT))
+      best[(long long)r * n_groups + j] = (uint8_t)bi;
   }
 }
 
@@ -590,11 +619,17 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
     for (int r = 0; r < PACK_ROWS; ++r)
 #pragma unroll
       for (int q = 0; q < CPT / 8; ++q)
-        wraw[r][q] = (active && row0 + r < d_out)
+        wraw[r][q] = (active && row0 + r < d_out &&
+                      AWQ_SPAN_OK((long long)(row0 + r) * d_in + c0 + 8 * q, 8, (long long)d_out * d_in, BS_PACK_W))
                          ? __ldcs(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0) + q)
                          : make_uint4(0, 0, 0, 0);
     float sc[CPT];
-    load_f32<CPT>(s + c0, sc);
+    if (AWQ_SPAN_OK(c0, CPT, d_in, BS_PACK_S)) {
+      load_f32<CPT>(s + c0, sc);
+    } else {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) sc[j] = 0.f;
+    }
 #pragma unroll
     for (int r = 0; r < PACK_ROWS; ++r) {
       float v[CPT];
@@ -607,7 +642,8 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
       }
       // per-group clip ratio (index into clips) when given, else the scalar one
       float c = clip;
-      if (group_clip && active && row0 + r < d_out) {
+      if (group_clip && active && row0 + r < d_out &&
+          AWQ_IDX_OK((long long)(row0 + r) * groups + chunk / GL, (long long)d_out * groups, BS_PACK_CLIP)) {
         const int idx = group_clip[(long long)(row0 + r) * groups + chunk / GL];
         c = idx < MAX_ALPHA ? clips.c[idx] : 1.0f;
       }
@@ -624,12 +660,15 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
           uint32_t word = 0;
 #pragma unroll
           for (int j = 0; j < 8; ++j) word |= (fq_code(fr, 8 * q + j) & 0xFu) << (4 * j);
-          __stcs(wp + q, word);
+          if (AWQ_IDX_OK((long long)row * words + c0 / 8 + q, (long long)d_out * words, BS_PACK_Q))
+            __stcs(wp + q, word);
         }
         if (PT ? (row == 0 && chunk == 0) : (chunk & (GL - 1)) == 0) {
           const long long gidx = PT ? 0 : (long long)row * groups + chunk / GL;
-          scales[gidx] = __float2half_rn(fr.delta);
-          zeros[gidx] = __float2half_rn(fr.zero);
+          if (AWQ_IDX_OK(gidx, PT ? 1 : (long long)d_out * groups, BS_PACK_SZ)) {
+            scales[gidx] = __float2half_rn(fr.delta);
+            zeros[gidx] = __float2half_rn(fr.zero);
+          }
         }
       }
     }

@@ -51,6 +51,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "check.cuh"
 #include "ptx.cuh"
 
 namespace awq {
@@ -424,8 +425,10 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         for (int q = 0; q < GPH; ++q) {
           const int ch = kb * BK + h * (BK / 2) + q * ((BK / 2) / GPH);
           const int gi = min(ch >> args.group_shift, args.ng - 1);
-          dq[q] = valid ? srow[gi] : __float2half_rn(0.0f);
-          zq[q] = valid ? zrow[gi] : __float2half_rn(0.0f);
+          const bool ld = valid && AWQ_IDX_OK((long long)row * args.ng + gi, (long long)args.d_out * args.ng,
+                                              BS_W4_PARAMS);
+          dq[q] = ld ? srow[gi] : __float2half_rn(0.0f);
+          zq[q] = ld ? zrow[gi] : __float2half_rn(0.0f);
         }
       };
       __half d0[GPH], z0[GPH], d1[GPH], z1[GPH], d2[GPH], z2[GPH];  // steps kb, kb + 1, kb + 2
@@ -527,12 +530,15 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
             typename W4Type<F16>::T* y = static_cast<typename W4Type<F16>::T*>(args.Y) + e0;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < jn) y[(long long)j * args.d_out] = W4Type<F16>::from_float(__uint_as_float(v[j]));
+              if (j < jn && AWQ_IDX_OK(e0 + (long long)j * args.d_out, (long long)args.N * args.d_out, BS_W4_Y))
+                y[(long long)j * args.d_out] = W4Type<F16>::from_float(__uint_as_float(v[j]));
           } else {
             float* P = args.P + (long long)split * args.p_stride + e0;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < jn) P[(long long)j * args.d_out] = __uint_as_float(v[j]);
+              if (j < jn && AWQ_IDX_OK(e0 + (long long)j * args.d_out, (long long)args.N * args.d_out, BS_W4_P) &&
+                  AWQ_IDX_OK(split, args.splits, BS_W4_P))
+                P[(long long)j * args.d_out] = __uint_as_float(v[j]);
           }
         }
       }
@@ -560,6 +566,7 @@ __global__ void w4a16_split_reduce(const float* __restrict__ P, int splits, long
   T* Y = static_cast<T*>(Yv);
   const long long n4 = n >> 2;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    if (!AWQ_SPAN_OK(4 * i, 4, n, BS_SPLIT_Y) || !AWQ_SPAN_OK(4 * i, 4, stride, BS_SPLIT_P)) continue;
     float4 acc = reinterpret_cast<const float4*>(P)[i];
     for (int s = 1; s < splits; ++s) {
       const float4 p = reinterpret_cast<const float4*>(P + (long long)s * stride)[i];
@@ -572,7 +579,7 @@ __global__ void w4a16_split_reduce(const float* __restrict__ P, int splits, long
   }
   // tail (n not a multiple of 4)
   const long long i = (n4 << 2) + (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (blockIdx.x == 0 && i < n) {
+  if (blockIdx.x == 0 && i < n && AWQ_IDX_OK(i, stride, BS_SPLIT_P)) {
     float acc = P[i];
     for (int s = 1; s < splits; ++s) acc += P[(long long)s * stride + i];
     Y[i] = W4Type<F16>::from_float(acc);
@@ -591,6 +598,7 @@ __global__ void fold_inv_scales_kernel(const float* __restrict__ s, long long d_
   for (long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x; u < units;
        u += (long long)gridDim.x * blockDim.x) {
     const long long e = u * VEC;
+    if (!AWQ_IDX_OK(e / inner, d_in, BS_FOLD_S) || !AWQ_SPAN_OK(e, VEC, d_in * inner, BS_FOLD_P)) continue;
     const float si = s[e / inner];
     if constexpr (VEC == 8) {
       uint4 w = reinterpret_cast<const uint4*>(p)[u];
