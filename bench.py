@@ -632,9 +632,11 @@ def cpu_threads():
 
 def cpu_baseline_entry(wl, rows):
     t_layer, r, spent = oracle_sample(wl, rows)
+    part = (f"the whole layer ({r} rows) x {wl.n_alpha} alphas" if r == wl.d_out else
+            f"{r} of {wl.d_out} rows x {wl.n_alpha} alphas, extrapolated by rows")
     return {"value": round(wl.n_alpha / t_layer, 4), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{wl.key}: full statistics + search and pack of {r} of {wl.d_out} rows x {wl.n_alpha} alphas "
-                      f"(float64 numpy, BLAS matmul), extrapolated by rows; {spent:.1f} s of CPU work"}
+            "sample": f"{wl.key}: statistics, search and pack of {part} (float64 numpy, BLAS matmul); "
+                      f"{spent:.1f} s of CPU work"}
 
 
 def run_reference(args, wl):
@@ -668,7 +670,7 @@ def main():
     ap.add_argument("--form", default="auto", choices=["auto", "direct", "gram"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=512)
-    ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--cpu-rows", type=int, default=4096)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-group-clip", action="store_true", help="skip the per-group clipping pass")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 inference-side timing")
