@@ -630,6 +630,15 @@ def cpu_threads():
     return os.cpu_count() or 1
 
 
+def cpu_sample_rows(wl, budget=4096 * 4096 * 4096):
+    """Rows of W for the CPU baseline: the oracle's cost per row grows with
+    d_in * N, so the sample holds budget / (d_in * N) rows (the whole 4096-row
+    layer at 4096 x 4096 x 4096, about 10 s on 16 host threads), in multiples
+    of 256, at least 256 and at most d_out."""
+    rows = budget // (wl.d_in * wl.N) // 256 * 256
+    return int(min(wl.d_out, max(256, rows)))
+
+
 def cpu_baseline_entry(wl, rows):
     t_layer, r, spent = oracle_sample(wl, rows)
     part = (f"the whole layer ({r} rows) x {wl.n_alpha} alphas" if r == wl.d_out else
@@ -670,7 +679,8 @@ def main():
     ap.add_argument("--form", default="auto", choices=["auto", "direct", "gram"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=512)
-    ap.add_argument("--cpu-rows", type=int, default=4096)
+    ap.add_argument("--cpu-rows", type=int, default=None,
+                    help="rows of W in the CPU baseline's sample (default: cpu_sample_rows)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-group-clip", action="store_true", help="skip the per-group clipping pass")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 inference-side timing")
@@ -708,7 +718,8 @@ def main():
         line = run_ours(args, rank, world, local_rank)
         if rank == 0:
             if not args.no_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline_entry(wl, args.cpu_rows)
+                rows = args.cpu_rows if args.cpu_rows is not None else cpu_sample_rows(wl)
+                line["cpu_baseline"] = cpu_baseline_entry(wl, rows)
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

@@ -81,3 +81,13 @@ def test_reference_arm_json_line():
     assert line["impl"] == "reference" and line["unit"] == bench.UNIT and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["higher_is_better"] is True
+
+
+def test_cpu_sample_rows_bounded_and_whole_layer_at_c2():
+    from awq_inputs import configs
+    for key, wl in configs.WORKLOADS.items():
+        r = bench.cpu_sample_rows(wl)
+        assert 256 <= r <= max(256, wl.d_out) and (r % 256 == 0 or r == wl.d_out), key
+        # per-row oracle cost ~ d_in * N: the sample stays within the 4096^3 budget unless at its floor
+        assert r == 256 or r * wl.d_in * wl.N <= 4096 ** 3, key
+    assert bench.cpu_sample_rows(configs.WORKLOADS["C2"]) == 4096
