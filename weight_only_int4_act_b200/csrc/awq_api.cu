@@ -404,8 +404,9 @@ awq_status awq_step_scales(const float* a, int64_t d_out, int64_t d_in, int64_t 
   for (int k = 0; k < cfg->n_alpha; ++k) grid.v[k] = alpha_value(cfg, k);
   cudaStream_t s = as_stream(stream);
   if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return AWQ_ERR_CUDA;
-  candidate_scales<<<cfg->n_alpha, 512, 0, s>>>(a, (int)d_in, grid, eps_value(cfg), at<float>(ws, L.off_s),
-                                                at<float>(ws, L.off_inv));
+  const dim3 sgrid((unsigned)cdiv(d_in, SCALES_THREADS), (unsigned)cfg->n_alpha);
+  candidate_scales<<<sgrid, SCALES_THREADS, 0, s>>>(a, (int)d_in, grid, eps_value(cfg), at<float>(ws, L.off_s),
+                                                   at<float>(ws, L.off_inv));
   return launch_status();
 }
 

@@ -95,48 +95,51 @@ __global__ void act_absmean_final(const double* __restrict__ part, int n_chunks,
 }
 
 // ---------------------------------------------------------------------------
-// a2: s_k,i = max(a_i, eps)^alpha_k / sqrt(max_j t_j * min_j t_j), and 1/s.
-// ([P5] §4.1 s_i = a_i^alpha.) One block per alpha; the power and the
-// normalisation are taken in fp64 and rounded once to fp32.
+// a2: s_k,i = t_k,i / sqrt(max_j t_k,j * min_j t_k,j) with t_k,i =
+// max(a_i, eps)^alpha_k, and 1/s. ([P5] §4.1 s_i = a_i^alpha.) For alpha >= 0
+// the power does not decrease as its base grows, so the largest and smallest
+// t_k,j are the powers of the largest and smallest floored a_j: each block
+// first takes those two extremes of a (d_in floats, read from L2), then each
+// thread computes one element on its own. Grid: (column blocks of
+// SCALES_THREADS, alpha). The power and the normalisation are taken in fp64
+// and rounded once to fp32.
 // ---------------------------------------------------------------------------
-__global__ void candidate_scales(const float* __restrict__ a, int d_in, AlphaGrid grid, float eps_a,
-                                 float* __restrict__ s_all, float* __restrict__ inv_all) {
-  __shared__ double smax[32], smin[32];
-  const double alpha = grid.v[blockIdx.x];
+constexpr int SCALES_THREADS = 256;
+
+__global__ void __launch_bounds__(SCALES_THREADS) candidate_scales(const float* __restrict__ a, int d_in,
+                                                                   AlphaGrid grid, float eps_a,
+                                                                   float* __restrict__ s_all,
+                                                                   float* __restrict__ inv_all) {
+  __shared__ double smax[SCALES_THREADS / 32], smin[SCALES_THREADS / 32];
   double mx = 0.0, mn = 1e300;
-  for (int i = threadIdx.x; i < d_in; i += blockDim.x) {
-    const double t = pow(fmax((double)a[i], (double)eps_a), alpha);
-    mx = fmax(mx, t);
-    mn = fmin(mn, t);
+  for (int i = threadIdx.x; i < d_in; i += SCALES_THREADS) {
+    const double v = fmax((double)a[i], (double)eps_a);
+    mx = fmax(mx, v);
+    mn = fmin(mn, v);
   }
   for (int off = 16; off > 0; off >>= 1) {
     mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, off));
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) {
     smax[warp] = mx;
     smin[warp] = mn;
   }
   __syncthreads();
-  if (warp == 0) {
-    mx = lane < nw ? smax[lane] : 0.0;
-    mn = lane < nw ? smin[lane] : 1e300;
-    for (int off = 16; off > 0; off >>= 1) {
-      mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-    }
-    if (lane == 0) {
-      smax[0] = mx;
-      smin[0] = mn;
-    }
+#pragma unroll
+  for (int w = 0; w < SCALES_THREADS / 32; ++w) {
+    mx = fmax(mx, smax[w]);
+    mn = fmin(mn, smin[w]);
   }
-  __syncthreads();
-  const double norm = sqrt(smax[0] * smin[0]);
-  for (int i = threadIdx.x; i < d_in; i += blockDim.x) {
+  const int k = blockIdx.y;
+  const double alpha = grid.v[k];
+  const double norm = sqrt(pow(mx, alpha) * pow(mn, alpha));
+  const int i = blockIdx.x * SCALES_THREADS + threadIdx.x;
+  if (i < d_in) {
     const double s = pow(fmax((double)a[i], (double)eps_a), alpha) / norm;
-    s_all[(long long)blockIdx.x * d_in + i] = (float)s;
-    inv_all[(long long)blockIdx.x * d_in + i] = (float)(1.0 / s);
+    s_all[(long long)k * d_in + i] = (float)s;
+    inv_all[(long long)k * d_in + i] = (float)(1.0 / s);
   }
 }
 
