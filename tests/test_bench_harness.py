@@ -72,12 +72,14 @@ def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("CZ", "gram") is None
 
 
-def test_reference_arm_json_line():
+def test_reference_arm_json_line(tmp_path):
+    dest = tmp_path / "ref.json"
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "C1",
-                          "--steps", "1", "--warmup", "3", "--ref-rows", "64"],
+                          "--steps", "1", "--warmup", "3", "--ref-rows", "64", "--json-out", str(dest)],
                          capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert out.returncode == 0, out.stderr
     line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert json.loads(dest.read_text()) == line
     assert line["impl"] == "reference" and line["unit"] == bench.UNIT and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["higher_is_better"] is True
@@ -91,3 +93,20 @@ def test_cpu_sample_rows_bounded_and_whole_layer_at_c2():
         # per-row oracle cost ~ d_in * N: the sample stays within the 4096^3 budget unless at its floor
         assert r == 256 or r * wl.d_in * wl.N <= 4096 ** 3, key
     assert bench.cpu_sample_rows(configs.WORKLOADS["C2"]) == 4096
+
+
+def test_golden_parity_reads_stored_oracle_runs():
+    import json as _json
+    from awq_inputs import configs, custom
+    for key in ("C1", "C2", "C3", "C4", "C5"):
+        wl = configs.WORKLOADS[key]
+        with open(os.path.join(ROOT, "tests", "golden", f"search_{key}.json")) as f:
+            g = _json.load(f)
+        a_const = [g["a_checksum"] / wl.d_in] * wl.d_in
+        near = bench.golden_parity(wl, [v * (1 + 1e-4) for v in g["losses"]], g["best"], a_const)
+        assert near["ok"] and abs(near["loss_max_rel"] - 1e-4) < 1e-9 and near["a_sum_rel"] < 1e-9, key
+        far = bench.golden_parity(wl, [v * 1.05 for v in g["losses"]], g["best"], a_const)
+        assert not far["ok"], key
+        wrong = [k for k in range(wl.n_alpha) if k not in g["acceptable"]][0]
+        assert not bench.golden_parity(wl, g["losses"], wrong, a_const)["ok"], key
+    assert bench.golden_parity(custom(64, 256, 32), [1.0] * 20, 0, [1.0] * 256) is None
