@@ -729,6 +729,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=16, help="tokens for --only w4a16")
     ap.add_argument("--dtype", default="f16", choices=["f16", "bf16"], help="activations for --only w4a16")
     ap.add_argument("--json-out", default=None, help="also write the JSON line to this file")
+    ap.add_argument("--seed", type=int, default=None,
+                    help="seed of the synthetic inputs (default: the workload's own; parity then has no stored run)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -736,6 +738,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.seed is not None:  # every reader of WORKLOADS[args.config] below sees the new seed
+        import dataclasses
+        WORKLOADS[args.config] = dataclasses.replace(WORKLOADS[args.config], seed=args.seed)
     wl = WORKLOADS[args.config]
 
     def emit(line):

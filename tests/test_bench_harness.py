@@ -110,3 +110,24 @@ def test_golden_parity_reads_stored_oracle_runs():
         wrong = [k for k in range(wl.n_alpha) if k not in g["acceptable"]][0]
         assert not bench.golden_parity(wl, g["losses"], wrong, a_const)["ok"], key
     assert bench.golden_parity(custom(64, 256, 32), [1.0] * 20, 0, [1.0] * 256) is None
+
+
+def test_seed_flag_changes_the_inputs(tmp_path):
+    """--seed reseeds the workload (here through the oracle arm, which needs no GPU)."""
+    lines = []
+    for seed in ("", "123"):
+        cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "C1",
+               "--steps", "1", "--warmup", "3", "--ref-rows", "32"] + (["--seed", seed] if seed else [])
+        out = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+        assert out.returncode == 0, out.stderr
+        lines.append(json.loads(out.stdout.strip().splitlines()[-1]))
+    assert all(ln["impl"] == "reference" and ln["value"] > 0 for ln in lines)
+    from awq_inputs import configs
+    wl = configs.WORKLOADS["C1"]
+    import dataclasses
+    a0 = configs.make_inputs(wl)[1]
+    a1 = configs.make_inputs(dataclasses.replace(wl, seed=123))[1]
+    assert not (a0 == a1).all()
+    # a reseeded workload has no stored oracle run to compare with
+    g = bench.golden_parity(dataclasses.replace(wl, seed=123), [1.0] * 20, 0, [1.0] * 512)
+    assert g is not None and "error" in g
