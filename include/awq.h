@@ -282,7 +282,9 @@ awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p, awq_dtype 
  * The dequantised weights enter the tensor cores in that type: fp16 rounds
  * (code - z) * Delta once; bf16 rounds Delta to bf16 and then the product.
  * Accumulation is fp32; Y is rounded once. Requires d_in a multiple of 32
- * and of g (AWQ_ERR_SHAPE).
+ * and of g (AWQ_ERR_SHAPE). cfg->group must be a group size (8 ... 256): the
+ * per-tensor layout (group 0, one step for the layer) is not read by this
+ * kernel and gives AWQ_ERR_INVALID_ARG.
  * Workspace: awq_w4a16_workspace_size (error word, split-K partials when
  * there are fewer output tiles than SMs); AWQ_ERR_WORKSPACE if smaller.
  * Asynchronous; device-side errors land in the workspace (awq_workspace_error). */

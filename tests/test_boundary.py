@@ -214,6 +214,8 @@ def test_w4a16_and_fold_validation():
     assert call(d_in=4000) == 2
     assert call(N=0) == 2
     assert call(cfg_=awq.make_cfg(4, 96, False, 1)) == 1
+    assert call(cfg_=awq.make_cfg(4, 0, False, 1)) == 1   # the per-tensor layout is not read by this kernel
+    assert awq.w4a16_workspace_size(16, 256, 4096, awq.make_cfg(4, 0, False, 1)) == 0
     assert call(X=None) == 1
     assert call(Y=None) == 1
     assert call(ws=None) == 1
