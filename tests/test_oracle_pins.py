@@ -282,6 +282,24 @@ def test_candidate_scales_closed_forms():
     assert np.allclose(O.alpha_grid(20), [k / 20 for k in range(20)])
 
 
+def test_normalisation_extremes_are_powers_of_the_extreme_statistics():
+    """For alpha >= 0, t = max(a, eps)^alpha does not decrease as a grows, so
+    max_j t_j and min_j t_j are the powers of the largest and smallest floored
+    a_j (the GPU kernel takes the normalisation from those two values alone);
+    the oracle's scales, built from every t_j, agree to float64 rounding."""
+    rng = np.random.default_rng(17)
+    for trial in range(20):
+        a = np.exp(rng.standard_normal(rng.integers(8, 600)) * 2.0)
+        a[rng.integers(0, a.size, 3)] = 0.0  # dead channels hit the floor
+        for al in O.alpha_grid(20):
+            t = np.maximum(a, O.EPS_A) ** al
+            fl = np.maximum(a, O.EPS_A)
+            assert t.max() == pytest.approx(fl.max() ** al, rel=1e-15)
+            assert t.min() == pytest.approx(fl.min() ** al, rel=1e-15)
+            shortcut = t / np.sqrt(fl.max() ** al * fl.min() ** al)
+            assert np.allclose(O.candidate_scales(a, al), shortcut, rtol=1e-14, atol=0)
+
+
 def test_scale_equivariance_of_normalisation():
     """Q(cV) = c Q(V) for c a power of two, so multiplying every s_i by c leaves
     Q(WS)S^-1 bit-identical; the sqrt(max*min) normalisation therefore only
