@@ -22,6 +22,9 @@ Generator
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 _GOLDEN = np.uint64(0x9E3779B97F4A7C15)
@@ -36,6 +39,22 @@ STREAM_CHANNEL_STD = 4
 STREAM_OUTLIER = 5
 
 _CHUNK = 1 << 22  # samples per vectorised chunk (bounds temporary memory)
+_THREADS = min(8, os.cpu_count() or 1)  # chunks are independent: filled by a thread pool
+
+
+def _fill_rows(n_rows, rows_per, fill):
+    """Call fill(r0, r1) over [0, n_rows) in blocks of rows_per rows, on a
+    thread pool (numpy releases the GIL in its array loops). Every sample
+    depends only on its position in its stream, so the bytes do not depend on
+    the blocking or the order."""
+    blocks = [(r0, min(n_rows, r0 + rows_per)) for r0 in range(0, n_rows, rows_per)]
+    if len(blocks) <= 1 or _THREADS <= 1:
+        for r0, r1 in blocks:
+            fill(r0, r1)
+        return
+    with ThreadPoolExecutor(_THREADS) as ex:
+        for f in [ex.submit(fill, r0, r1) for r0, r1 in blocks]:
+            f.result()
 
 
 def _mix64(z: np.ndarray) -> np.ndarray:
@@ -112,11 +131,12 @@ def make_weight(seed: int, d_out: int, d_in: int, w_std: float) -> np.ndarray:
     """W[d_out, d_in] ~ N(0, w_std^2), bf16 bits, row-major."""
     key = stream_key(seed, STREAM_W)
     out = np.empty((d_out, d_in), dtype=np.uint16)
-    rows_per = max(1, _CHUNK // max(d_in, 1))
-    for r0 in range(0, d_out, rows_per):
-        r1 = min(d_out, r0 + rows_per)
+
+    def fill(r0, r1):
         z = normal(key, r0 * d_in, (r1 - r0) * d_in)
         out[r0:r1] = f64_to_bf16_bits(w_std * z).reshape(r1 - r0, d_in)
+
+    _fill_rows(d_out, max(1, _CHUNK // max(d_in, 1)), fill)
     return out
 
 
@@ -138,14 +158,15 @@ def make_activations(seed: int, N: int, d_in: int, kind: str,
     outl = pick_channels(seed, d_in, outlier_count)
     chan[outl] *= outlier_factor
     out = np.empty((N, d_in), dtype=np.uint16)
-    rows_per = max(1, _CHUNK // max(d_in, 1))
-    for t0 in range(0, N, rows_per):
-        t1 = min(N, t0 + rows_per)
+
+    def fill(t0, t1):
         n = (t1 - t0) * d_in
         z = normal(key_x, t0 * d_in, n).reshape(t1 - t0, d_in)
         if kind == "absnormal":
             z = np.abs(z) * normal(key_x2, t0 * d_in, n).reshape(t1 - t0, d_in)
-        elif kind != "normal":
-            raise ValueError(f"unknown activation kind {kind!r}")
         out[t0:t1] = f64_to_bf16_bits(z * chan[None, :])
+
+    if kind not in ("normal", "absnormal"):
+        raise ValueError(f"unknown activation kind {kind!r}")
+    _fill_rows(N, max(1, _CHUNK // max(d_in, 1)), fill)
     return out

@@ -370,32 +370,47 @@ def pack(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bo
 
 
 def boundary_mask(W_bits: np.ndarray, s: np.ndarray, bits: int, group: int, symmetric: bool,
-                  band: float = 1e-4, clip: float = 1.0) -> np.ndarray:
+                  band: float = 1e-4, clip: float = 1.0, parts: bool = False):
     """Elements whose code the float64 oracle decides within ``band`` of a
-    rounding boundary: v/Delta (or -min/Delta for the zero point of the
-    element's group) lies within ``band`` of a half-integer. A float32
-    computation may round those either way; everything else must match."""
+    rounding boundary. Rounding to the nearest grid point ([P5] §2.3,
+    Q(w) = Delta round(w / Delta)) changes its answer only where w / Delta
+    crosses a half-integer, so an element is flagged when its own v / Delta
+    lies within ``band`` of one; with a zero point (asymmetric) every element
+    of a group also depends on z = round(-min v / Delta), so the whole group is
+    flagged when -min v / Delta lies within ``band`` of a half-integer. A
+    float32 computation may round flagged elements either way; everything else
+    must match.
+
+    Returns the combined [rows, d_in] mask, or with ``parts`` the pair
+    (element flags [rows, d_in], zero-point flags [rows, groups]) (for
+    group = 0: [1, 1] zero-point flags)."""
     W = widen_bf16(W_bits)
     V = W * np.asarray(s, dtype=np.float64)[None, :]
     if group == 0:  # per tensor: one group of all elements
         flat = W_bits.reshape(1, -1)
         s_flat = np.tile(np.asarray(s, dtype=np.float64), W_bits.shape[0])
-        return boundary_mask(flat, s_flat, bits, flat.shape[1], symmetric, band, clip).reshape(W_bits.shape)
+        el, zn = boundary_mask(flat, s_flat, bits, flat.shape[1], symmetric, band, clip, parts=True)
+        el = el.reshape(W_bits.shape)
+        return (el, zn) if parts else (el | zn[0, 0])
     rows, d_in = V.shape
     G = V.reshape(rows, d_in // group, group)
+
+    def near_half(r):
+        return np.abs(r - np.floor(r) - 0.5) < band
+
     if symmetric:
         delta = np.maximum(clip * np.abs(G).max(axis=-1), EPS_DELTA) / (2 ** (bits - 1) - 1)
-        r = G / delta[..., None]
-        near = np.abs(r - np.floor(r) - 0.5) < band
+        el = near_half(G / delta[..., None])
+        zn = np.zeros(delta.shape, dtype=bool)   # the zero point is fixed
     else:
         mx, mn = clip * G.max(axis=-1), clip * G.min(axis=-1)
         delta = np.maximum(mx - mn, EPS_DELTA) / (2 ** bits - 1)
-        r = G / delta[..., None]
-        near = np.abs(r - np.floor(r) - 0.5) < band
-        rz = -mn / delta
-        zn = np.abs(rz - np.floor(rz) - 0.5) < band
-        near |= zn[..., None]
-    return near.reshape(rows, d_in)
+        el = near_half(G / delta[..., None])
+        zn = near_half(-mn / delta)
+    el = el.reshape(rows, d_in)
+    if parts:
+        return el, zn
+    return el | np.repeat(zn, group, axis=1)
 
 
 # ---------------------------------------------------------------------------

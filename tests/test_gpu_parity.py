@@ -39,18 +39,33 @@ def check_stats(Xb, a_gpu):
     return a_ref
 
 
+EXCLUDE_FRAC = 1e-3  # bound on the fraction of codes (and of groups) left out near a rounding boundary
+
+
+def check_exclusions(el, zn):
+    """The band of rounding boundaries excludes about 2e-4 of the elements (and
+    of the groups, for their zero point) at random; bound each part by 1e-3,
+    plus a count of 3 elements / 1 group so that tiny layers, where a single
+    flagged group is already more than 1e-3 of them, do not fail by chance."""
+    n_el, n_g = int(el.sum()), int(zn.sum())
+    assert n_el <= EXCLUDE_FRAC * el.size + 3, f"{n_el} of {el.size} codes excluded"
+    assert n_g <= EXCLUDE_FRAC * zn.size + 1, f"{n_g} of {zn.size} zero points excluded"
+    return n_el, n_g
+
+
 def check_pack(Wb, s_ref, q, sc, zr, bits, g, sym):
     d_out, d_in = Wb.shape
     qw, sc_ref, zr_ref, codes_ref, delta_ref, zero_ref = O.pack(Wb, s_ref, bits, g, sym)
     codes = unpack_words(q, d_in)
-    near = O.boundary_mask(Wb, s_ref, bits, g, sym)
+    el, zn = O.boundary_mask(Wb, s_ref, bits, g, sym, parts=True)
+    near = el | np.repeat(zn, g, axis=1)
     bad = (codes != codes_ref) & ~near
     assert not bad.any(), f"{bad.sum()} codes differ away from rounding boundaries"
-    groups_near = near.reshape(d_out, d_in // g, g).any(axis=-1)
+    check_exclusions(el, zn)
     sc_g = sc.cpu().numpy().astype(np.float64)
     zr_g = zr.cpu().numpy().astype(np.float64)
     assert np.all(np.abs(sc_g - sc_ref.astype(np.float64)) <= 2.0 ** -10 * np.abs(sc_ref.astype(np.float64)) + 1e-12)
-    zbad = (zr_g != zr_ref.astype(np.float64)) & ~groups_near
+    zbad = (zr_g != zr_ref.astype(np.float64)) & ~zn
     assert not zbad.any(), f"{zbad.sum()} zero points differ"
     return int((codes != codes_ref).sum()), int(near.sum())
 

@@ -765,3 +765,129 @@ def test_per_tensor_pack_and_search_shapes():
     qw, sc, zr, codes, delta, zero = O.pack(Wb, res["s_best"], 4, 0, True)
     assert sc.shape == (1, 1) and zr.shape == (1, 1) and qw.shape == (4, 4)
     assert O.boundary_mask(Wb, res["s_best"], 4, 0, True).shape == (4, 32)
+
+
+# ---------------------------------------------------------------------------
+# the rounding-boundary band: which codes a float32 computation may decide
+# either way (AWQ (scholia-log) §2.3: Q(w) = Delta round(w / Delta) changes its
+# answer only where w / Delta crosses a half-integer)
+# ---------------------------------------------------------------------------
+BAND = 1e-4
+_IN, _OUT = 5e-5, 2e-4   # offsets inside and outside the band
+
+
+def test_boundary_band_asymmetric_elements():
+    """One asymmetric INT4 group of 8 with min 0 and max 1 (Delta = 1/15,
+    z = 0, -min/Delta = 0 far from any boundary); the other six elements are
+    0.5 * s_i with s_i placing v/Delta at chosen distances from a half-integer
+    or an integer. Only those within the band are flagged, and no zero point."""
+    targets = [2.5 + _IN, 4.5 - _IN, 6.5 + _OUT, 8.5 - _OUT, 10.5, 12.0 + _IN]
+    expect = [False, False, True, True, False, False, True, False]
+    W = _bits([[0.0, 1.0] + [0.5] * 6])
+    s = np.array([1.0, 1.0] + [2.0 * t / 15.0 for t in targets])
+    el, zn = O.boundary_mask(W, s, 4, 8, False, parts=True)
+    assert el[0].tolist() == expect
+    assert not zn.any()
+    assert O.boundary_mask(W, s, 4, 8, False)[0].tolist() == expect
+    # the band's width is the argument: widened past 2e-4, the outer pair joins
+    wide = O.boundary_mask(W, s, 4, 8, False, band=3e-4)[0]
+    assert wide.tolist() == [False, False, True, True, True, True, True, False]
+
+
+def test_boundary_band_symmetric_negative_side():
+    """Symmetric INT4, max |v| = 1 so Delta = 1/7 (AWQ (scholia-log) §3.1):
+    negative values at v/Delta = -(k + 1/2 +- e) are flagged inside the band
+    only (the fractional part is taken from below, floor, not by rounding);
+    the symmetric zero point is fixed and never flags a group."""
+    targets = [1.5 + _IN, 2.5 - _IN, 3.5 + _OUT, 4.5 - _OUT, 5.5, 3.0 - _IN, 0.5 + _IN]
+    expect = [False, True, True, False, False, True, False, True]
+    W = _bits([[1.0] + [-0.5] * 7])
+    s = np.array([1.0] + [2.0 * t / 7.0 for t in targets])
+    el, zn = O.boundary_mask(W, s, 4, 8, True, parts=True)
+    assert el[0].tolist() == expect
+    assert not zn.any()
+
+
+def test_boundary_band_zero_point_flags_the_whole_group():
+    """Asymmetric INT4, two groups of 8 in one row. Group A: v = (-m, 1, 0 ...)
+    with m chosen so that -min/Delta = 15 m / (1 + m) = 3.5 + e, so z sits at a
+    rounding boundary; group B is an ordinary group. Inside the band the whole
+    of group A is flagged (every code depends on z) and nothing of group B;
+    outside the band nothing is flagged at all."""
+    for e, flagged in ((_IN, True), (-_IN, True), (_OUT, False), (-_OUT, False)):
+        c = 3.5 + e
+        m = c / (15.0 - c)
+        W = _bits([[-0.5, 1.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0,
+                    0.25, -0.75, 0.5, 0.125, 1.0, -1.0, 0.0, 0.375]])
+        s = np.ones(16)
+        s[0] = 2.0 * m
+        s[8:] = [1.0, 1.0, 1.1, 0.9, 1.0, 0.8, 1.0, 1.3]   # group B: -min/Delta = 15*0.8/1.8 = 6.67
+        el, zn = O.boundary_mask(W, s, 4, 8, False, parts=True)
+        assert zn[0].tolist() == [flagged, False]
+        mask = O.boundary_mask(W, s, 4, 8, False)[0]
+        assert mask[:8].all() == flagged and mask[:8].any() == flagged
+        assert not mask[8:].any()
+        # the group's extremes sit at c and 15 - c on the grid: flagged with z
+        assert el[0, 0] == flagged and el[0, 1] == flagged and not el[0, 2:8].any()
+
+
+def test_boundary_band_per_tensor():
+    """group = 0: the layer is one group. Symmetric: Delta = 1/7 from the
+    layer's max wherever it sits; elements flagged as in a group. Asymmetric:
+    a zero point at a boundary flags every element of the layer."""
+    targets = [1.5 + _IN, 2.5 + _OUT, 3.5 - _IN]
+    W = _bits([[1.0, -0.5, -0.5, -0.5], [0.0, 0.0, 0.0, 0.0]])
+    s = np.array([1.0] + [2.0 * t / 7.0 for t in targets])
+    el, zn = O.boundary_mask(W, s, 4, 0, True, parts=True)
+    assert el.tolist() == [[False, True, False, True], [False] * 4]
+    assert zn.shape == (1, 1) and not zn.any()
+    for e, flagged in ((_IN, True), (_OUT, False)):
+        c = 3.5 + e
+        m = c / (15.0 - c)
+        Wa = _bits([[-0.5, 1.0, 0.0, 0.0], [0.0, 0.0, 0.0, 0.0]])
+        sa = np.array([2.0 * m, 1.0, 1.0, 1.0])
+        mask = O.boundary_mask(Wa, sa, 4, 0, False)
+        assert mask.all() == flagged and mask.any() == flagged
+
+
+def test_boundary_band_clip_uses_the_clipped_step():
+    """With clip ratio c the step comes from the shrunk range (max|v| -> c
+    max|v|): at c = 1/2, Delta = 1/14, so v = (2.5 + e)/14 is flagged and the
+    same v is not flagged at c = 1 (v/Delta = 1.25)."""
+    W = _bits([[1.0, 0.5, 0.0, 0.0]])
+    s = np.array([1.0, 2.0 * (2.5 + _IN) / 14.0, 1.0, 1.0])
+    assert O.boundary_mask(W, s, 4, 4, True, clip=0.5)[0].tolist() == [False, True, False, False]
+    assert not O.boundary_mask(W, s, 4, 4, True)[0].any()
+
+
+@pytest.mark.parametrize("bits,sym", [(4, False), (4, True), (3, True), (2, False)])
+def test_boundary_band_covers_every_float32_disagreement(bits, sym):
+    """Outside the band a float32 evaluation of the same quantiser (products,
+    step and 1/Delta in float32, round to nearest even) takes every code and
+    zero point the float64 oracle takes: the band is wide enough. Inside the
+    band the excluded fraction stays near its expectation 2 * band per
+    element (and per group for the zero point)."""
+    rng = np.random.default_rng(100 + bits + 10 * sym)
+    rows, d_in, g = 512, 1024, 64
+    Wb = gen.f64_to_bf16_bits(rng.standard_normal((rows, d_in)) * 0.02)
+    s = np.exp(rng.standard_normal(d_in))
+    codes64 = O.pack(Wb, s, bits, g, sym)[3]
+    el, zn = O.boundary_mask(Wb, s, bits, g, sym, parts=True)
+    # float32 restatement of the quantiser, written here for this check only
+    v = (O.widen_bf16(Wb).astype(np.float32) * s.astype(np.float32)).reshape(rows, -1, g)
+    if sym:
+        qmax = np.float32(2 ** (bits - 1) - 1)
+        d = np.abs(v).max(-1) / qmax
+        q = np.clip(np.rint(v * (np.float32(1) / d)[..., None]), -qmax - 1, qmax) + qmax + 1
+    else:
+        lv = np.float32(2 ** bits - 1)
+        mx, mn = v.max(-1), v.min(-1)
+        d = (mx - mn) / lv
+        inv = np.float32(1) / d
+        z = np.clip(np.rint(-mn * inv), 0, lv)
+        q = np.clip(np.rint(v * inv[..., None]) + z[..., None], 0, lv)
+    q = q.reshape(rows, d_in).astype(np.int64)
+    mask = el | np.repeat(zn, g, axis=1)
+    assert np.array_equal(q[~mask], codes64[~mask])
+    assert el.mean() <= 2 * BAND * 2
+    assert zn.mean() <= 2 * BAND * 5 + 1.0 / zn.size
