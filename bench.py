@@ -53,13 +53,17 @@ LOSS_RTOL = 1e-2  # candidate losses against the oracle's (relative)
 STATS_RTOL = 1e-5  # activation statistics against the oracle's (relative)
 
 
-def golden_parity(wl, losses, best, a):
+def golden_parity(wl, losses, best, a, packed=None):
     """The timed run's outputs against the stored oracle run of the same seeded
-    workload (tests/golden/search_<key>.json, written by
-    tests/golden/make_search_golden.py, which calls only the oracle): every
-    candidate loss, the choice (inside the oracle's set of choices within 0.5 %
-    of its best), and the sum of the activation statistics. Reads stored
-    numbers only; None if the workload has no stored run."""
+    workload (tests/golden/search_<key>.json and pack_<key>.{json,npz},
+    written by tests/golden/make_search_golden.py and make_pack_golden.py,
+    which call only the oracle): every candidate loss, the choice (inside the
+    oracle's set of choices within 0.5 % of its best), the sum of the
+    activation statistics, and, when ``packed`` = (qweight, scales, zeros) is
+    given, every packed code and zero point (a SHA-256 of the layer's codes
+    with the oracle's rounding-boundary positions blanked must equal the
+    stored one; the codes inside the band are counted) and the sum of the fp16
+    steps. Reads stored numbers only; None if the workload has no stored run."""
     path = os.path.join(ROOT, "tests", "golden", f"search_{wl.key}.json")
     if not os.path.exists(path):
         return None
@@ -73,14 +77,73 @@ def golden_parity(wl, losses, best, a):
     got = np.asarray(losses, dtype=np.float64)
     rel = float(np.max(np.abs(got - ref) / ref))
     a_rel = abs(float(np.sum(np.asarray(a, dtype=np.float64))) - g["a_checksum"]) / g["a_checksum"]
-    out.update({
-        "loss_max_rel": rel, "loss_rtol": LOSS_RTOL,
-        "alpha_index": int(best), "oracle_alpha_set": g["acceptable"],
-        "a_sum_rel": a_rel,
-        "ok": bool(rel <= LOSS_RTOL and int(best) in g["acceptable"] and a_rel <= STATS_RTOL),
-        "codes": "compared element by element in the GPU parity tests, not here",
-    })
+    ok = bool(rel <= LOSS_RTOL and int(best) in g["acceptable"] and a_rel <= STATS_RTOL)
+    out.update({"loss_max_rel": rel, "loss_rtol": LOSS_RTOL,
+                "alpha_index": int(best), "oracle_alpha_set": g["acceptable"], "a_sum_rel": a_rel})
+    if packed is not None:
+        codes = pack_parity(wl, int(best), *packed)
+        out["codes"] = codes
+        ok = ok and bool(codes.get("ok"))
+    out["ok"] = ok
     return out
+
+
+def unpack_codes_host(words, d_in):
+    """uint32 words [rows, d_in/8] -> codes uint8 [rows, d_in] (nibble j of
+    word w is channel 8w + j)."""
+    rows = words.shape[0]
+    out = np.empty((rows, d_in // 8, 8), dtype=np.uint8)
+    for j in range(8):
+        out[:, :, j] = (words >> np.uint32(4 * j)) & np.uint32(0xF)
+    return out.reshape(rows, d_in)
+
+
+def pack_parity(wl, best, qweight, scales, zeros):
+    """Every code and zero point of the timed run's pack against the stored
+    oracle digests of the same choice of alpha (see golden_parity)."""
+    jpath = os.path.join(ROOT, "tests", "golden", f"pack_{wl.key}.json")
+    npath = os.path.join(ROOT, "tests", "golden", f"pack_{wl.key}.npz")
+    if not (os.path.exists(jpath) and os.path.exists(npath)):
+        return {"ok": False, "error": f"no stored pack digest for {wl.key}"}
+    with open(jpath) as f:
+        meta = json.load(f)
+    if meta.get("workload") != wl.as_dict() or str(best) not in meta["choices"]:
+        return {"ok": False, "error": "no stored pack digest for this workload and choice"}
+    ch = meta["choices"][str(best)]
+    arr = np.load(npath)
+    el_idx = arr[f"k{best}_near_idx"].astype(np.int64)
+    near_ref = arr[f"k{best}_near_codes"]
+    zn_idx = arr[f"k{best}_zero_near_groups"].astype(np.int64)
+    codes = unpack_codes_host(qweight.cpu().numpy().view(np.uint32), wl.d_in)
+    zbits = zeros.cpu().numpy().view(np.uint16).copy()
+    ng = wl.d_in // wl.group
+    flipped = int((codes.reshape(-1)[el_idx] != near_ref).sum())
+    codes.reshape(-1)[el_idx] = 0xFF
+    r, j = np.divmod(zn_idx, ng)
+    codes.reshape(codes.shape[0], ng, wl.group)[r, j, :] = 0xFF
+    zbits.reshape(-1)[zn_idx] = 0xFFFF
+    codes_ok = hashlib.sha256(codes.tobytes()).hexdigest() == ch["codes_sha256"]
+    zeros_ok = hashlib.sha256(zbits.tobytes()).hexdigest() == ch["zeros_sha256"]
+    sc_sum = float(scales.cpu().numpy().astype(np.float64).sum())
+    sc_rel = abs(sc_sum - ch["scale_sum"]) / ch["scale_sum"]
+    return {"against": f"tests/golden/pack_{wl.key}.json (stored oracle pack digests)",
+            "compared": ch["codes"], "zero_points_compared": ch["groups"],
+            "codes_equal_off_band": bool(codes_ok), "zero_points_equal_off_band": bool(zeros_ok),
+            "near_boundary_codes": ch["near_codes"], "near_boundary_zero_points": ch["near_zero_points"],
+            "excluded_fraction": round((ch["near_codes"] + ch["near_zero_points"] * wl.group) / ch["codes"], 7),
+            "codes_differing_inside_band": flipped, "scale_sum_rel": sc_rel,
+            "ok": bool(codes_ok and zeros_ok and sc_rel <= 1e-3)}
+
+
+L2_NOTE = ("flushed: 256 MiB write between timed GPU steps, outside the step events "
+           "(the CPU oracle arm has no device cache to flush)")
+
+
+def workload_config(wl, world):
+    """The workload as both arms name it (same keys and values)."""
+    return {"workload": f"{wl.key}: {wl.title}", "d_out": wl.d_out, "d_in": wl.d_in, "N": wl.N,
+            "bits": wl.bits, "group": wl.group, "symmetric": wl.symmetric, "n_alpha": wl.n_alpha,
+            "l2": L2_NOTE, "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 def kernel_source_hash():
@@ -328,7 +391,8 @@ def run_ours(args, rank, world, local_rank):
     clk = clocks.stop()
     # the last timed step's outputs against the stored oracle run (stored numbers only)
     try:
-        parity = golden_parity(wl, outs["losses"].cpu().numpy(), int(outs["best"].item()), a.cpu().numpy())
+        parity = golden_parity(wl, outs["losses"].cpu().numpy(), int(outs["best"].item()), a.cpu().numpy(),
+                               packed=packed)
     except Exception as e:  # report it; the timing stands
         parity = {"error": f"{type(e).__name__}: {e}"}
 
@@ -551,11 +615,9 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"{wl.key}: {wl.title}", "d_out": d_out, "d_in": d_in, "N": N, "bits": wl.bits,
-                   "group": wl.group, "symmetric": wl.symmetric, "n_alpha": n_a, "form": form,
-                   "l2": "flushed: 256 MiB write between timed steps, outside the step events",
-                   "timing": graph_note,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": workload_config(wl, world),
+        "form": form,
+        "timing": graph_note,
         "roofline": {"kernel": "gemm_pair_bf16_tcgen05 (CTA pairs, " + ("direct, sum-of-squares epilogue)" if form == "direct"
                                                                  else "block-triangular Gram, dot epilogue)"),
                      "bound": "tensor", "achieved": round(achieved_tflops, 2),
@@ -584,7 +646,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "wall_s_timed_region": round(t_wall, 3),
     }
-    return line
+    return line, (Wb, Xb)
 
 
 # ----------------------------------------------------------------------------- W4A16 alone
@@ -634,78 +696,91 @@ def run_w4a16_only(args):
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_sample(wl, rows_total, block=256):
-    """Time the CPU oracle on a bounded sample of one layer: the full
-    statistics, the search on `rows_total` rows (the per-row cost is uniform)
-    and their pack; extrapolated to the whole layer."""
+ORACLE_ROW_COST_S = 7e-10  # single-thread oracle seconds per row per (d_in * N), 20 alphas (measured)
+
+
+def sample_rows(wl, seconds):
+    """Rows of W whose search by the single-thread oracle takes about
+    ``seconds`` (the cost per row grows with d_in * N): a multiple of 8, at
+    least 8, at most d_out."""
+    rows = int(seconds / (ORACLE_ROW_COST_S * wl.d_in * wl.N)) // 8 * 8
+    return int(min(wl.d_out, max(8, rows)))
+
+
+def oracle_sample(wl, Wb, Xb, rows, r0=0, tokens=None, a_full=None, block=256):
+    """Time the CPU oracle, as it stands, on a bounded sample of one layer:
+    the statistics over ``tokens`` tokens (all by default; the cost is linear
+    in tokens), the search of ``rows`` rows starting at r0 over all N tokens
+    and every alpha, and their pack; scaled to the whole layer by tokens and
+    rows. With a token slice the search reads ``a_full``, the statistics of
+    all tokens (computed once by the caller). Returns (layer seconds, seconds
+    actually spent)."""
     from oracle import awq_oracle as O
-    Wb, Xb = make_inputs(wl)
+    tokens = wl.N if tokens is None else min(tokens, wl.N)
     t0 = time.perf_counter()
-    a = O.act_stats(Xb)
+    a = O.act_stats(Xb[:tokens])
     t_stats = time.perf_counter() - t0
-    rows_total = min(rows_total, wl.d_out)
-    t_search = 0.0
-    t_pack = 0.0
-    for r0 in range(0, rows_total, block):
-        rows = np.arange(r0, min(rows_total, r0 + block))
+    if tokens < wl.N:
+        a = a_full  # the search needs the statistics of all tokens
+    t_rows = 0.0
+    idx = (r0 + np.arange(rows)) % wl.d_out
+    for b0 in range(0, rows, block):
+        sel = idx[b0:b0 + block]
         t0 = time.perf_counter()
-        res = O.search(Wb, Xb, a, wl.bits, wl.group, wl.symmetric, wl.n_alpha, rows=rows)
-        t_search += time.perf_counter() - t0
-        t0 = time.perf_counter()
-        O.pack(Wb[rows], res["s_best"], wl.bits, wl.group, wl.symmetric)
-        t_pack += time.perf_counter() - t0
-    scale = wl.d_out / rows_total
-    t_layer = t_stats + (t_search + t_pack) * scale
-    return t_layer, rows_total, t_stats + t_search + t_pack
+        res = O.search(Wb, Xb, a, wl.bits, wl.group, wl.symmetric, wl.n_alpha, rows=sel)
+        O.pack(Wb[sel], res["s_best"], wl.bits, wl.group, wl.symmetric)
+        t_rows += time.perf_counter() - t0
+    t_layer = t_stats * (wl.N / tokens) + t_rows * (wl.d_out / rows)
+    return t_layer, t_stats + t_rows
 
 
-def cpu_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("internal_api") == "openblas"]
-        if n:
-            return int(max(n))
-    except Exception:
-        pass
-    return os.cpu_count() or 1
+def single_thread():
+    """The oracle is single-threaded: BLAS limited to one thread."""
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=1)
 
 
-def cpu_sample_rows(wl, budget=4096 * 4096 * 4096):
-    """Rows of W for the CPU baseline: the oracle's cost per row grows with
-    d_in * N, so the sample holds budget / (d_in * N) rows (the whole 4096-row
-    layer at 4096 x 4096 x 4096, about 10 s on 16 host threads), in multiples
-    of 256, at least 256 and at most d_out."""
-    rows = budget // (wl.d_in * wl.N) // 256 * 256
-    return int(min(wl.d_out, max(256, rows)))
+def cpu_baseline_entry(wl, Wb, Xb, rows):
+    with single_thread():
+        t_layer, spent = oracle_sample(wl, Wb, Xb, rows)
+    part = (f"the whole layer ({rows} rows) x {wl.n_alpha} alphas" if rows == wl.d_out else
+            f"{rows} of {wl.d_out} rows x {wl.n_alpha} alphas, extrapolated by rows")
+    return {"value": round(wl.n_alpha / t_layer, 4), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{wl.key}: statistics of all {wl.N} tokens, search and pack of {part} "
+                      f"(float64 numpy, BLAS limited to 1 thread); {spent:.1f} s of CPU work",
+            "extrapolated": rows < wl.d_out}
 
 
-def cpu_baseline_entry(wl, rows):
-    t_layer, r, spent = oracle_sample(wl, rows)
-    part = (f"the whole layer ({r} rows) x {wl.n_alpha} alphas" if r == wl.d_out else
-            f"{r} of {wl.d_out} rows x {wl.n_alpha} alphas, extrapolated by rows")
-    return {"value": round(wl.n_alpha / t_layer, 4), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{wl.key}: statistics, search and pack of {part} (float64 numpy, BLAS matmul); "
-                      f"{spent:.1f} s of CPU work"}
-
-
-def run_reference(args, wl):
+def run_reference(args, wl, world):
+    """The oracle arm: each step times the oracle on a bounded sample of the
+    layer (statistics over a token slice, search and pack of a row slice over
+    all tokens and alphas, the slice moving from step to step), scaled to the
+    whole layer; inputs generated once, before the steps."""
+    Wb, Xb = make_inputs(wl)
+    rows = args.ref_rows if args.ref_rows else sample_rows(wl, 3.0)
+    tokens = min(wl.N, args.ref_tokens)
     K = args.steps
-    times = []
-    rows = args.ref_rows
-    for k in range(args.warmup + K):
-        t_layer, r, _ = oracle_sample(wl, rows)
-        if k >= args.warmup:
-            times.append(t_layer)
+    times, spent = [], []
+    with single_thread():
+        from oracle import awq_oracle as O
+        a_full = O.act_stats(Xb) if tokens < wl.N else None
+        for k in range(args.warmup + K):
+            t_layer, sp = oracle_sample(wl, Wb, Xb, rows, r0=(k * rows) % wl.d_out, tokens=tokens, a_full=a_full)
+            if k >= args.warmup:
+                times.append(t_layer)
+                spent.append(sp)
     ms = 1e3 * sum(times) / K
     value = wl.n_alpha / (ms * 1e-3)
+    sample = (f"per step: statistics of {tokens} of {wl.N} tokens (scaled by tokens), search and pack of "
+              f"{rows} of {wl.d_out} rows x {wl.n_alpha} alphas over all tokens (scaled by rows); float64 numpy, "
+              f"BLAS limited to 1 thread")
     return {
-        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 1, "steps": K,
-        "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms, 2), "extrapolated": True,
+        "sample_s_per_step": round(float(np.mean(spent)), 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{wl.key}: {wl.title}", "d_out": wl.d_out, "d_in": wl.d_in, "N": wl.N},
-        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                         "sample": f"per step: full statistics + search and pack of {min(rows, wl.d_out)} of "
-                                   f"{wl.d_out} rows, extrapolated by rows"},
+        "config": workload_config(wl, world),
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -715,12 +790,15 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="C2", choices=sorted(WORKLOADS))
+    ap.add_argument("--config", default="C5", choices=sorted(WORKLOADS),
+                    help="workload (default C5, the 70B MLP layer: the largest single-GPU configuration)")
     ap.add_argument("--form", default="auto", choices=["auto", "direct", "gram"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--ref-rows", type=int, default=None,
+                    help="rows of W per step of the oracle arm (default: about 3 s of single-thread work)")
+    ap.add_argument("--ref-tokens", type=int, default=8192, help="tokens of the oracle arm's statistics sample")
     ap.add_argument("--cpu-rows", type=int, default=None,
-                    help="rows of W in the CPU baseline's sample (default: cpu_sample_rows)")
+                    help="rows of W in the CPU baseline's sample (default: about 15 s of single-thread work)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-group-clip", action="store_true", help="skip the per-group clipping pass")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 inference-side timing")
@@ -757,7 +835,7 @@ def main():
 
     if args.impl == "reference":
         if rank == 0:
-            emit(run_reference(args, wl))
+            emit(run_reference(args, wl, world))
         return
 
     if world > 1:
@@ -768,11 +846,11 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line, (Wb, Xb) = run_ours(args, rank, world, local_rank)
         if rank == 0:
-            if not args.no_cpu_baseline:
-                rows = args.cpu_rows if args.cpu_rows is not None else cpu_sample_rows(wl)
-                line["cpu_baseline"] = cpu_baseline_entry(wl, rows)
+            if world == 1 and not args.no_cpu_baseline:
+                rows = args.cpu_rows if args.cpu_rows is not None else sample_rows(wl, 15.0)
+                line["cpu_baseline"] = cpu_baseline_entry(wl, Wb, Xb, rows)
             emit(line)
     finally:
         if world > 1:

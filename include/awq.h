@@ -93,10 +93,13 @@ awq_status awq_act_stats(const void* X_bf16, int64_t N, int64_t d_in, float* a, 
  * loads the library holds until the process exits. No cudaMalloc, cudaFree or
  * other allocating call is made.
  *   - Limits: N >= 1, d_in a multiple of 8 and at most 524288; larger d_in
- *     returns AWQ_ERR_SHAPE (tall inputs use fewer, taller row chunks).
+ *     returns AWQ_ERR_SHAPE. Any N within those limits fits the array.
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and caches it with the
+ *     id of the device's current context; make that first call before any
+ *     stream capture. After the context is destroyed and rebuilt
+ *     (cudaDeviceReset), the next call sees a new context id and looks the
+ *     address up again (so that call, too, belongs before any capture).
  *   - All calls in the process share the one array: calls whose work overlaps
  *     on the GPU (different streams or threads) race and give wrong results.
  *     Calls ordered on one stream are safe; nothing needs clearing between

@@ -83,16 +83,55 @@ def test_reference_arm_json_line(tmp_path):
     assert line["impl"] == "reference" and line["unit"] == bench.UNIT and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["higher_is_better"] is True
+    assert line["extrapolated"] is True and line["sample_s_per_step"] > 0 and line["cpu_baseline"]["cores"] == 1
+    from awq_inputs import configs
+    assert line["config"] == bench.workload_config(configs.WORKLOADS["C1"], 1)
 
 
-def test_cpu_sample_rows_bounded_and_whole_layer_at_c2():
+def test_sample_rows_bounded():
     from awq_inputs import configs
     for key, wl in configs.WORKLOADS.items():
-        r = bench.cpu_sample_rows(wl)
-        assert 256 <= r <= max(256, wl.d_out) and (r % 256 == 0 or r == wl.d_out), key
-        # per-row oracle cost ~ d_in * N: the sample stays within the 4096^3 budget unless at its floor
-        assert r == 256 or r * wl.d_in * wl.N <= 4096 ** 3, key
-    assert bench.cpu_sample_rows(configs.WORKLOADS["C2"]) == 4096
+        for secs in (3.0, 15.0):
+            r = bench.sample_rows(wl, secs)
+            assert 8 <= r <= wl.d_out and (r % 8 == 0 or r == wl.d_out), key
+            # per-row oracle cost ~ d_in * N: the sample stays within its time unless at its floor
+            assert r == 8 or r * wl.d_in * wl.N * bench.ORACLE_ROW_COST_S <= secs, key
+    assert bench.sample_rows(configs.WORKLOADS["C1"], 15.0) == 256  # the whole small layer
+
+
+def test_pack_parity_against_stored_digests():
+    """bench's code check: the oracle's own pack of C1 passes; a code changed
+    away from the rounding-boundary band fails it; a code changed inside the
+    band is counted and passes."""
+    import numpy as np
+    import torch
+    from awq_inputs import configs
+    from oracle import awq_oracle as O
+    wl = configs.WORKLOADS["C1"]
+    with open(os.path.join(ROOT, "tests", "golden", "search_C1.json")) as f:
+        k = json.load(f)["best"]
+    Wb, Xb = configs.make_inputs(wl)
+    s = O.candidate_scales(O.act_stats(Xb), O.alpha_grid(wl.n_alpha)[k])
+    qw, sc, zr, codes, _, _ = O.pack(Wb, s, wl.bits, wl.group, wl.symmetric)
+    el = O.boundary_mask(Wb, s, wl.bits, wl.group, wl.symmetric)
+
+    def as_torch(q, c=None):
+        if c is not None:
+            q = O.pack_codes(c)
+        return (torch.from_numpy(q.view(np.int32)), torch.from_numpy(sc), torch.from_numpy(zr))
+
+    res = bench.pack_parity(wl, k, *as_torch(qw))
+    assert res["ok"] and res["codes_differing_inside_band"] == 0 and res["compared"] == Wb.size
+    far = codes.copy()
+    r, c = np.argwhere(~el)[5]
+    far[r, c] ^= 1
+    assert not bench.pack_parity(wl, k, *as_torch(None, far))["ok"]
+    inside = codes.copy()
+    r, c = np.argwhere(el)[0]
+    inside[r, c] ^= 1
+    res = bench.pack_parity(wl, k, *as_torch(None, inside))
+    assert res["ok"] and res["codes_differing_inside_band"] == 1
+    assert not bench.pack_parity(wl, (k + 5) % wl.n_alpha, *as_torch(qw))["ok"]  # no digest for that choice
 
 
 def test_golden_parity_reads_stored_oracle_runs():

@@ -869,23 +869,64 @@ constexpr int kNoallocMaxDevices = 64;
 // Loaded on every device that loads the library and held until the process exits.
 static __device__ __align__(256) double g_noalloc_stats_scratch[kNoallocScratchDoubles];
 
+// One call's partial sums are n_chunks * d_in doubles. stats_layout gives a
+// single chunk when a row of column blocks already fills its target grid, and
+// otherwise at most target / col_blocks + 1 chunks, so the partials never
+// exceed (2 * target) * STATS_COLS doubles for any d_in the array admits.
+static_assert(2ll * kStatsTargetBlocks * STATS_COLS <= kNoallocScratchDoubles,
+              "the statistics' partial sums must fit the scratch array for every admitted d_in");
+
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+struct NoallocSlot {
+  unsigned long long ctx_id;  // context the address belongs to (0: none yet)
+  void* ptr;
+};
+NoallocSlot g_noalloc_slot[kNoallocMaxDevices] = {};
+
+// Process-unique id of the current context, or 0 when the runtime has not made
+// one current yet (cuCtxGetId ids are never reused within a process).
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of the scratch array on the current device. In host code the
-// array's name is only a host-side stand-in, so its address is looked up once
-// per device (with that device current) and cached.
+// array's name is only a host-side stand-in, so its address is looked up with
+// the device current and cached per device, together with the id of the
+// context it was found in. If that context is destroyed and another one takes
+// its place (cudaDeviceReset), the library's module, and the array with it, is
+// loaded anew at another address: the changed context id makes the next call
+// look the address up again instead of using the stale one.
 awq_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return AWQ_ERR_CUDA;
   if (dev < 0 || dev >= kNoallocMaxDevices) return AWQ_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  const unsigned long long id = current_context_id();
+  if (!slot.ptr || id == 0 || id != slot.ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_stats_scratch) != cudaSuccess || !p) return AWQ_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx_id = current_context_id();  // the lookup made the device's context current
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return AWQ_OK;
 }
 
@@ -895,16 +936,9 @@ extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t d_
   if (!X || !a) return AWQ_ERR_INVALID_ARG;
   if (!aligned(X, 16)) return AWQ_ERR_INVALID_ARG;
   if (check_tokens(N) != AWQ_OK || d_in < 8 || d_in % 8 != 0 || d_in > kNoallocScratchDoubles) return AWQ_ERR_SHAPE;
-  // same chunking as awq_act_stats, with fewer, taller row chunks when the
-  // partial sums (one fp64 per chunk and channel) would not fit the array
-  StatsLayout L = stats_layout(N, d_in);
-  const long long max_chunks = kNoallocScratchDoubles / d_in;
-  if ((long long)L.n_chunks > max_chunks) {
-    long long rpc = cdiv(N, max_chunks);
-    rpc = cdiv(rpc, 32) * 32;
-    L.rows_per_chunk = (int)rpc;
-    L.n_chunks = (int)cdiv(N, rpc);
-  }
+  // same chunking as awq_act_stats; its partial sums always fit the array (see
+  // the static_assert above), checked again here before anything is enqueued
+  const StatsLayout L = stats_layout(N, d_in);
   if ((long long)L.n_chunks * d_in > kNoallocScratchDoubles) return AWQ_ERR_SHAPE;
   awq_status st = check_device(nullptr);
   if (st != AWQ_OK) return st;
