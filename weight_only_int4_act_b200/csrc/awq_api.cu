@@ -744,7 +744,8 @@ awq_status pack_impl(const void* W, const float* s, int64_t d_out, int64_t d_in,
   }
   if (!(clip > 0.f && clip <= 1.f)) return AWQ_ERR_INVALID_ARG;
   if (!W || !s || !qweight || !scales || !zeros) return AWQ_ERR_INVALID_ARG;
-  if (!aligned(W, 16) || !aligned(s, 16) || !aligned(qweight, 4) || !aligned(scales, 2) || !aligned(zeros, 2))
+  // qweight: the kernel stores 8-byte pairs of words
+  if (!aligned(W, 16) || !aligned(s, 16) || !aligned(qweight, 8) || !aligned(scales, 2) || !aligned(zeros, 2))
     return AWQ_ERR_INVALID_ARG;
   int sms = 0;
   if ((st = check_device(&sms)) != AWQ_OK) return st;

@@ -658,13 +658,16 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
       if (active && row0 + r < d_out) {
         const int row = row0 + r;
         uint32_t* wp = qweight + (long long)row * words + c0 / 8;
+        uint32_t wd[CPT / 8];
 #pragma unroll
-        for (int q = 0; q < CPT / 8; ++q) {
-          uint32_t word = 0;
+        for (int q = 0; q < CPT / 8; ++q) wd[q] = fq_word(fr, q);
+        if (AWQ_SPAN_OK((long long)row * words + c0 / 8, CPT / 8, (long long)d_out * words, BS_PACK_Q)) {
+          if constexpr (CPT == 16) {
+            __stcs(reinterpret_cast<uint2*>(wp), make_uint2(wd[0], wd[1]));  // 8-byte aligned: c0 % 16 == 0
+          } else {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) word |= (fq_code(fr, 8 * q + j) & 0xFu) << (4 * j);
-          if (AWQ_IDX_OK((long long)row * words + c0 / 8 + q, (long long)d_out * words, BS_PACK_Q))
-            __stcs(wp + q, word);
+            for (int q = 0; q < CPT / 8; ++q) __stcs(wp + q, wd[q]);
+          }
         }
         if (PT ? (row == 0 && chunk == 0) : (chunk & (GL - 1)) == 0) {
           const long long gidx = PT ? 0 : (long long)row * groups + chunk / GL;

@@ -177,4 +177,20 @@ __device__ __forceinline__ unsigned fq_code(const FqGroup<CPT>& r, int j) {
   return (unsigned)(r.c[j] - kRoundMagic);
 }
 
+// Word q of the packed codes: nibble j holds the code of element 8q + j.
+// A magic-form code c = 1.5*2^23 + code (0 <= code < 2^22) has the fp32 bit
+// pattern 0x4B400000 + code, so sum_j bits(c_j) 16^j (mod 2^32) is the word
+// plus the constant 0x4B400000 * 0x11111111: a Horner chain of integer
+// multiply-adds and one subtraction, with no float-to-integer conversion.
+constexpr uint32_t kMagicBits = 0x4B400000u;  // fp32 bits of kRoundMagic
+constexpr uint32_t kMagicWordBias = (uint32_t)((unsigned long long)kMagicBits * 0x11111111ull);
+
+template <int CPT>
+__device__ __forceinline__ uint32_t fq_word(const FqGroup<CPT>& r, int q) {
+  uint32_t acc = __float_as_uint(r.c[8 * q + 7]);
+#pragma unroll
+  for (int j = 6; j >= 0; --j) acc = acc * 16u + __float_as_uint(r.c[8 * q + j]);
+  return acc - kMagicWordBias;
+}
+
 }  // namespace awq
