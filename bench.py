@@ -649,50 +649,163 @@ def run_ours(args, rank, world, local_rank):
     return line, (Wb, Xb)
 
 
-# ----------------------------------------------------------------------------- W4A16 alone
-def run_w4a16_only(args):
-    """The W4A16 kernel alone on the workload's layer shape with `--tokens`
-    tokens: W packed at s = 1 by the library's own pack, activations from the
-    workload's generator. For profiling the kernel on its own."""
+# ----------------------------------------------------------------------------- one entry point alone
+ONLY = ("stats", "pack", "fake_quant", "gram", "contract", "group_clip", "fold", "per_tensor", "segmented", "w4a16")
+
+
+def run_only(args):
+    """One entry point of the library alone on the workload's shapes (for
+    per-kernel timing and for single-kernel profiler captures): `--steps`
+    timed calls after `--warmup` untimed ones, L2 flushed before each, CUDA
+    events around each call on the launching stream. W and X come from the
+    workload's generator; where the call needs scale vectors that the search
+    would produce, it gets s = (a / mean a)^0.4 computed from the workload's
+    statistics (a vector of the search's form; the time does not depend on
+    which one). The JSON line gives the median time and the call's rate
+    against its roofline."""
     import torch
     import weight_only_int4_act_b200 as awq
+    from weight_only_int4_act_b200 import binding as B
     from awq_inputs import gen
 
+    import ctypes
     wl = WORKLOADS[args.config]
     dev = torch.device("cuda", 0)
-    Wb = gen.make_weight(wl.seed, wl.d_out, wl.d_in, wl.w_std)
-    Xb = gen.make_activations(wl.seed, args.tokens, wl.d_in, wl.x_kind, wl.x_lognormal_sigma, wl.outlier_count,
-                              wl.outlier_factor)
-    W = torch.from_numpy(Wb.view(np.int16)).view(torch.bfloat16).to(dev)
-    X = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).to(dev)
-    if args.dtype == "f16":
-        X = X.to(torch.float16)
-    cfg = awq.make_cfg(wl.bits, wl.group, wl.symmetric, 1)
-    pk = awq.quantize_pack(W, torch.ones(wl.d_in, dtype=torch.float32, device=dev), cfg)
-    ws = awq.workspace(awq.w4a16_workspace_size(args.tokens, wl.d_out, wl.d_in, cfg))
-    Y = torch.empty((args.tokens, wl.d_out), dtype=X.dtype, device=dev)
+    peaks = load_peaks()
+    what = args.only
+    d_out, d_in, N = wl.d_out, wl.d_in, wl.N
+    ng = d_in // wl.group
+    cfg = awq.make_cfg(wl.bits, wl.group, wl.symmetric, wl.n_alpha)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    tokens = args.tokens if what == "w4a16" else N
+    W = bf16(gen.make_weight(wl.seed, d_out, d_in, wl.w_std))
+    X = bf16(gen.make_activations(wl.seed, tokens, d_in, wl.x_kind, wl.x_lognormal_sigma, wl.outlier_count,
+                                  wl.outlier_factor))
+    a = awq.act_stats(X)
+    s = ((a / a.mean()).clamp_min(1e-4) ** 0.4).contiguous()
+    note, byts, flops, kernels = "", None, None, []
+    keep = []  # buffers the timed call uses
+
+    if what == "stats":
+        ws = awq.workspace(awq.stats_workspace_size(N, d_in))
+        keep.append(ws)
+        fn = lambda: awq.act_stats(X, ws, out=a)  # noqa: E731
+        byts = N * d_in * 2 + d_in * 4
+        kernels = ["act_absmean_partial", "act_absmean_final"]
+    elif what in ("pack", "per_tensor"):
+        del X
+        pcfg = cfg if what == "pack" else awq.make_cfg(wl.bits, 0, wl.symmetric, 1)
+        shape = (d_out, ng) if what == "pack" else (1, 1)
+        outs = (torch.empty((d_out, d_in // 8), dtype=torch.int32, device=dev),
+                torch.empty(shape, dtype=torch.float16, device=dev), torch.empty(shape, dtype=torch.float16, device=dev))
+        ws = awq.workspace(max(awq.pack_workspace_size(d_out, d_in, pcfg), 256)) if what == "per_tensor" else None
+        keep += [outs, ws]
+        fn = lambda: awq.quantize_pack(W, s, pcfg, outputs=outs, ws=ws)  # noqa: E731
+        byts = d_out * d_in * 2 + d_out * d_in // 2 + d_in * 4 + (4 * d_out * ng if what == "pack" else d_out * d_in * 2)
+        kernels = ["quantize_pack"] if what == "pack" else ["col_minmax", "tensor_extremes", "quantize_pack"]
+        if what == "per_tensor":
+            note = "per tensor (group 0): W is read twice (extremes, then the pack)"
+    elif what in ("fake_quant", "gram", "contract"):
+        ws = awq.workspace(awq.search_workspace_size(d_out, d_in, N, cfg))
+        keep.append(ws)
+        awq.search_scales(W, X, a, cfg, ws=ws)
+        L, cptr, st = B.lib(), ctypes.byref(cfg), B._stream()
+        wsp, wsn = ctypes.c_void_p(ws.data_ptr()), ws.numel()
+        form = awq.search_form(d_out, d_in, N, cfg)
+        tri = tri_macs_per_row(d_in)
+        if what == "fake_quant":
+            fn = lambda: B._check(L.awq_step_fake_quant(ctypes.c_void_p(W.data_ptr()), d_out, d_in, N, cptr, wsp,  # noqa: E731
+                                                        wsn, st), "fq")
+            byts = d_out * d_in * 2 + wl.n_alpha * d_out * d_in * 2
+            kernels = ["fake_quant_delta"]
+        elif what == "gram":
+            if form != "gram":
+                raise SystemExit(f"{wl.key} runs the direct form: no Gram product")
+            fn = lambda: B._check(L.awq_step_gram(ctypes.c_void_p(X.data_ptr()), d_out, d_in, N, cptr, wsp, wsn, st),  # noqa: E731
+                                  "gram")
+            flops = 2.0 * N * tri
+            kernels = ["gemm_bf16_tcgen05 (EPI_STORE, MN-major, lower block triangle)"]
+        else:
+            fn = lambda: B._check(L.awq_step_contract(ctypes.c_void_p(X.data_ptr()), d_out, d_in, N, cptr, wsp,  # noqa: E731
+                                                      wsn, st), "contract")
+            flops = 2.0 * wl.n_alpha * d_out * (tri if form == "gram" else d_in * N)
+            kernels = [f"gemm_pair_bf16_tcgen05 ({form} form)"]
+    elif what == "group_clip":
+        ccfg = awq.make_cfg(wl.bits, wl.group, wl.symmetric, len(GROUP_CLIPS))
+        ws = awq.workspace(awq.group_clip_workspace_size(d_out, d_in, N, ccfg))
+        keep.append(ws)
+        fn = lambda: awq.search_group_clip(W, X, s, GROUP_CLIPS, ccfg, ws=ws)  # noqa: E731
+        flops = 2.0 * N * 256 * d_in + 2.0 * len(GROUP_CLIPS) * d_out * 256 * d_in
+        kernels = ["repeat_scales", "fake_quant_delta", "gemm_bf16_tcgen05 (EPI_STORE, TRI_DIAG_STORE)",
+                   "gemm_bf16_tcgen05 (EPI_DOT32, TRI_DIAG)", "group_clip_argmin"]
+        note = f"{len(GROUP_CLIPS)} clip ratios; flops are those issued (the diagonal 256-blocks)"
+    elif what == "fold":
+        Xt = X.t().contiguous()  # [d_in, N]: channel on the first axis, as a producer's weight
+        del X
+        keep.append(Xt)
+        fn = lambda: awq.fold_inv_scales(s, Xt)  # noqa: E731
+        byts = 4 * N * d_in + 4 * d_in
+        kernels = ["fold_inv_scales_kernel"]
+        note = "in place on a [d_in, N] bf16 parameter"
+    elif what == "segmented":
+        seg = [d_out // 3, d_out // 3, d_out - 2 * (d_out // 3)]
+        ws = awq.workspace(awq.search_workspace_size(d_out, d_in, N, cfg))
+        keep.append(ws)
+        fn = lambda: awq.search_scales_segmented(W, X, a, cfg, seg, ws=ws)  # noqa: E731
+        kernels = ["candidate_scales", "fake_quant_delta", "gemm (Gram / contraction)", "segment_loss_reduce",
+                   "segment_argmin"]
+        note = f"three layers of {seg} rows sharing X"
+    elif what == "w4a16":
+        dt = torch.float16 if args.dtype == "f16" else torch.bfloat16
+        pk = awq.quantize_pack(W, torch.ones(d_in, dtype=torch.float32, device=dev), cfg)
+        Xp = X.to(dt).contiguous()
+        wsw = awq.workspace(awq.w4a16_workspace_size(tokens, d_out, d_in, cfg))
+        Y = torch.empty((tokens, d_out), dtype=dt, device=dev)
+        keep += [pk, Xp, wsw, Y]
+        fn = lambda: awq.w4a16_gemm(Xp, *pk, cfg, ws=wsw, out=Y)  # noqa: E731
+        byts = d_out * d_in // 2 + 4 * d_out * ng + tokens * (d_in + d_out) * 2
+        flops = 2.0 * tokens * d_out * d_in
+        kernels = ["w4a16_gemm_tcgen05", "w4a16_split_reduce"]
+        note = f"{tokens} tokens, {args.dtype} activations, W packed at s = 1"
+    else:
+        raise SystemExit(f"unknown --only {what}")
+
     for _ in range(args.warmup):
-        awq.w4a16_gemm(X, *pk, cfg, ws=ws, out=Y)
+        fn()
     torch.cuda.synchronize()
     ms = []
     for k in range(args.steps):
         flush.fill_(k & 0xFF)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        awq.w4a16_gemm(X, *pk, cfg, ws=ws, out=Y)
+        fn()
         e1.record()
         e1.synchronize()
         ms.append(e0.elapsed_time(e1))
-    awq.workspace_error(ws)
-    t = float(np.mean(ms))
-    byts = wl.d_out * wl.d_in // 2 + 4 * wl.d_out * (wl.d_in // wl.group) + args.tokens * (wl.d_in + wl.d_out) * 2
-    return {"metric": "W4A16 product (awq_w4a16_gemm)", "value": round(t, 4), "unit": "ms",
-            "higher_is_better": False, "steps": args.steps, "warmup": args.warmup,
-            "config": {"workload": f"{wl.key} layer {wl.d_out}x{wl.d_in}, {args.tokens} tokens",
-                       "bits": wl.bits, "group": wl.group, "activations": args.dtype, "l2": "flushed between runs"},
-            "gbs": round(byts / (t * 1e-3) / 1e9, 1),
-            "tflops": round(2.0 * args.tokens * wl.d_out * wl.d_in / (t * 1e-3) / 1e12, 2)}
+    for t in keep:
+        if t is not None and hasattr(t, "dtype") and t.dtype == torch.uint8 and t.dim() == 1:
+            awq.workspace_error(t)
+    t = float(np.median(ms))
+    line = {"metric": f"{what} alone", "value": round(t, 4), "unit": "ms", "higher_is_better": False,
+            "steps": args.steps, "warmup": args.warmup, "kernels": kernels,
+            "config": {"workload": f"{wl.key}: {wl.title}", "d_out": d_out, "d_in": d_in,
+                       "N": tokens, "bits": wl.bits, "group": wl.group, "symmetric": wl.symmetric,
+                       "l2": "flushed before each call"}}
+    if byts is not None:
+        line["gbs"] = round(byts / (t * 1e-3) / 1e9, 1)
+        line["hbm_frac"] = round(byts / (t * 1e-3) / 1e9 / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), 4)
+        line["algorithmic_bytes"] = int(byts)
+    if flops is not None:
+        line["tflops"] = round(flops / (t * 1e-3) / 1e12, 2)
+        line["tensor_frac"] = round(flops / (t * 1e-3) / 1e12 / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]), 4)
+        line["flops"] = flops
+    if note:
+        line["note"] = note
+    return line
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -803,7 +916,7 @@ def main():
     ap.add_argument("--no-group-clip", action="store_true", help="skip the per-group clipping pass")
     ap.add_argument("--no-w4a16", action="store_true", help="skip the W4A16 inference-side timing")
     ap.add_argument("--no-graph", action="store_true", help="time the eager public calls only")
-    ap.add_argument("--only", default=None, choices=["w4a16"], help="time one component alone (its own JSON line)")
+    ap.add_argument("--only", default=None, choices=ONLY, help="time one entry point alone (its own JSON line)")
     ap.add_argument("--tokens", type=int, default=16, help="tokens for --only w4a16")
     ap.add_argument("--dtype", default="f16", choices=["f16", "bf16"], help="activations for --only w4a16")
     ap.add_argument("--json-out", default=None, help="also write the JSON line to this file")
@@ -828,9 +941,9 @@ def main():
             with open(args.json_out, "w") as f:
                 f.write(text + "\n")
 
-    if args.only == "w4a16":
+    if args.only:
         if rank == 0:
-            emit(run_w4a16_only(args))
+            emit(run_only(args))
         return
 
     if args.impl == "reference":
