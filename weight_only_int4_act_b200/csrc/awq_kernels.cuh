@@ -603,29 +603,56 @@ __global__ void __launch_bounds__(256) quantize_pack(const __nv_bfloat16* __rest
                                                      const float* __restrict__ ext) {
   const int chunks = d_in / CPT;
   const int row_groups = (d_out + PACK_ROWS - 1) / PACK_ROWS;
-  const long long total = (long long)row_groups * chunks;
-  const long long warp_global = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const long long n_warps = ((long long)gridDim.x * blockDim.x) >> 5;
+  // A warp task is 32 consecutive chunks (lanes) of one group of PACK_ROWS rows,
+  // task t = (row group t / citers, chunk pass t % citers). Warps stride over
+  // the tasks (the grid works on neighbouring rows at any time); the stride is
+  // split into row groups and passes once, so stepping needs no division.
+  const int citers = (chunks + 31) >> 5;
+  const int n_warps = (int)((gridDim.x * blockDim.x) >> 5);
+  const int warp_global = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int step_rg = n_warps / citers, step_ci = n_warps - step_rg * citers;
+  int rg = warp_global / citers;
+  int ci = warp_global - rg * citers;
   const int lane = threadIdx.x & 31;
   const bool sym = symmetric != 0;
   const int groups = d_in / (GL * CPT);
   const int words = d_in / 8;
-  for (long long base = warp_global * 32; base < total; base += n_warps * 32) {
-    const long long u = base + lane;
-    const bool active = u < total;
-    const int rg = active ? (int)(u / chunks) : 0;
-    const int chunk = active ? (int)(u - (long long)rg * chunks) : 0;
-    const int c0 = chunk * CPT;
+  // W of the next task is loaded while this one is quantised (one task of
+  // loads in flight per warp during the arithmetic)
+  auto load_w = [&](int rg_, int ci_, uint4 (&dst)[PACK_ROWS][CPT / 8]) {
+    const int ch = ci_ * 32 + lane;
+    const bool act = rg_ < row_groups && ch < chunks;
+    const int cc = act ? ch * CPT : 0;
+#pragma unroll
+    for (int r = 0; r < PACK_ROWS; ++r)
+#pragma unroll
+      for (int q = 0; q < CPT / 8; ++q)
+        dst[r][q] = (act && rg_ * PACK_ROWS + r < d_out &&
+                     AWQ_SPAN_OK((long long)(rg_ * PACK_ROWS + r) * d_in + cc + 8 * q, 8, (long long)d_out * d_in,
+                                 BS_PACK_W))
+                        ? __ldcs(reinterpret_cast<const uint4*>(W + (long long)(rg_ * PACK_ROWS + r) * d_in + cc) + q)
+                        : make_uint4(0, 0, 0, 0);
+  };
+  uint4 wnext[PACK_ROWS][CPT / 8];
+  load_w(rg, ci, wnext);
+  for (; rg < row_groups; rg += step_rg, ci += step_ci, rg += (ci >= citers), ci -= (ci >= citers) ? citers : 0) {
+    const int chunk = ci * 32 + lane;
+    const bool active = chunk < chunks;
+    const int c0 = active ? chunk * CPT : 0;
     const int row0 = rg * PACK_ROWS;
     uint4 wraw[PACK_ROWS][CPT / 8];
 #pragma unroll
     for (int r = 0; r < PACK_ROWS; ++r)
 #pragma unroll
-      for (int q = 0; q < CPT / 8; ++q)
-        wraw[r][q] = (active && row0 + r < d_out &&
-                      AWQ_SPAN_OK((long long)(row0 + r) * d_in + c0 + 8 * q, 8, (long long)d_out * d_in, BS_PACK_W))
-                         ? __ldcs(reinterpret_cast<const uint4*>(W + (long long)(row0 + r) * d_in + c0) + q)
-                         : make_uint4(0, 0, 0, 0);
+      for (int q = 0; q < CPT / 8; ++q) wraw[r][q] = wnext[r][q];
+    {
+      int ci2 = ci + step_ci, rg2 = rg + step_rg;
+      if (ci2 >= citers) {
+        ci2 -= citers;
+        ++rg2;
+      }
+      load_w(rg2, ci2, wnext);
+    }
     float sc[CPT];
     if (AWQ_SPAN_OK(c0, CPT, d_in, BS_PACK_S)) {
       load_f32<CPT>(s + c0, sc);

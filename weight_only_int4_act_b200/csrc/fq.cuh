@@ -14,8 +14,11 @@
 //               z = clamp(rne(-min v / Delta), 0, 2^b - 1)
 //               q = clamp(rne(v / Delta) + z, 0, 2^b - 1),   v_hat = (q - z) Delta
 // Arithmetic is fp32; Delta is the range times the fp32 constant 1/levels,
-// 1/Delta is the correctly rounded reciprocal, and rne(v / Delta) is rounded
-// from the exact product v * (1/Delta).
+// 1/Delta is the hardware reciprocal (at most 1 ulp from the correctly rounded
+// one), and rne(v / Delta) is rounded from the exact product v * (1/Delta):
+// v / Delta is off by a few 1e-7 relative, so a code can differ from the
+// exact decision only where v / Delta lies within ~5e-6 of a rounding
+// boundary.
 #pragma once
 #include <cuda_runtime.h>
 
@@ -58,6 +61,14 @@ __device__ __forceinline__ float group_min(float x) {
 #pragma unroll
   for (int off = 1; off < GL; off <<= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, off));
   return x;
+}
+
+// 1/x by the special-function unit (rcp.approx: at most 1 ulp of error; x is a
+// quantisation step, normal and positive).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 // Three-input max / min (one instruction on sm_100).
@@ -113,7 +124,7 @@ __device__ __forceinline__ void fq_group(const float (&v)[CPT], int bits, bool s
     const float amax = clip * group_max<GL>(fmaxf(maxN(v), -minN(v)));
     const float half = (float)(1 << (bits - 1));  // -qmin
     r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
-    const float inv = __frcp_rn(r.delta);
+    const float inv = rcp_approx(r.delta);
     r.zero = half;
     r.off = kRoundMagic + half;
     a = inv * inv_span;
@@ -122,7 +133,7 @@ __device__ __forceinline__ void fq_group(const float (&v)[CPT], int bits, bool s
     const float mx = clip * group_max<GL>(maxN(v));
     const float mn = clip * group_min<GL>(minN(v));
     r.delta = fmaxf(mx - mn, kEpsDelta) * inv_span;
-    const float inv = __frcp_rn(r.delta);
+    const float inv = rcp_approx(r.delta);
     r.zero = fminf(fmaxf(__fmaf_rn(-mn, inv, kRoundMagic) - kRoundMagic, 0.f), span);  // clamp(rne(-min / Delta))
     r.off = kRoundMagic + r.zero;
     a = inv * inv_span;
@@ -146,7 +157,7 @@ __device__ __forceinline__ void fq_from_extremes(const float (&v)[CPT], int bits
     const float amax = clip * fmaxf(mx, -mn);
     const float half = (float)(1 << (bits - 1));
     r.delta = fmaxf(amax, kEpsDelta) * inv_levels(bits - 1);
-    const float inv = __frcp_rn(r.delta);
+    const float inv = rcp_approx(r.delta);
     r.zero = half;
     r.off = kRoundMagic + half;
     a = inv * inv_span;
@@ -155,7 +166,7 @@ __device__ __forceinline__ void fq_from_extremes(const float (&v)[CPT], int bits
     mx *= clip;
     mn *= clip;
     r.delta = fmaxf(mx - mn, kEpsDelta) * inv_span;
-    const float inv = __frcp_rn(r.delta);
+    const float inv = rcp_approx(r.delta);
     r.zero = fminf(fmaxf(__fmaf_rn(-mn, inv, kRoundMagic) - kRoundMagic, 0.f), span);
     r.off = kRoundMagic + r.zero;
     a = inv * inv_span;
