@@ -689,10 +689,12 @@ def run_only(args):
     s = ((a / a.mean()).clamp_min(1e-4) ** 0.4).contiguous()
     note, byts, flops, kernels = "", None, None, []
     keep = []  # buffers the timed call uses
+    err_ws = []  # of those, the workspaces with a device error word (all but the pack's)
 
     if what == "stats":
         ws = awq.workspace(awq.stats_workspace_size(N, d_in))
         keep.append(ws)
+        err_ws.append(ws)
         fn = lambda: awq.act_stats(X, ws, out=a)  # noqa: E731
         byts = N * d_in * 2 + d_in * 4
         kernels = ["act_absmean_partial", "act_absmean_final"]
@@ -712,6 +714,7 @@ def run_only(args):
     elif what in ("fake_quant", "gram", "contract"):
         ws = awq.workspace(awq.search_workspace_size(d_out, d_in, N, cfg))
         keep.append(ws)
+        err_ws.append(ws)
         awq.search_scales(W, X, a, cfg, ws=ws)
         L, cptr, st = B.lib(), ctypes.byref(cfg), B._stream()
         wsp, wsn = ctypes.c_void_p(ws.data_ptr()), ws.numel()
@@ -738,6 +741,7 @@ def run_only(args):
         ccfg = awq.make_cfg(wl.bits, wl.group, wl.symmetric, len(GROUP_CLIPS))
         ws = awq.workspace(awq.group_clip_workspace_size(d_out, d_in, N, ccfg))
         keep.append(ws)
+        err_ws.append(ws)
         fn = lambda: awq.search_group_clip(W, X, s, GROUP_CLIPS, ccfg, ws=ws)  # noqa: E731
         flops = 2.0 * N * 256 * d_in + 2.0 * len(GROUP_CLIPS) * d_out * 256 * d_in
         kernels = ["repeat_scales", "fake_quant_delta", "gemm_bf16_tcgen05 (EPI_STORE, TRI_DIAG_STORE)",
@@ -755,6 +759,7 @@ def run_only(args):
         seg = [d_out // 3, d_out // 3, d_out - 2 * (d_out // 3)]
         ws = awq.workspace(awq.search_workspace_size(d_out, d_in, N, cfg))
         keep.append(ws)
+        err_ws.append(ws)
         fn = lambda: awq.search_scales_segmented(W, X, a, cfg, seg, ws=ws)  # noqa: E731
         kernels = ["candidate_scales", "fake_quant_delta", "gemm (Gram / contraction)", "segment_loss_reduce",
                    "segment_argmin"]
@@ -766,6 +771,7 @@ def run_only(args):
         wsw = awq.workspace(awq.w4a16_workspace_size(tokens, d_out, d_in, cfg))
         Y = torch.empty((tokens, d_out), dtype=dt, device=dev)
         keep += [pk, Xp, wsw, Y]
+        err_ws.append(wsw)
         fn = lambda: awq.w4a16_gemm(Xp, *pk, cfg, ws=wsw, out=Y)  # noqa: E731
         byts = d_out * d_in // 2 + 4 * d_out * ng + tokens * (d_in + d_out) * 2
         flops = 2.0 * tokens * d_out * d_in
@@ -786,9 +792,8 @@ def run_only(args):
         e1.record()
         e1.synchronize()
         ms.append(e0.elapsed_time(e1))
-    for t in keep:
-        if t is not None and hasattr(t, "dtype") and t.dtype == torch.uint8 and t.dim() == 1:
-            awq.workspace_error(t)
+    for t in err_ws:  # workspaces that carry the device error word
+        awq.workspace_error(t)
     t = float(np.median(ms))
     line = {"metric": f"{what} alone", "value": round(t, 4), "unit": "ms", "higher_is_better": False,
             "steps": args.steps, "warmup": args.warmup, "kernels": kernels,
