@@ -295,13 +295,20 @@ awq_status run_gemm(const void* A, long long M, long long lda, const void* B, lo
   return launch_status();
 }
 
-// The contraction on CTA pairs (gemm_pair_sm100.cuh): 256 x 256 tiles.
-template <int MODE>
+// The contraction and the Gram product on CTA pairs (gemm_pair_sm100.cuh):
+// 256 x 256 tiles. MN = true: A and B are row-major [K, M] / [K, Nr]
+// matrices read transposed.
+template <int MODE, bool MN = false>
 awq_status run_gemm_pair(const void* A, long long M, long long lda, const void* B, long long Nr, long long ldb,
                          long long K, GemmArgs args, int tri, int num_sms, cudaStream_t st, const GemmExtents& ext) {
   CUtensorMap ta, tb;
-  if (!make_map(&ta, A, M, K, lda, 128)) return AWQ_ERR_CUDA;
-  if (!make_map(&tb, B, Nr, K, ldb, 128)) return AWQ_ERR_CUDA;
+  if (MN) {
+    if (!make_map(&ta, A, K, M, lda, GEMM_BK)) return AWQ_ERR_CUDA;
+    if (!make_map(&tb, B, K, Nr, ldb, GEMM_BK)) return AWQ_ERR_CUDA;
+  } else {
+    if (!make_map(&ta, A, M, K, lda, 128)) return AWQ_ERR_CUDA;
+    if (!make_map(&tb, B, Nr, K, ldb, 128)) return AWQ_ERR_CUDA;
+  }
   args.M = (int)M;
   args.N = (int)Nr;
   args.K = (int)K;
@@ -309,22 +316,25 @@ awq_status run_gemm_pair(const void* A, long long M, long long lda, const void* 
   args.n_blocks_n = (int)cdiv(Nr, PAIR_BN);
   args.group_n = kGroupN < args.n_blocks_n ? kGroupN : args.n_blocks_n;
   args.tri = tri;
-  const long long tiles = (long long)args.n_blocks_m * args.n_blocks_n;
+  // TRI_LOWER_STORE: the tiles of the lower block triangle (row block mb, column blocks 0 .. mb)
+  const long long tiles = tri == TRI_LOWER_STORE ? (long long)args.n_blocks_m * (args.n_blocks_m + 1) / 2
+                                                 : (long long)args.n_blocks_m * args.n_blocks_n;
   if (tiles > INT32_MAX) return AWQ_ERR_SHAPE;
   args.num_tiles = (int)tiles;
   if (!gemm_extents_ok<MODE>(args, PAIR_BN, ext)) return AWQ_ERR_BOUNDS;
-  if (cudaFuncSetAttribute(gemm_pair_bf16_tcgen05<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(gemm_pair_bf16_tcgen05<MODE, MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            PAIR_SMEM_BYTES) != cudaSuccess)
     return AWQ_ERR_CUDA;
   if (cudaMemsetAsync(args.tile_counter, 0, sizeof(int), st) != cudaSuccess) return AWQ_ERR_CUDA;
   const long long pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
-  gemm_pair_bf16_tcgen05<MODE><<<(unsigned)(2 * pairs), GEMM_THREADS, PAIR_SMEM_BYTES, st>>>(ta, tb, args);
+  gemm_pair_bf16_tcgen05<MODE, MN><<<(unsigned)(2 * pairs), GEMM_THREADS, PAIR_SMEM_BYTES, st>>>(ta, tb, args);
   return launch_status();
 }
 
 #ifndef AWQ_GEMM_PAIR
 #define AWQ_GEMM_PAIR 1
 #endif
+
 
 // Grid of a grid-stride kernel with 256-thread blocks: enough blocks for the
 // work, at most one wave of resident blocks.
@@ -531,8 +541,8 @@ awq_status awq_step_gram(const void* X, int64_t d_out, int64_t d_in, int64_t N, 
   GemmExtents ext;
   ext.C = (long long)d_in * d_in;
   // G = X^T X with both operands read transposed from X [N, d_in] (MN-major)
-  return run_gemm<EPI_STORE, true>(X, d_in, d_in, X, d_in, d_in, N, ga, TRI_LOWER_STORE, sms, as_stream(stream),
-                                   ext);
+  return run_gemm_pair<EPI_STORE, true>(X, d_in, d_in, X, d_in, d_in, N, ga, TRI_LOWER_STORE, sms,
+                                        as_stream(stream), ext);
 }
 
 awq_status awq_step_contract(const void* X, int64_t d_out, int64_t d_in, int64_t N, const awq_qcfg* cfg, void* ws,

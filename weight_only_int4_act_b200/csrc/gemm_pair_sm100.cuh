@@ -1,7 +1,10 @@
-// The loss contraction on CTA pairs (tcgen05 cta_group::2) for sm_100a.
+// The loss contraction and the Gram product on CTA pairs (tcgen05
+// cta_group::2) for sm_100a.
 //
-// Same product and epilogues as gemm_sm100.cuh (EPI_SUMSQ, EPI_DOT; TRI_NONE
-// or TRI_K), but each 256 x 256 tile is computed by a cluster of two CTAs on
+// Same products and epilogues as gemm_sm100.cuh (EPI_SUMSQ, EPI_DOT with
+// TRI_NONE or TRI_K; EPI_STORE with TRI_LOWER_STORE and MN-major operands for
+// G' = the lower block triangle of X^T X), but each 256 x 256 tile is computed
+// by a cluster of two CTAs on
 // two SMs: CTA r of the pair loads rows [128 r, 128 r + 128) of the tile's A
 // panel and of its B panel (64-wide K stages, TMA, no multicast), and one
 // thread of the even CTA issues M=256 N=256 K=16 MMAs that read both CTAs'
@@ -39,7 +42,29 @@ constexpr int PAIR_SLOTS = 4;
 constexpr int PAIR_SMEM_BYTES = 1024 + PAIR_STAGES * (PAIR_A_STAGE + PAIR_B_STAGE) + 512;
 static_assert(PAIR_SMEM_BYTES <= 232448, "shared memory per CTA");
 
-template <int MODE>
+// Tile t of the lower block triangle of 256 x 256 tiles: row block mb holds
+// column blocks 0 .. mb (t = mb (mb + 1) / 2 + nb).
+__device__ __forceinline__ void pair_tri_coords(int t, int& mb, int& nb) {
+  int q = (int)((sqrtf(8.0f * (float)t + 1.0f) - 1.0f) * 0.5f);
+  while ((long long)(q + 1) * (q + 2) / 2 <= t) ++q;
+  while ((long long)q * (q + 1) / 2 > t) --q;
+  mb = q;
+  nb = t - q * (q + 1) / 2;
+}
+
+__device__ __forceinline__ void pair_tile_coords(int t, const GemmArgs& a, int& mb, int& nb) {
+  if (a.tri == TRI_LOWER_STORE)
+    pair_tri_coords(t, mb, nb);
+  else
+    gemm_tile_coords(t, a, mb, nb);
+}
+
+// MN = false: A [M, K] and B [N, K] row-major (K-major operands); each CTA loads
+// one box of 64 (K) x 128 rows of each per stage.
+// MN = true: A and B are the same row-major [K, M] matrix read transposed
+// (G = X^T X straight from X): each CTA loads two boxes of 64 (M or N) x 64
+// (K) per operand and stage, at 64-column offsets.
+template <int MODE, bool MN = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_bf16_tcgen05(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const GemmArgs args) {
@@ -128,7 +153,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         }
         if (t < 0) break;
         int mb, nb;
-        gemm_tile_coords(t, args, mb, nb);
+        pair_tile_coords(t, args, mb, nb);
         const int num_kb = gemm_num_kb(args, nb);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.err, ERR_WAIT_EMPTY)) {
@@ -137,10 +162,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           }
           const uint32_t full_even = mapa_shared(full_bar(stage), 0);
           if (even) mbar_arrive_expect_tx(full_bar(stage), 2 * (PAIR_A_STAGE + PAIR_B_STAGE));
-          tma_load_2d_pair(smem_u32(sA + stage * PAIR_A_STAGE), &tmA, full_even, kb * PAIR_BK,
-                           mb * PAIR_BM + (int)rank * 128);
-          tma_load_2d_pair(smem_u32(sB + stage * PAIR_B_STAGE), &tmB, full_even, kb * PAIR_BK,
-                           nb * PAIR_BN + (int)rank * 128);
+          if constexpr (MN) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              tma_load_2d_pair(smem_u32(sA + stage * PAIR_A_STAGE + c * GEMM_MN_CHUNK), &tmA, full_even,
+                               mb * PAIR_BM + (int)rank * 128 + c * 64, kb * PAIR_BK);
+              tma_load_2d_pair(smem_u32(sB + stage * PAIR_B_STAGE + c * GEMM_MN_CHUNK), &tmB, full_even,
+                               nb * PAIR_BN + (int)rank * 128 + c * 64, kb * PAIR_BK);
+            }
+          } else {
+            tma_load_2d_pair(smem_u32(sA + stage * PAIR_A_STAGE), &tmA, full_even, kb * PAIR_BK,
+                             mb * PAIR_BM + (int)rank * 128);
+            tma_load_2d_pair(smem_u32(sB + stage * PAIR_B_STAGE), &tmB, full_even, kb * PAIR_BK,
+                             nb * PAIR_BN + (int)rank * 128);
+          }
           issued |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == PAIR_STAGES) {
@@ -163,7 +198,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && even) {
       // ---------------- MMA issuer (even CTA)
-      constexpr uint32_t IDESC = idesc_bf16_f32(PAIR_BM, PAIR_BN);
+      constexpr uint32_t IDESC = idesc_bf16_f32(PAIR_BM, PAIR_BN, MN);
       int stage = 0;
       uint32_t phase = 0;
       int slot = 0;
@@ -184,7 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * PAIR_BN;
         int mb, nb;
-        gemm_tile_coords(t, args, mb, nb);
+        pair_tile_coords(t, args, mb, nb);
         const int num_kb = gemm_num_kb(args, nb);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, args.err, ERR_WAIT_FULL)) {
@@ -195,9 +230,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           const uint32_t a_base = smem_u32(sA + stage * PAIR_A_STAGE);
           const uint32_t b_base = smem_u32(sB + stage * PAIR_B_STAGE);
 #pragma unroll
-          for (int k = 0; k < PAIR_BK / 16; ++k)
-            mma_bf16_pair(d_tmem, desc_kmajor_sw128(a_base + k * 32), desc_kmajor_sw128(b_base + k * 32), IDESC,
-                          (kb | k) != 0);
+          for (int k = 0; k < PAIR_BK / 16; ++k) {
+            // K-major: 16 elements = 32 B along the swizzled row; MN-major: 16 rows of 128 B
+            const uint64_t ad = MN ? desc_mnmajor_sw128(a_base + k * 2048, GEMM_MN_CHUNK)
+                                   : desc_kmajor_sw128(a_base + k * 32);
+            const uint64_t bd = MN ? desc_mnmajor_sw128(b_base + k * 2048, GEMM_MN_CHUNK)
+                                   : desc_kmajor_sw128(b_base + k * 32);
+            mma_bf16_pair(d_tmem, ad, bd, IDESC, (kb | k) != 0);
+          }
           mma_commit_pair(empty_bar(stage), 0x3);
           if (++stage == PAIR_STAGES) {
             stage = 0;
@@ -232,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       }
       if (t < 0) break;
       int mb, nb;
-      gemm_tile_coords(t, args, mb, nb);
+      pair_tile_coords(t, args, mb, nb);
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       const bool ready = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, args.err, ERR_WAIT_TFULL);
@@ -262,6 +302,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
             const float d = __uint_as_float(r[j]);
             sum = fmaf(d, d, sum);
           }
+        } else if constexpr (MODE == EPI_STORE) {
+          // G' = 2 G on strictly lower blocks, G on diagonal blocks (TRI_LOWER_STORE)
+          const int col = n0 + c * 32;
+          const float scale = nb < mb ? 2.0f : 1.0f;
+          if (m < args.M) {
+            __nv_bfloat16* crow = args.C + (long long)m * args.ldC + col;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              if (col + v * 8 < args.N) {
+                uint32_t w[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  __nv_bfloat162 p = __floats2bfloat162_rn(scale * __uint_as_float(r[v * 8 + 2 * h]),
+                                                           scale * __uint_as_float(r[v * 8 + 2 * h + 1]));
+                  w[h] = *reinterpret_cast<uint32_t*>(&p);
+                }
+                *reinterpret_cast<uint4*>(crow + v * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+          }
         } else {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -282,7 +342,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         else
           mbar_arrive_remote(mapa_shared(tempty_bar(acc), 0));
       }
-      if (m < args.M) args.part[(long long)nb * args.part_ld + m] = sum;
+      if constexpr (MODE != EPI_STORE) {
+        if (m < args.M) args.part[(long long)nb * args.part_ld + m] = sum;
+      }
     }
   }
 
