@@ -36,6 +36,7 @@ METRIC = "AWQ search: alpha-candidate layer evals/s, TFLOP/s vs bf16 peak; stats
 UNIT = "alpha-candidate layer evals/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 L2_FLUSH_BYTES = 256 << 20
+LONG_STEP_MS = 10.0  # steps at least this long are timed against the sustained (power-capped) peak
 GROUP_CLIPS = [1.0, 0.95, 0.9, 0.85, 0.8, 0.75, 0.7, 0.6, 0.5]  # ratios of the per-group clipping pass
 
 
@@ -592,9 +593,13 @@ def run_ours(args, rank, world, local_rank):
     flops_gram = 0.0 if form == "direct" else 2.0 * N * tri
     c_ms = breakdown["contraction"]
     achieved_tflops = flops_search / (c_ms * 1e-3) / 1e12
-    # the timed region is short and runs at full clock (see "clocks"): burst peak
-    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     peak_sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # a step of tens of milliseconds repeated for the timed region runs under the
+    # power cap: the sustained peak is its denominator; short steps run at full
+    # clock against the burst peak (the other fraction is reported beside it)
+    long_step = ms_per_step >= LONG_STEP_MS
+    peak = peak_sustained if long_step else peak_burst
     stats_bytes = N * d_in * 2 + d_in * 4
     pack_bytes = d_out * d_in * 2 + d_out * d_in // 2 + 2 * 2 * d_out * (d_in // wl.group) + d_in * 4
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
@@ -622,7 +627,9 @@ def run_ours(args, rank, world, local_rank):
                                                                  else "block-triangular Gram, dot epilogue)"),
                      "bound": "tensor", "achieved": round(achieved_tflops, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved_tflops / peak, 4),
-                     "peak_kind": f"bf16 dense burst ({peaks.get('source')})",
+                     "peak_kind": (f"bf16 dense sustained ({peaks.get('source')}; step >= {LONG_STEP_MS} ms)"
+                                   if long_step else f"bf16 dense burst ({peaks.get('source')})"),
+                     "frac_of_burst": round(achieved_tflops / peak_burst, 4),
                      "frac_of_sustained": round(achieved_tflops / peak_sustained, 4),
                      "traffic": profiled_traffic(wl.key, form),
                      "algorithmic_flops_per_launch": flops_search},
@@ -761,7 +768,7 @@ def run_only(args):
         keep.append(ws)
         err_ws.append(ws)
         fn = lambda: awq.search_scales_segmented(W, X, a, cfg, seg, ws=ws)  # noqa: E731
-        kernels = ["candidate_scales", "fake_quant_delta", "gemm (Gram / contraction)", "segment_loss_reduce",
+        kernels = ["candidate_scales", "fake_quant_delta", "gemm (Gram / contraction)", "row_loss_rows", "segment_loss_reduce",
                    "segment_argmin"]
         note = f"three layers of {seg} rows sharing X"
     elif what == "w4a16":

@@ -25,6 +25,9 @@ constexpr size_t kAlign = 1024;
 constexpr size_t kTileCounterOffset = 256;
 constexpr int kStatsTargetBlocks = 148 * 4;  // one wave at 4 resident blocks per SM
 constexpr int kGroupN = 8;
+#ifndef AWQ_PAIR_GROUP_N
+#define AWQ_PAIR_GROUP_N 8
+#endif
 
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
@@ -114,7 +117,7 @@ struct SearchLayout {
   long long M;      // rows of the dW stack
   int n_blocks_n;   // column tiles of the contraction
   int n_red_chunks; // blocks per alpha in the row reduction
-  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_seg, off_ext, off_g, total;
+  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_seg, off_rows64, off_ext, off_g, total;
 };
 
 // sum over 256-wide column blocks J of width(J) * min(d_in, 256 (J + 1)): the
@@ -159,6 +162,7 @@ SearchLayout search_layout(int64_t d_out, int64_t d_in, int64_t N, const awq_qcf
   L.off_blk = off;    off += align_up((size_t)L.n_alpha * L.n_red_chunks * sizeof(double));
   L.off_loss64 = off; off += align_up((size_t)L.n_alpha * sizeof(double));
   L.off_seg = off;    off += align_up((size_t)MAX_ALPHA * MAX_SEG * sizeof(double));
+  L.off_rows64 = off; off += align_up((size_t)L.M * sizeof(double));  // segmented search: fp64 row losses
   L.off_ext = off;    off += ext_bytes(d_in);  // per tensor: column extremes and candidate extremes
   if (L.form == AWQ_FORM_GRAM) {
     L.off_g = off;    off += align_up((size_t)d_in * d_in * 2);
@@ -314,7 +318,7 @@ awq_status run_gemm_pair(const void* A, long long M, long long lda, const void* 
   args.K = (int)K;
   args.n_blocks_m = (int)cdiv(M, PAIR_BM);
   args.n_blocks_n = (int)cdiv(Nr, PAIR_BN);
-  args.group_n = kGroupN < args.n_blocks_n ? kGroupN : args.n_blocks_n;
+  args.group_n = AWQ_PAIR_GROUP_N < args.n_blocks_n ? AWQ_PAIR_GROUP_N : args.n_blocks_n;
   args.tri = tri;
   // TRI_LOWER_STORE: the tiles of the lower block triangle (row block mb, column blocks 0 .. mb)
   const long long tiles = tri == TRI_LOWER_STORE ? (long long)args.n_blocks_m * (args.n_blocks_m + 1) / 2
@@ -614,11 +618,14 @@ awq_status awq_search_scales_segmented(const void* W, const void* X, const float
   if ((st = awq_step_gram(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
   if ((st = awq_step_contract(X, d_out, d_in, N, cfg, ws, ws_bytes, stream)) != AWQ_OK) return st;
   cudaStream_t s = as_stream(stream);
-  segment_loss_reduce<<<dim3(n_seg, L.n_alpha), REDUCE_THREADS, 0, s>>>(
-      at<float>(ws, L.off_part), L.n_blocks_n, L.M, (int)d_out, L.d_out_pad, seg, row_losses, at<double>(ws, L.off_seg));
+  row_loss_rows<<<dim3((unsigned)cdiv(d_out, REDUCE_THREADS), L.n_alpha), REDUCE_THREADS, 0, s>>>(
+      at<float>(ws, L.off_part), L.n_blocks_n, L.M, (int)d_out, L.d_out_pad, row_losses, at<double>(ws, L.off_rows64));
   if ((st = launch_status()) != AWQ_OK) return st;
-  segment_argmin<<<1, 32 * MAX_SEG, 0, s>>>(at<double>(ws, L.off_seg), n_seg, L.n_alpha, at<float>(ws, L.off_s),
-                                            (int)d_in, losses, best, s_best, at<int>(ws, 0));
+  segment_loss_reduce<<<dim3(n_seg, L.n_alpha), REDUCE_THREADS, 0, s>>>(at<double>(ws, L.off_rows64), L.M,
+                                                                        L.d_out_pad, seg, at<double>(ws, L.off_seg));
+  if ((st = launch_status()) != AWQ_OK) return st;
+  segment_argmin<<<n_seg, 256, 0, s>>>(at<double>(ws, L.off_seg), n_seg, L.n_alpha, at<float>(ws, L.off_s),
+                                       (int)d_in, losses, best, s_best, at<int>(ws, 0));
   return launch_status();
 }
 

@@ -358,28 +358,45 @@ __global__ void loss_argmin(const double* __restrict__ block_sums, int n_chunks,
 // each): fp64 loss per (segment, alpha) in a fixed order, then an argmin per
 // segment. part layout as for row_loss_reduce.
 // ---------------------------------------------------------------------------
+// a6 for several layers sharing X (the segmented search): per-row fp64 losses
+// (column tiles summed in order, one thread per row), then per segment and
+// alpha a fixed-order sum of its rows, then the argmin per segment. part
+// layout as for row_loss_reduce.
+// ---------------------------------------------------------------------------
 constexpr int MAX_SEG = 16;
 
 struct SegTable {
   int start[MAX_SEG + 1];  // segment s holds rows [start[s], start[s+1])
 };
 
-__global__ void __launch_bounds__(REDUCE_THREADS) segment_loss_reduce(const float* __restrict__ part, int n_blocks_n,
-                                                                      long long M, int d_out, int d_out_pad,
-                                                                      SegTable seg, float* __restrict__ row_losses,
+__global__ void __launch_bounds__(REDUCE_THREADS) row_loss_rows(const float* __restrict__ part, int n_blocks_n,
+                                                                long long M, int d_out, int d_out_pad,
+                                                                float* __restrict__ row_losses,
+                                                                double* __restrict__ rows64) {
+  const int k = blockIdx.y;
+  const int r = blockIdx.x * REDUCE_THREADS + threadIdx.x;
+  if (r >= d_out) return;
+  const long long m = (long long)k * d_out_pad + r;
+  double s = 0.0;
+  for (int nb = 0; nb < n_blocks_n; ++nb)
+    if (AWQ_IDX_OK((long long)nb * M + m, (long long)n_blocks_n * M, BS_LOSS_PART))
+      s += (double)part[(long long)nb * M + m];
+  if (row_losses && AWQ_IDX_OK((long long)k * d_out + r, (long long)gridDim.y * d_out, BS_LOSS_ROW))
+    row_losses[(long long)k * d_out + r] = (float)s;
+  if (AWQ_IDX_OK(m, M, BS_LOSS_PART)) rows64[m] = s;
+}
+
+// seg_sums[k][sg] = sum of the row losses of segment sg at alpha k (thread-
+// strided, then a fixed tree)
+__global__ void __launch_bounds__(REDUCE_THREADS) segment_loss_reduce(const double* __restrict__ rows64, long long M,
+                                                                      int d_out_pad, SegTable seg,
                                                                       double* __restrict__ seg_sums) {
   __shared__ double red[REDUCE_THREADS];
   const int sg = blockIdx.x, k = blockIdx.y;
   double acc = 0.0;
   for (int r = seg.start[sg] + threadIdx.x; r < seg.start[sg + 1]; r += REDUCE_THREADS) {
     const long long m = (long long)k * d_out_pad + r;
-    double s = 0.0;
-    for (int nb = 0; nb < n_blocks_n; ++nb)
-      if (AWQ_IDX_OK((long long)nb * M + m, (long long)n_blocks_n * M, BS_LOSS_PART))
-        s += (double)part[(long long)nb * M + m];
-    if (row_losses && AWQ_IDX_OK((long long)k * d_out + r, (long long)gridDim.y * d_out, BS_LOSS_ROW))
-      row_losses[(long long)k * d_out + r] = (float)s;
-    acc += s;
+    if (AWQ_IDX_OK(m, M, BS_LOSS_PART)) acc += rows64[m];
   }
   red[threadIdx.x] = acc;
   __syncthreads();
@@ -390,40 +407,47 @@ __global__ void __launch_bounds__(REDUCE_THREADS) segment_loss_reduce(const floa
   if (threadIdx.x == 0) seg_sums[(long long)k * MAX_SEG + sg] = red[0];
 }
 
-// One warp per segment: losses[sg][k], warp-shuffle argmin (lowest k on ties),
-// s_best[sg][:] = s(alpha_best).
-__global__ void segment_argmin(const double* __restrict__ seg_sums, int n_seg, int n_alpha,
-                               const float* __restrict__ s_all, int d_in, float* __restrict__ losses,
-                               int* __restrict__ best_out, float* __restrict__ s_best, int* err) {
-  const int sg = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// One block per segment: warp 0 takes losses[sg][k] and the warp-shuffle
+// argmin (lowest k on ties); the block copies s_best[sg][:] = s(alpha_best).
+__global__ void __launch_bounds__(256) segment_argmin(const double* __restrict__ seg_sums, int n_seg, int n_alpha,
+                                                      const float* __restrict__ s_all, int d_in,
+                                                      float* __restrict__ losses, int* __restrict__ best_out,
+                                                      float* __restrict__ s_best, int* err) {
+  __shared__ int b_shared;
+  const int sg = blockIdx.x, lane = threadIdx.x & 31;
   if (sg >= n_seg) return;
-  double bv = INFINITY;
-  int bi = MAX_ALPHA;
-  bool finite = true;
-  for (int k = lane; k < n_alpha; k += 32) {
-    const double v = seg_sums[(long long)k * MAX_SEG + sg];
-    losses[(long long)sg * n_alpha + k] = (float)v;
-    if (!isfinite(v)) finite = false;
-    if (v < bv) {
-      bv = v;
-      bi = k;
+  if (threadIdx.x < 32) {
+    double bv = INFINITY;
+    int bi = MAX_ALPHA;
+    bool finite = true;
+    for (int k = lane; k < n_alpha; k += 32) {
+      const double v = seg_sums[(long long)k * MAX_SEG + sg];
+      losses[(long long)sg * n_alpha + k] = (float)v;
+      if (!isfinite(v)) finite = false;
+      if (v < bv) {
+        bv = v;
+        bi = k;
+      }
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (ov < bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    finite = __all_sync(0xffffffffu, finite);
+    const int b = finite ? bi : -1;
+    if (lane == 0) {
+      best_out[sg] = b;
+      b_shared = b;
+      if (!finite && err) atomicCAS(err, 0, ERR_NONFINITE);
     }
   }
-  for (int off = 16; off > 0; off >>= 1) {
-    const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
-    const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-    if (ov < bv || (ov == bv && oi < bi)) {
-      bv = ov;
-      bi = oi;
-    }
-  }
-  finite = __all_sync(0xffffffffu, finite);
-  const int b = finite ? bi : -1;
-  if (lane == 0) {
-    best_out[sg] = b;
-    if (!finite && err) atomicCAS(err, 0, ERR_NONFINITE);
-  }
-  for (int i = lane; i < d_in; i += 32)
+  __syncthreads();
+  const int b = b_shared;
+  for (int i = threadIdx.x; i < d_in; i += blockDim.x)
     s_best[(long long)sg * d_in + i] =
         (b >= 0 && AWQ_IDX_OK((long long)b * d_in + i, (long long)n_alpha * d_in, BS_ARGMIN_S))
             ? s_all[(long long)b * d_in + i]
