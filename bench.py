@@ -149,7 +149,7 @@ def workload_config(wl, world):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("gemm_pair_sm100.cuh", "gemm_sm100.cuh", "ptx.cuh"):
+    for f in ("gemm_pair_sm100.cuh", "gemm_sm100.cuh", "ptx.cuh", "awq_api.cu"):  # kernels and their launch
         with open(os.path.join(ROOT, "weight_only_int4_act_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -64,7 +64,7 @@ def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
     (prof / "contract_pair_gram_CY.md").write_text("- source_sha256: `0000`\n- traffic_bytes_per_launch: `456`\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     (tmp_path / "weight_only_int4_act_b200" / "csrc").mkdir(parents=True)
-    for f in ("gemm_pair_sm100.cuh", "gemm_sm100.cuh", "ptx.cuh"):
+    for f in ("gemm_pair_sm100.cuh", "gemm_sm100.cuh", "ptx.cuh", "awq_api.cu"):
         src = os.path.join(ROOT, "weight_only_int4_act_b200", "csrc", f)
         (tmp_path / "weight_only_int4_act_b200" / "csrc" / f).write_bytes(open(src, "rb").read())
     assert bench.profiled_traffic("CX", "gram") == 123.0
