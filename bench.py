@@ -782,7 +782,7 @@ def run_only(args):
         fn = lambda: awq.w4a16_gemm(Xp, *pk, cfg, ws=wsw, out=Y)  # noqa: E731
         byts = d_out * d_in // 2 + 4 * d_out * ng + tokens * (d_in + d_out) * 2
         flops = 2.0 * tokens * d_out * d_in
-        kernels = ["w4a16_gemm_tcgen05", "w4a16_split_reduce"]
+        kernels = ["w4a16_gemm_tcgen05", "w4a16_streamk_reduce"]
         note = f"{tokens} tokens, {args.dtype} activations, W packed at s = 1"
     else:
         raise SystemExit(f"unknown --only {what}")

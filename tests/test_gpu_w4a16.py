@@ -45,6 +45,11 @@ CASES = [
     ("g8", 64, 128, 512, 4, 8, False),
     ("g16_2bit_sym", 130, 256, 1024, 2, 16, True),
     ("prefill_4096", 4096, 4096, 4096, 4, 128, False),   # no split, 512 tiles
+    ("decode_17_odd_steps", 17, 384, 1216, 4, 64, False),  # last unit of 3 K steps: a half pair
+    ("decode_33", 33, 256, 2048, 4, 128, False),         # 64-row token boxes
+    ("decode_long_k", 8, 128, 16384, 4, 128, False),     # one tile split over many CTAs
+    ("decode_whole_tiles", 64, 1024, 2048, 4, 128, False),
+    ("decode_g16", 24, 256, 1024, 4, 16, False),
 ]
 
 
@@ -90,7 +95,8 @@ def test_w4a16_against_oracle(name, N, d_out, d_in, bits, group, symmetric, dtyp
 
 
 def test_w4a16_deterministic_and_workspace_error_clear():
-    N, d_out, d_in = 16, 512, 1024
+    # 2 tiles of 32 K steps on 16 CTAs: every tile summed from 8 partial slabs
+    N, d_out, d_in = 16, 256, 8192
     Wb, _, Xp, s32 = _scaled_layer(N, d_out, d_in, 4, 128, False, seed=11)
     qw, sc, zr, _, _, _ = O.pack(Wb, s32.astype(np.float64), 4, 128, False)
     cfg = awq.make_cfg(4, 128, False, 1)
@@ -102,6 +108,7 @@ def test_w4a16_deterministic_and_workspace_error_clear():
     torch.cuda.synchronize()
     awq.workspace_error(ws)
     assert torch.equal(a, b)
+    _check_product(a, Xp, qw, sc, zr, 128)
 
 
 def test_pack_then_product_on_the_gpu():

@@ -982,12 +982,28 @@ namespace {
 constexpr int kW4TargetCtas = 148;  // split K until the tiles cover this many CTAs
 
 struct W4Plan {
-  int bn, bk, n_mb, n_nb, n_kb, splits, kb_per_split;
+  int bn, bk, n_mb, n_nb, n_kb;
   int as, xs, rs;  // ring depths
-  long long tiles, p_stride;
+  bool sk;         // stream-K ranges (few tiles) or whole tiles
+  int grid, slots;
+  long long tiles, units, p_stride;
   int smem;
   size_t ws;
 };
+static_assert(kW4TargetCtas - 1 <= W4_MAX_FIX, "split tiles per launch");
+
+// The tiles of a stream-K plan that two or more ranges touch (each found at
+// its first inner range boundary), with their slab counts.
+void w4_fixups(const W4Plan& p, W4Fixups& fx) {
+  fx.n = 0;
+  for (long long c = 1; c < p.grid; ++c) {
+    const long long b = w4_sk_begin(c, p.grid, p.units), tile = b / p.n_kb, t0 = tile * p.n_kb;
+    if (b == t0 || w4_sk_cta(t0, p.grid, p.units) != c - 1) continue;
+    fx.tile[fx.n] = (int)tile;
+    fx.ns[fx.n] = (int)(w4_sk_cta(t0 + p.n_kb - 1, p.grid, p.units) - (c - 1) + 1);
+    ++fx.n;
+  }
+}
 
 W4Plan w4_plan(int64_t N, int64_t d_out, int64_t d_in, int group) {
   W4Plan p{};
@@ -1008,18 +1024,27 @@ W4Plan w4_plan(int64_t N, int64_t d_out, int64_t d_in, int group) {
   p.n_mb = (int)cdiv(d_out, W4_BM);
   p.n_nb = (int)cdiv(N, p.bn);
   p.n_kb = (int)cdiv(d_in, p.bk);
-  const long long mn = (long long)p.n_mb * p.n_nb;
-  int splits = 1;
-  if (mn < kW4TargetCtas) {
-    const long long want = cdiv(kW4TargetCtas, mn);
-    const int most = p.n_kb / 4 > 1 ? p.n_kb / 4 : 1;  // at least 4 K steps per split
-    splits = (int)(want < most ? want : most);
+  p.tiles = (long long)p.n_mb * p.n_nb;
+  p.units = p.tiles * p.n_kb;
+  // Fewer than two waves of whole tiles: stream-K over equal ranges of
+  // (tile, K step) units, at least 4 K steps per CTA (the rings' fill and
+  // drain is paid per CTA). The grid is fixed by the shapes alone, so that
+  // the workspace can be sized without a device.
+  p.sk = p.tiles < 2 * kW4TargetCtas && p.n_kb > 1;
+  if (p.sk) {
+    const long long g = p.units / 4 < kW4TargetCtas ? p.units / 4 : kW4TargetCtas;
+    p.grid = (int)(g > 1 ? g : 1);
+    p.slots = 1;
+    for (long long t = 0; t < p.tiles; ++t) {
+      const long long n = w4_sk_cta(t * p.n_kb + p.n_kb - 1, p.grid, p.units) - w4_sk_cta(t * p.n_kb, p.grid, p.units) + 1;
+      if (n > p.slots) p.slots = (int)n;
+    }
+  } else {
+    p.grid = (int)(p.tiles < kW4TargetCtas ? p.tiles : kW4TargetCtas);
+    p.slots = 1;
   }
-  p.kb_per_split = (int)cdiv(p.n_kb, splits);
-  p.splits = (int)cdiv(p.n_kb, p.kb_per_split);
-  p.tiles = mn * p.splits;
   p.p_stride = (N * d_out + 3) / 4 * 4;
-  p.ws = kAlign + (p.splits > 1 ? align_up((size_t)p.splits * p.p_stride * sizeof(float)) : 0);
+  p.ws = kAlign + (p.slots > 1 ? align_up((size_t)p.slots * p.p_stride * sizeof(float)) : 0);
   return p;
 }
 
@@ -1070,10 +1095,10 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, awq_dtype dtype, const uint3
   a.bn = p.bn;
   a.n_mb = p.n_mb;
   a.n_nb = p.n_nb;
-  a.splits = p.splits;
-  a.kb_per_split = p.kb_per_split;
+  a.sk = p.sk ? 1 : 0;
   a.n_kb = p.n_kb;
   a.num_tiles = (int)p.tiles;
+  a.units = p.units;
   a.ng = (int)(d_in / cfg->group);
   int sh = 0;
   while ((1 << sh) < cfg->group) ++sh;
@@ -1085,11 +1110,11 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, awq_dtype dtype, const uint3
   a.scales = static_cast<const __half*>(scales);
   a.zeros = static_cast<const __half*>(zeros);
   a.Y = Y;
-  a.P = p.splits > 1 ? at<float>(ws, kAlign) : nullptr;
+  a.P = p.slots > 1 ? at<float>(ws, kAlign) : nullptr;
   a.p_stride = p.p_stride;
   a.err = at<int>(ws, 0);
   if (cudaMemsetAsync(ws, 0, sizeof(int), cs) != cudaSuccess) return AWQ_ERR_CUDA;
-  const int grid = (int)(p.tiles < sms ? p.tiles : sms);
+  const int grid = p.grid;
   auto launch = [&](auto kernel) -> awq_status {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem) != cudaSuccess)
       return AWQ_ERR_CUDA;
@@ -1119,18 +1144,17 @@ extern "C" awq_status awq_w4a16_gemm(const void* X, awq_dtype dtype, const uint3
     st = p.bk == 256 ? dispatch(T{}, K256{}) : dispatch(T{}, K128{});
   else
     st = p.bk == 256 ? dispatch(Fa{}, K256{}) : dispatch(Fa{}, K128{});
-  if (st != AWQ_OK) return st;
-  if (p.splits > 1) {
-    const long long n = N * d_out;
-    const long long blocks = cdiv(n / 4 > 0 ? n / 4 : 1, 256);
-    const unsigned rgrid = (unsigned)(blocks < 4 * sms ? blocks : 4 * sms);
-    if (f16)
-      w4a16_split_reduce<true><<<rgrid, 256, 0, cs>>>(a.P, p.splits, n, p.p_stride, Y);
-    else
-      w4a16_split_reduce<false><<<rgrid, 256, 0, cs>>>(a.P, p.splits, n, p.p_stride, Y);
-    return launch_status();
-  }
-  return AWQ_OK;
+  if (st != AWQ_OK || p.slots == 1) return st;
+  W4Fixups fx;
+  w4_fixups(p, fx);
+  if (fx.n == 0) return AWQ_OK;
+  const dim3 rgrid((unsigned)fx.n, (unsigned)cdiv((long long)W4_BM * p.bn, 1024));
+  if (f16)
+    w4a16_streamk_reduce<true><<<rgrid, 256, 0, cs>>>(a.P, p.p_stride, p.slots, (int)N, (int)d_out, p.bn, p.n_mb, fx, Y);
+  else
+    w4a16_streamk_reduce<false><<<rgrid, 256, 0, cs>>>(a.P, p.p_stride, p.slots, (int)N, (int)d_out, p.bn, p.n_mb, fx,
+                                                       Y);
+  return launch_status();
 }
 
 extern "C" awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p, awq_dtype dtype, int64_t inner,

@@ -44,9 +44,8 @@ enum BoundsSite : int {
   BS_PACK_SZ,       // quantize_pack: scales / zeros
   BS_W4_PARAMS,     // w4a16_gemm_tcgen05: step / zero loads
   BS_W4_Y,          // w4a16_gemm_tcgen05: Y stores
-  BS_W4_P,          // w4a16_gemm_tcgen05: split-K partial stores
-  BS_SPLIT_P,       // w4a16_split_reduce: partials
-  BS_SPLIT_Y,       // w4a16_split_reduce: Y
+  BS_W4_P,          // w4a16_gemm_tcgen05: stream-K partial stores
+  BS_W4_FIXUP,      // w4a16_streamk_reduce: split tiles, partials and Y
   BS_FOLD_S,        // fold_inv_scales_kernel: s
   BS_FOLD_P,        // fold_inv_scales_kernel: the folded tensor
   BS_SELFTEST = 0x7F,

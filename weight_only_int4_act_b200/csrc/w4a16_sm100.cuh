@@ -41,8 +41,17 @@
 // The MMA issuer is the critical path: every other role waits with a short
 // sleep between polls, so that waiting warps leave the issue slots of their
 // scheduler (which the issuer shares with two dequantising warps) free.
-// K may be split across CTAs when there are fewer tiles than SMs; the
-// partials are then summed in split order by a second kernel.
+// Work split: with many tiles, CTA c takes whole tiles c, c + G, ... (G
+// CTAs). With few (decode widths, where 224 tiles on 148 SMs would leave a
+// tail of half the CTAs idle), a static "stream-K" split: the (tile, K step)
+// units, tile-major, are cut into G contiguous ranges of equal length and
+// CTA c takes range c, cut at tile boundaries into segments. A tile that two
+// or more CTAs touch is written by each as fp32 partials, CTA c into slab
+// (c - first CTA of the tile), and w4a16_streamk_reduce adds the slabs in
+// slab order. The split depends only on the shapes, so the result is
+// deterministic. (Finishing a tile inside the kernel, by whichever CTA takes
+// the last ticket of an atomic counter, measured slower: the fix-up lands on
+// the critical path of the last CTAs.)
 // Every wait is bounded; on a timeout the CTA records an error in *err,
 // drains its in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
@@ -141,27 +150,72 @@ struct W4Args {
   int N, d_out, d_in;
   int bn;            // tokens per tile
   int n_mb, n_nb;    // ceil(d_out / 128), ceil(N / bn)
-  int splits;        // K splits (1: no split)
-  int kb_per_split;  // K steps per split
-  int n_kb;          // ceil(d_in / 64)
-  int num_tiles;     // n_mb * n_nb * splits
+  int sk;            // 1: stream-K ranges of units, 0: whole tiles
+  int n_kb;          // K steps per tile, ceil(d_in / BK)
+  int num_tiles;     // n_mb * n_nb
+  long long units;   // num_tiles * n_kb (stream-K)
   int ng;            // groups per row (d_in / group)
   int group_shift;   // log2(group)
   int as, xs, rs;    // ring depths: dequantised weights, activations, packed codes
   const __half* scales;  // [d_out, ng]
   const __half* zeros;   // [d_out, ng]
-  void* Y;               // [N, d_out] in the activation type (splits == 1)
-  float* P;              // [splits][p_stride] with [N, d_out] in each slab (splits > 1)
+  void* Y;               // [N, d_out] in the activation type
+  float* P;              // [slots][p_stride]: [N, d_out] fp32 partials in each slab (stream-K)
   long long p_stride;    // N * d_out rounded up to a multiple of 4
   int* err;
 };
 
-__device__ __forceinline__ void w4_tile_coords(int t, const W4Args& a, int& mb, int& nb, int& split) {
-  mb = t % a.n_mb;
-  const int rest = t / a.n_mb;
-  nb = rest % a.n_nb;
-  split = rest / a.n_nb;
-}
+// First unit of stream-K range c of G over U units, and the range that holds unit u.
+__host__ __device__ inline long long w4_sk_begin(long long c, long long G, long long U) { return c * U / G; }
+__host__ __device__ inline long long w4_sk_cta(long long u, long long G, long long U) { return ((u + 1) * G - 1) / U; }
+
+// One segment of a CTA's work: output tile (mb, nb), K steps [kb0, kb1);
+// whole: no other CTA touches the tile (written to Y), else written to
+// partial slab `slot`.
+struct W4Seg {
+  int mb, nb, kb0, kb1, slot, ns;  // ns: CTAs that touch the tile
+  bool whole;
+};
+
+// The segments of this CTA, in order; every role walks the same sequence.
+struct W4Sched {
+  long long u, u1;
+  __device__ explicit W4Sched(const W4Args& a) {
+    if (a.sk) {
+      u = w4_sk_begin(blockIdx.x, gridDim.x, a.units);
+      u1 = w4_sk_begin(blockIdx.x + 1, gridDim.x, a.units);
+    } else {
+      u = blockIdx.x;
+      u1 = a.num_tiles;
+    }
+  }
+  __device__ bool next(const W4Args& a, W4Seg& g) {
+    if (u >= u1) return false;
+    long long tile;
+    if (a.sk) {
+      tile = u / a.n_kb;
+      const long long t0 = tile * a.n_kb;
+      g.kb0 = (int)(u - t0);
+      g.kb1 = (int)min((long long)a.n_kb, (long long)g.kb0 + (u1 - u));
+      const long long first = w4_sk_cta(t0, gridDim.x, a.units);
+      g.ns = (int)(w4_sk_cta(t0 + a.n_kb - 1, gridDim.x, a.units) - first + 1);
+      g.whole = g.ns == 1;
+      g.slot = (int)(blockIdx.x - first);
+      u += g.kb1 - g.kb0;
+    } else {
+      tile = u;
+      g.kb0 = 0;
+      g.kb1 = a.n_kb;
+      g.whole = true;
+      g.slot = 0;
+      g.ns = 1;
+      u += gridDim.x;
+    }
+    g.mb = (int)(tile % a.n_mb);
+    g.nb = (int)(tile / a.n_mb);
+    return true;
+  }
+};
 
 __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -318,11 +372,10 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       Ring ring;
       uint32_t issued = 0, last_parity = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
-        int mb, nb, split;
-        w4_tile_coords(t, args, mb, nb, split);
-        const int kb0 = split * args.kb_per_split;
-        const int kb1 = min(args.n_kb, kb0 + args.kb_per_split);
+      W4Sched sched(args);
+      W4Seg g;
+      while (ok && sched.next(args, g)) {
+        const int mb = g.mb, nb = g.nb, kb0 = g.kb0, kb1 = g.kb1;
         for (int kb = kb0; kb < kb1; kb += codes ? St::RK : 1) {
           const uint32_t full = codes ? rfull(ring.stage) : xfull(ring.stage);
           const uint32_t empty = codes ? rempty(ring.stage) : xempty(ring.stage);
@@ -362,11 +415,10 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       Ring xr, ar;
       bool ok = true;
       int local = 0;
-      for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x, ++local) {
-        int mb, nb, split;
-        w4_tile_coords(t, args, mb, nb, split);
-        const int kb0 = split * args.kb_per_split;
-        const int kb1 = min(args.n_kb, kb0 + args.kb_per_split);
+      W4Sched sched(args);
+      W4Seg g;
+      for (; ok && sched.next(args, g); ++local) {
+        const int kb0 = g.kb0, kb1 = g.kb1;
         const int acc = local % nacc;
         const uint32_t use = (uint32_t)(local / nacc);
         if (!mbar_wait(tempty(acc), (use & 1u) ^ 1u, abort_flag, args.err, ERR_W4_TEMPTY)) break;
@@ -407,12 +459,11 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     const int sw = r & 7;
     Ring rr, ar;
     bool ok = true;
-    for (int t = blockIdx.x; ok && t < args.num_tiles; t += gridDim.x) {
-      int mb, nb, split;
-      w4_tile_coords(t, args, mb, nb, split);
-      const int kb0 = split * args.kb_per_split;
-      const int kb1 = min(args.n_kb, kb0 + args.kb_per_split);
-      const int row = mb * W4_BM + r;
+    W4Sched sched(args);
+    W4Seg g;
+    while (ok && sched.next(args, g)) {
+      const int kb0 = g.kb0, kb1 = g.kb1;
+      const int row = g.mb * W4_BM + r;
       const bool valid = row < args.d_out;
       const __half* srow = args.scales + (long long)(valid ? row : 0) * args.ng;
       const __half* zrow = args.zeros + (long long)(valid ? row : 0) * args.ng;
@@ -506,9 +557,10 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     int local = 0;
-    for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x, ++local) {
-      int mb, nb, split;
-      w4_tile_coords(t, args, mb, nb, split);
+    W4Sched sched(args);
+    W4Seg g;
+    for (; sched.next(args, g); ++local) {
+      const int mb = g.mb, nb = g.nb;
       const int acc = local % nacc;
       const uint32_t use = (uint32_t)(local / nacc);
       // the accumulator takes a whole tile: wait without spinning
@@ -526,18 +578,17 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         const int jn = min(32, min(bn - c * 32, args.N - (t0 + c * 32)));
         if (o < args.d_out) {
           const long long e0 = (long long)(t0 + c * 32) * args.d_out + o;
-          if (args.splits == 1) {
+          if (g.whole) {
             typename W4Type<F16>::T* y = static_cast<typename W4Type<F16>::T*>(args.Y) + e0;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (j < jn && AWQ_IDX_OK(e0 + (long long)j * args.d_out, (long long)args.N * args.d_out, BS_W4_Y))
                 y[(long long)j * args.d_out] = W4Type<F16>::from_float(__uint_as_float(v[j]));
           } else {
-            float* P = args.P + (long long)split * args.p_stride + e0;
+            float* P = args.P + (long long)g.slot * args.p_stride + e0;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (j < jn && AWQ_IDX_OK(e0 + (long long)j * args.d_out, (long long)args.N * args.d_out, BS_W4_P) &&
-                  AWQ_IDX_OK(split, args.splits, BS_W4_P))
+              if (j < jn && AWQ_IDX_OK(e0 + (long long)j * args.d_out, (long long)args.N * args.d_out, BS_W4_P))
                 P[(long long)j * args.d_out] = __uint_as_float(v[j]);
           }
         }
@@ -556,34 +607,48 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   }
 }
 
-// Y = sum over splits of P[split] in split order, rounded to the activation
-// type; 4 outputs per thread. Slabs are `stride` floats apart (a multiple of
-// 4, so every float4 is aligned).
+// Tiles that two or more CTAs touch, found on the host from the shapes: tile
+// index and the number of partial slabs.
+constexpr int W4_MAX_FIX = 160;
+struct W4Fixups {
+  int n;
+  int tile[W4_MAX_FIX];
+  int ns[W4_MAX_FIX];
+};
+
+// Stream-K fix-up: block (b, y) sums the partial slabs of split tile
+// fx.tile[b] in slab order for 1024 of its elements (token-major, output
+// channel fastest; 4 per thread, 256 apart, so that each load instruction is
+// coalesced) and writes them rounded to the activation type.
 template <bool F16>
-__global__ void w4a16_split_reduce(const float* __restrict__ P, int splits, long long n, long long stride,
-                                   void* __restrict__ Yv) {
+__global__ void w4a16_streamk_reduce(const float* __restrict__ P, long long p_stride, int slots, int N, int d_out,
+                                     int bn, int n_mb, const __grid_constant__ W4Fixups fx, void* __restrict__ Yv) {
   using T = typename W4Type<F16>::T;
   T* Y = static_cast<T*>(Yv);
-  const long long n4 = n >> 2;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
-    if (!AWQ_SPAN_OK(4 * i, 4, n, BS_SPLIT_Y) || !AWQ_SPAN_OK(4 * i, 4, stride, BS_SPLIT_P)) continue;
-    float4 acc = reinterpret_cast<const float4*>(P)[i];
-    for (int s = 1; s < splits; ++s) {
-      const float4 p = reinterpret_cast<const float4*>(P + (long long)s * stride)[i];
-      acc.x += p.x;
-      acc.y += p.y;
-      acc.z += p.z;
-      acc.w += p.w;
-    }
-    reinterpret_cast<uint2*>(Y)[i] = make_uint2(pack2<F16>(acc.x, acc.y), pack2<F16>(acc.z, acc.w));
+  if (!AWQ_IDX_OK(blockIdx.x, fx.n, BS_W4_FIXUP)) return;
+  const int tile = fx.tile[blockIdx.x], ns = min(fx.ns[blockIdx.x], slots);
+  const int o0 = (tile % n_mb) * W4_BM, tok0 = (tile / n_mb) * bn;
+  const int rows = min(W4_BM, d_out - o0), toks = min(bn, N - tok0);
+  long long idx[4];
+  bool in[4];
+  float acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int e = blockIdx.y * 1024 + k * 256 + threadIdx.x;
+    const int j = e / rows, r = e - j * rows;
+    idx[k] = (long long)(tok0 + j) * d_out + o0 + r;
+    in[k] = e < rows * toks && AWQ_IDX_OK(idx[k], (long long)N * d_out, BS_W4_FIXUP);
+    acc[k] = 0.0f;
   }
-  // tail (n not a multiple of 4)
-  const long long i = (n4 << 2) + (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (blockIdx.x == 0 && i < n && AWQ_IDX_OK(i, stride, BS_SPLIT_P)) {
-    float acc = P[i];
-    for (int s = 1; s < splits; ++s) acc += P[(long long)s * stride + i];
-    Y[i] = W4Type<F16>::from_float(acc);
+  for (int sl = 0; sl < ns; ++sl) {
+    const float* Ps = P + (long long)sl * p_stride;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (in[k]) acc[k] += Ps[idx[k]];
   }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (in[k]) Y[idx[k]] = W4Type<F16>::from_float(acc[k]);
 }
 
 // Fold S^-1 into the producer of X: row i of p [d_in, inner] (bf16 or fp16)
