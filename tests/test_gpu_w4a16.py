@@ -45,6 +45,7 @@ CASES = [
     ("g8", 64, 128, 512, 4, 8, False),
     ("g16_2bit_sym", 130, 256, 1024, 2, 16, True),
     ("prefill_4096", 4096, 4096, 4096, 4, 128, False),   # no split, 512 tiles
+    ("prefill_ragged", 777, 640, 1152, 4, 128, False),   # ragged rows and tokens, an odd number of K steps
     ("decode_17_odd_steps", 17, 384, 1216, 4, 64, False),  # last unit of 3 K steps: a half pair
     ("decode_33", 33, 256, 2048, 4, 128, False),         # 64-row token boxes
     ("decode_long_k", 8, 128, 16384, 4, 128, False),     # one tile split over many CTAs
