@@ -395,7 +395,8 @@ awq_status awq_act_stats(const void* X, int64_t N, int64_t d_in, float* a, void*
   act_absmean_partial<<<grid, STATS_THREADS, 0, s>>>(static_cast<const __nv_bfloat16*>(X), N, (int)d_in,
                                                      L.rows_per_chunk, at<double>(ws, L.off_part));
   if ((st = launch_status()) != AWQ_OK) return st;
-  act_absmean_final<<<(unsigned)cdiv(d_in, 256), 256, 0, s>>>(at<double>(ws, L.off_part), L.n_chunks, N, (int)d_in, a);
+  act_absmean_final<<<(unsigned)cdiv(d_in, FINAL_COLS), STATS_FINAL_THREADS, 0, s>>>(at<double>(ws, L.off_part),
+                                                                                   L.n_chunks, N, (int)d_in, a);
   return launch_status();
 }
 
@@ -973,7 +974,7 @@ extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t d_
   act_absmean_partial<<<dim3(L.col_blocks, L.n_chunks), STATS_THREADS, 0, s>>>(
       static_cast<const __nv_bfloat16*>(X), N, (int)d_in, L.rows_per_chunk, part);
   if ((st = launch_status()) != AWQ_OK) return st;
-  act_absmean_final<<<(unsigned)cdiv(d_in, 256), 256, 0, s>>>(part, L.n_chunks, N, (int)d_in, a);
+  act_absmean_final<<<(unsigned)cdiv(d_in, FINAL_COLS), STATS_FINAL_THREADS, 0, s>>>(part, L.n_chunks, N, (int)d_in, a);
   return launch_status();
 }
 

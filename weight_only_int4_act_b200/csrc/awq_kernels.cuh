@@ -38,6 +38,7 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4 u, float (&f)[8]) {
 // ---------------------------------------------------------------------------
 constexpr int STATS_THREADS = 256;
 constexpr int STATS_COLS = 256;
+constexpr int STATS_FINAL_THREADS = 256;
 constexpr int STATS_UNROLL = 8;  // rows summed in fp32 (and loads in flight) per thread and step
 
 __global__ void __launch_bounds__(STATS_THREADS) act_absmean_partial(const __nv_bfloat16* __restrict__ X, long long N,
@@ -85,13 +86,30 @@ __global__ void __launch_bounds__(STATS_THREADS) act_absmean_partial(const __nv_
   }
 }
 
-__global__ void act_absmean_final(const double* __restrict__ part, int n_chunks, long long N, int d_in,
-                                  float* __restrict__ a) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= d_in) return;
+// a_i = (sum over row chunks of the partials) / N. A block takes 32 channels;
+// its 8 warps each sum every 8th chunk (chunk order within a warp), and the 8
+// sums are added in warp order: a fixed tree, so the result depends only on
+// the shapes, with 8 times fewer dependent loads per thread than one serial
+// sum per channel.
+constexpr int FINAL_COLS = 32, FINAL_SLICES = STATS_FINAL_THREADS / 32;
+__global__ void __launch_bounds__(STATS_FINAL_THREADS) act_absmean_final(const double* __restrict__ part, int n_chunks,
+                                                                         long long N, int d_in, float* __restrict__ a) {
+  __shared__ double red[FINAL_SLICES][FINAL_COLS];
+  const int cl = threadIdx.x & 31, sl = threadIdx.x >> 5;
+  const int c = blockIdx.x * FINAL_COLS + cl;
   double t = 0.0;
-  for (int k = 0; k < n_chunks; ++k) t += part[(long long)k * d_in + c];
-  a[c] = (float)(t / (double)N);
+  if (c < d_in)
+    for (int k = sl; k < n_chunks; k += FINAL_SLICES)
+      if (AWQ_IDX_OK((long long)k * d_in + c, (long long)n_chunks * d_in, BS_STATS_PART))
+        t += part[(long long)k * d_in + c];
+  red[sl][cl] = t;
+  __syncthreads();
+  if (sl == 0 && c < d_in) {
+    double u = red[0][cl];
+#pragma unroll
+    for (int j = 1; j < FINAL_SLICES; ++j) u += red[j][cl];
+    a[c] = (float)(u / (double)N);
+  }
 }
 
 // ---------------------------------------------------------------------------
