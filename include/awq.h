@@ -288,8 +288,9 @@ awq_status awq_fold_inv_scales(const float* s, int64_t d_in, void* p, awq_dtype 
  * and of g (AWQ_ERR_SHAPE). cfg->group must be a group size (8 ... 256): the
  * per-tensor layout (group 0, one step for the layer) is not read by this
  * kernel and gives AWQ_ERR_INVALID_ARG.
- * Workspace: awq_w4a16_workspace_size (error word, split-K partials when
- * there are fewer output tiles than SMs); AWQ_ERR_WORKSPACE if smaller.
+ * Workspace: awq_w4a16_workspace_size (error word, and fp32 partials of the
+ * tiles that are split between CTAs when there are fewer than two waves of
+ * output tiles); AWQ_ERR_WORKSPACE if smaller.
  * Asynchronous; device-side errors land in the workspace (awq_workspace_error). */
 size_t awq_w4a16_workspace_size(int64_t N, int64_t d_out, int64_t d_in, const awq_qcfg* cfg);
 awq_status awq_w4a16_gemm(const void* X, awq_dtype dtype, const uint32_t* qweight, const void* scales_f16,

@@ -248,3 +248,69 @@ def test_per_tensor_validation():
                                            FAKE, big, FAKE, FAKE, FAKE, None, None) == 7
     assert awq.group_clip_workspace_size(256, 512, 256, cfg) == 0
     assert awq.w4a16_workspace_size(16, 256, 512, cfg) == 0
+
+
+# ---------------------------------------------------------------- W4A16 work split (host plan)
+def _w4_split(N, d_out, d_in, group, ctas=148):
+    """The W4A16 plan's work split, restated: 128-row tiles of bn tokens,
+    K steps of 256 channels at decode widths (bn <= 64, g > 8) else 128;
+    with fewer than two waves of tiles, G = min(ctas, units // 4) equal
+    ranges of the tile-major (tile, K step) units. Returns (segments per
+    CTA, slots, G): a segment is (tile, k0, k1, slab, whole)."""
+    bn = next(b for b in (16, 32, 64, 128, 256) if N <= b) if N <= 256 else 256
+    bk = 256 if bn <= 64 and group > 8 else 128
+    tiles = -(-d_out // 128) * -(-N // bn)
+    n_kb = -(-d_in // bk)
+    units = tiles * n_kb
+    if not (tiles < 2 * ctas and n_kb > 1):
+        return None, 1, min(tiles, ctas)
+    G = max(1, min(units // 4, ctas))
+    begin = lambda c: c * units // G  # noqa: E731
+    cta = lambda u: ((u + 1) * G - 1) // units  # noqa: E731
+    segs = []
+    for c in range(G):
+        u, u1, mine = begin(c), begin(c + 1), []
+        while u < u1:
+            t = u // n_kb
+            k0 = u - t * n_kb
+            k1 = min(n_kb, k0 + (u1 - u))
+            first, last = cta(t * n_kb), cta(t * n_kb + n_kb - 1)
+            mine.append((t, k0, k1, c - first, first == last))
+            u += k1 - k0
+        segs.append(mine)
+    slots = max(cta(t * n_kb + n_kb - 1) - cta(t * n_kb) + 1 for t in range(tiles))
+    return segs, slots, G
+
+
+@pytest.mark.parametrize("shape", [(16, 28672, 8192, 128), (64, 28672, 8192, 128), (16, 4096, 4096, 128),
+                                   (1, 256, 4096, 128), (8, 128, 16384, 128), (37, 200, 352, 32),
+                                   (17, 384, 1216, 64), (256, 4096, 4096, 128), (4096, 4096, 4096, 128),
+                                   (16, 512, 1024, 128), (64, 128, 512, 8)])
+def test_w4a16_stream_k_split(shape):
+    """Every (tile, K step) unit is taken exactly once, a tile that one CTA
+    covers is written whole, a split tile's CTAs fill slabs 0 .. n-1, and the
+    library's workspace holds exactly the error word plus those slabs."""
+    N, d_out, d_in, g = shape
+    cfg = awq.make_cfg(4, g, False, 1)
+    segs, slots, G = _w4_split(N, d_out, d_in, g)
+    p_stride = (N * d_out + 3) // 4 * 4
+    want = 1024 + ((slots * p_stride * 4 + 1023) // 1024 * 1024 if slots > 1 else 0)
+    assert awq.w4a16_workspace_size(N, d_out, d_in, cfg) == want
+    if segs is None:
+        return
+    seen, slabs = {}, {}
+    for c, mine in enumerate(segs):
+        for t, k0, k1, slab, whole in mine:
+            assert 0 <= slab < slots and k0 < k1
+            if whole:
+                assert slab == 0
+            for k in range(k0, k1):
+                assert (t, k) not in seen
+                seen[(t, k)] = whole
+            slabs.setdefault(t, set()).add(slab)
+    n_kb = max(k for _, k in seen) + 1
+    assert len(seen) == len({t for t, _ in seen}) * n_kb
+    for t, s in slabs.items():
+        assert s == set(range(len(s)))
+    if shape == (16, 28672, 8192, 128):
+        assert (G, slots) == (148, 2)  # 224 tiles x 32 steps: 48 or 49 steps per CTA

@@ -1,6 +1,6 @@
 // Debug build (-DAWQ_BOUNDS_CHECK): explicit index checks on the global loads
 // and stores that the kernels address by hand (the SIMT kernels, the W4A16
-// kernel's step / zero loads and output stores, the split-K reduce and the
+// kernel's step / zero loads and output stores, the stream-K fix-up and the
 // fold). A check compares the span an access touches with the extent that the
 // kernel's own arguments give the buffer. When it fails, the access is skipped
 // (a load yields zero) and ERR_BOUNDS | site goes to the device word

@@ -36,7 +36,7 @@
 //                each step's channels, two codes per packed subtract and
 //                multiply (dequant_word), 32 columns per tcgen05.st;
 //   warps 11..14 epilogue: tcgen05.ld of the accumulator (TMEM lane = output
-//                channel, column = token), stores of Y (or fp32 split-K
+//                channel, column = token), stores of Y (or the fp32
 //                partials), then release of the accumulator.
 // The MMA issuer is the critical path: every other role waits with a short
 // sleep between polls, so that waiting warps leave the issue slots of their
