@@ -824,6 +824,18 @@ def run_only(args):
 
 # ----------------------------------------------------------------------------- CPU oracle
 ORACLE_ROW_COST_S = 7e-10  # single-thread oracle seconds per row per (d_in * N), 20 alphas (measured)
+REF_STEP_S = 1.2  # oracle arm: single-thread seconds of work per step (100 + 10 steps in about 2-3 minutes)
+
+
+def ref_sample(wl, seconds):
+    """Rows and search tokens of the oracle arm's step: the rows of
+    sample_rows; where the minimum of 8 rows over all tokens would still take
+    longer than ``seconds``, the search runs over a token slice (a multiple of
+    1024) sized to it."""
+    rows = sample_rows(wl, seconds)
+    per_token = ORACLE_ROW_COST_S * wl.d_in * rows
+    tokens = int(min(wl.N, max(1024, seconds / per_token)))
+    return rows, (tokens // 1024 * 1024 if tokens < wl.N else wl.N)
 
 
 def sample_rows(wl, seconds):
@@ -834,31 +846,37 @@ def sample_rows(wl, seconds):
     return int(min(wl.d_out, max(8, rows)))
 
 
-def oracle_sample(wl, Wb, Xb, rows, r0=0, tokens=None, a_full=None, block=256):
+def oracle_sample(wl, Wb, Xb, rows, r0=0, tokens=None, a_full=None, block=256, search_tokens=None):
     """Time the CPU oracle, as it stands, on a bounded sample of one layer:
-    the statistics over ``tokens`` tokens (all by default; the cost is linear
-    in tokens), the search of ``rows`` rows starting at r0 over all N tokens
-    and every alpha, and their pack; scaled to the whole layer by tokens and
-    rows. With a token slice the search reads ``a_full``, the statistics of
-    all tokens (computed once by the caller). Returns (layer seconds, seconds
-    actually spent)."""
+    the statistics over ``tokens`` tokens (all by default), the search of
+    ``rows`` rows starting at r0 over every alpha and ``search_tokens``
+    tokens (all by default), and their pack; scaled to the whole layer by
+    tokens and rows (the statistics' cost is linear in tokens, the search's
+    in rows times tokens, the pack's in rows). With a token slice the search
+    reads ``a_full``, the statistics of all tokens (computed once by the
+    caller). Returns (layer seconds, seconds actually spent)."""
     from oracle import awq_oracle as O
     tokens = wl.N if tokens is None else min(tokens, wl.N)
+    search_tokens = wl.N if search_tokens is None else min(search_tokens, wl.N)
     t0 = time.perf_counter()
     a = O.act_stats(Xb[:tokens])
     t_stats = time.perf_counter() - t0
     if tokens < wl.N:
         a = a_full  # the search needs the statistics of all tokens
-    t_rows = 0.0
+    Xs = Xb[:search_tokens]
+    t_search = t_pack = 0.0
     idx = (r0 + np.arange(rows)) % wl.d_out
     for b0 in range(0, rows, block):
         sel = idx[b0:b0 + block]
         t0 = time.perf_counter()
-        res = O.search(Wb, Xb, a, wl.bits, wl.group, wl.symmetric, wl.n_alpha, rows=sel)
+        res = O.search(Wb, Xs, a, wl.bits, wl.group, wl.symmetric, wl.n_alpha, rows=sel)
+        t1 = time.perf_counter()
         O.pack(Wb[sel], res["s_best"], wl.bits, wl.group, wl.symmetric)
-        t_rows += time.perf_counter() - t0
-    t_layer = t_stats * (wl.N / tokens) + t_rows * (wl.d_out / rows)
-    return t_layer, t_stats + t_rows
+        t_pack += time.perf_counter() - t1
+        t_search += t1 - t0
+    t_layer = (t_stats * (wl.N / tokens) + t_search * (wl.d_out / rows) * (wl.N / search_tokens)
+               + t_pack * (wl.d_out / rows))
+    return t_layer, t_stats + t_search + t_pack
 
 
 def single_thread():
@@ -884,7 +902,9 @@ def run_reference(args, wl, world):
     all tokens and alphas, the slice moving from step to step), scaled to the
     whole layer; inputs generated once, before the steps."""
     Wb, Xb = make_inputs(wl)
-    rows = args.ref_rows if args.ref_rows else sample_rows(wl, 3.0)
+    rows, search_tokens = ref_sample(wl, REF_STEP_S)
+    if args.ref_rows:
+        rows, search_tokens = args.ref_rows, wl.N
     tokens = min(wl.N, args.ref_tokens)
     K = args.steps
     times, spent = [], []
@@ -892,15 +912,17 @@ def run_reference(args, wl, world):
         from oracle import awq_oracle as O
         a_full = O.act_stats(Xb) if tokens < wl.N else None
         for k in range(args.warmup + K):
-            t_layer, sp = oracle_sample(wl, Wb, Xb, rows, r0=(k * rows) % wl.d_out, tokens=tokens, a_full=a_full)
+            t_layer, sp = oracle_sample(wl, Wb, Xb, rows, r0=(k * rows) % wl.d_out, tokens=tokens, a_full=a_full,
+                                        search_tokens=search_tokens)
             if k >= args.warmup:
                 times.append(t_layer)
                 spent.append(sp)
     ms = 1e3 * sum(times) / K
     value = wl.n_alpha / (ms * 1e-3)
-    sample = (f"per step: statistics of {tokens} of {wl.N} tokens (scaled by tokens), search and pack of "
-              f"{rows} of {wl.d_out} rows x {wl.n_alpha} alphas over all tokens (scaled by rows); float64 numpy, "
-              f"BLAS limited to 1 thread")
+    over = "all tokens" if search_tokens == wl.N else f"{search_tokens} of {wl.N} tokens (scaled by tokens)"
+    sample = (f"per step: statistics of {tokens} of {wl.N} tokens (scaled by tokens), search of "
+              f"{rows} of {wl.d_out} rows x {wl.n_alpha} alphas over {over} and their pack (scaled by rows); "
+              f"float64 numpy, BLAS limited to 1 thread")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms, 2), "extrapolated": True,
@@ -922,7 +944,8 @@ def main():
     ap.add_argument("--form", default="auto", choices=["auto", "direct", "gram"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=None,
-                    help="rows of W per step of the oracle arm (default: about 3 s of single-thread work)")
+                    help="rows of W per step of the oracle arm, searched over all tokens (default: about "
+                         "REF_STEP_S s of single-thread work, over a token slice where 8 rows would exceed it)")
     ap.add_argument("--ref-tokens", type=int, default=8192, help="tokens of the oracle arm's statistics sample")
     ap.add_argument("--cpu-rows", type=int, default=None,
                     help="rows of W in the CPU baseline's sample (default: about 15 s of single-thread work)")
