@@ -980,7 +980,7 @@ extern "C" awq_status awq_act_stats_noalloc(const void* X, int64_t N, int64_t d_
 
 // ===================================================================== inference side
 namespace {
-constexpr int kW4TargetCtas = 148;  // split K until the tiles cover this many CTAs
+constexpr int kW4TargetCtas = 148;  // CTAs of the W4A16 grid: one per SM
 
 struct W4Plan {
   int bn, bk, n_mb, n_nb, n_kb;
