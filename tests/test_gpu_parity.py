@@ -127,6 +127,8 @@ SMALL = {
     "g256_300x1024_N520": custom(300, 1024, 520, group=256, seed=8),
     "g8_sym4_40x64_N1": custom(40, 64, 1, bits=4, symmetric=True, group=8, seed=9),
     "tokens_gt_din_129x256_N2000": custom(129, 256, 2000, seed=10),
+    # G' of 91 tiles on 74 CTA pairs: the last wave's 17 tiles run as 4 K pieces each
+    "gram_tail_64x3328_N512": custom(64, 3328, 512, seed=14),
 }
 
 
@@ -136,10 +138,30 @@ def test_search_small_auto(name):
     print(name, out)
 
 
-@pytest.mark.parametrize("name", ["C1", "ragged_200x384_N300", "sym3_g64_130x512_N77", "g256_300x1024_N520"])
+@pytest.mark.parametrize("name", ["C1", "ragged_200x384_N300", "sym3_g64_130x512_N77", "g256_300x1024_N520",
+                                  "gram_tail_64x3328_N512"])
 @pytest.mark.parametrize("form", ["direct", "gram"])
 def test_search_small_forced_form(name, form):
     run_case(SMALL[name], form=form, check_rows=False)
+
+
+def test_gram_tail_pieces_match_direct_form():
+    """The Gram form with its last wave split in K (the pieces' fp32 partials
+    summed by the fix-up) gives the direct form's losses, row by row, to the
+    bf16 rounding of G'."""
+    wl = SMALL["gram_tail_64x3328_N512"]
+    Wb, Xb = make_inputs(wl)
+    W, X = to_device(Wb), to_device(Xb)
+    a = awq.act_stats(X)
+    rows = {}
+    for form in ("direct", "gram"):
+        cfg = awq.make_cfg(wl.bits, wl.group, wl.symmetric, wl.n_alpha, form=form)
+        res = awq.search_scales(W, X, a, cfg, row_losses=True)
+        torch.cuda.synchronize()
+        awq.workspace_error(res["ws"])
+        rows[form] = res["row_losses"].cpu().numpy().astype(np.float64)
+    rel = np.abs(rows["gram"] - rows["direct"]) / np.abs(rows["direct"])
+    assert rel.max() < LOSS_RTOL, rel.max()
 
 
 def test_delta_weight_stack_elementwise():

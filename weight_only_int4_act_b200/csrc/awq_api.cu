@@ -23,6 +23,7 @@ namespace {
 constexpr size_t kAlign = 1024;
 // search workspace header: [0, 4) device error word, [256, 260) tile counter of the GEMMs
 constexpr size_t kTileCounterOffset = 256;
+constexpr long long kGramMaxPairs = 74;  // CTA pairs of the G' product (148 SMs)
 constexpr int kStatsTargetBlocks = 148 * 4;  // one wave at 4 resident blocks per SM
 constexpr int kGroupN = 8;
 // raster width (column tiles) of the CTA-pair contraction: with 16, concurrent
@@ -121,7 +122,7 @@ struct SearchLayout {
   long long M;      // rows of the dW stack
   int n_blocks_n;   // column tiles of the contraction
   int n_red_chunks; // blocks per alpha in the row reduction
-  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_seg, off_rows64, off_ext, off_g, total;
+  size_t off_s, off_inv, off_dw, off_part, off_blk, off_loss64, off_seg, off_rows64, off_ext, off_g, off_gpart, total;
 };
 
 // sum over 256-wide column blocks J of width(J) * min(d_in, 256 (J + 1)): the
@@ -170,6 +171,8 @@ SearchLayout search_layout(int64_t d_out, int64_t d_in, int64_t N, const awq_qcf
   L.off_ext = off;    off += ext_bytes(d_in);  // per tensor: column extremes and candidate extremes
   if (L.form == AWQ_FORM_GRAM) {
     L.off_g = off;    off += align_up((size_t)d_in * d_in * 2);
+    L.off_gpart = off;  // G' last wave split in K: at most one fp32 256 x 256 piece per pair
+    off += align_up((size_t)kGramMaxPairs * PAIR_BM * PAIR_BN * sizeof(float));
   }
   L.total = off;
   return L;
@@ -335,7 +338,27 @@ awq_status run_gemm_pair(const void* A, long long M, long long lda, const void* 
     return AWQ_ERR_CUDA;
   if (cudaMemsetAsync(args.tile_counter, 0, sizeof(int), st) != cudaSuccess) return AWQ_ERR_CUDA;
   const long long pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
+  // G' (tiles of equal K): a last wave of R <= pairs / 2 tiles runs as R x S
+  // pieces of K / S steps (S = pairs / R, at least 2 steps a piece)
+  args.tail_first = (int)tiles;
+  args.tail_split = 1;
+  long long R = 0;
+  if (MODE == EPI_STORE && tri == TRI_LOWER_STORE && args.tail_part && tiles > pairs) {
+    R = tiles % pairs;
+    const long long n_kb = cdiv(K, GEMM_BK);
+    long long S = R > 0 ? pairs / R : 0;
+    if (S > n_kb / 2) S = n_kb / 2;
+    if (R > 0 && S >= 2 && R * S <= kGramMaxPairs) {
+      args.tail_first = (int)(tiles - R);
+      args.tail_split = (int)S;
+    } else {
+      R = 0;
+    }
+  }
   gemm_pair_bf16_tcgen05<MODE, MN><<<(unsigned)(2 * pairs), GEMM_THREADS, PAIR_SMEM_BYTES, st>>>(ta, tb, args);
+  awq_status rs = launch_status();
+  if (rs != AWQ_OK || R == 0) return rs;
+  gram_tail_fixup<<<dim3((unsigned)R, (unsigned)(PAIR_BM * PAIR_BN / 1024)), 256, 0, st>>>(args);
   return launch_status();
 }
 
@@ -547,6 +570,7 @@ awq_status awq_step_gram(const void* X, int64_t d_out, int64_t d_in, int64_t N, 
   ga.ldC = d_in;
   ga.err = at<int>(ws, 0);
   ga.tile_counter = at<int>(ws, kTileCounterOffset);
+  ga.tail_part = at<float>(ws, L.off_gpart);
   GemmExtents ext;
   ext.C = (long long)d_in * d_in;
   // G = X^T X with both operands read transposed from X [N, d_in] (MN-major)

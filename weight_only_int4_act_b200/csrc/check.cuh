@@ -46,6 +46,7 @@ enum BoundsSite : int {
   BS_W4_Y,          // w4a16_gemm_tcgen05: Y stores
   BS_W4_P,          // w4a16_gemm_tcgen05: stream-K partial stores
   BS_W4_FIXUP,      // w4a16_streamk_reduce: split tiles, partials and Y
+  BS_GRAM_FIX,      // gram_tail_fixup: partial pieces and G'
   BS_FOLD_S,        // fold_inv_scales_kernel: s
   BS_FOLD_P,        // fold_inv_scales_kernel: the folded tensor
   BS_SELFTEST = 0x7F,

@@ -22,6 +22,12 @@
 //              writes them into both CTAs' rings and arrives on both sfull;
 //              sempty (even CTA) counts 10 readers (even MMA + 4 even
 //              epilogue warps + odd producer + 4 odd epilogue warps).
+// Last wave of the G' product: when the tiles leave a last wave of at most
+// half the pairs, those R tiles are handed out as R x S pieces of K/S steps
+// each (S = pairs / R), piece-major so that the pieces in flight together
+// cover the same K range of every split tile (the pairs keep sweeping X in
+// step, and each slice of X is still fetched once); each piece is written as
+// fp32 partials and gram_tail_fixup adds the S pieces of a tile in K order.
 // All waits are bounded (ptx.cuh); the CTAs meet at a cluster barrier before
 // freeing TMEM (both CTAs, cta_group::2) and exiting.
 #pragma once
@@ -50,6 +56,29 @@ __device__ __forceinline__ void pair_tri_coords(int t, int& mb, int& nb) {
   while ((long long)q * (q + 1) / 2 > t) --q;
   mb = q;
   nb = t - q * (q + 1) / 2;
+}
+
+// Work item i of the counter: a whole tile, or piece (part q of split tile
+// tail_first + r) when i >= tail_first, with its K steps [k0, k1) and slab.
+struct PairWork {
+  int t, k0, k1, slab;  // slab < 0: a whole tile
+};
+__device__ __forceinline__ PairWork pair_work(const GemmArgs& a, int i, int num_kb_tile) {
+  PairWork w;
+  if (i < a.tail_first) {
+    w.t = i;
+    w.k0 = 0;
+    w.k1 = num_kb_tile;
+    w.slab = -1;
+    return w;
+  }
+  const int R = a.num_tiles - a.tail_first, j = i - a.tail_first;
+  const int q = j / R, r = j - q * R;
+  w.t = a.tail_first + r;
+  w.k0 = q * num_kb_tile / a.tail_split;
+  w.k1 = (q + 1) * num_kb_tile / a.tail_split;
+  w.slab = j;  // = q R + r
+  return w;
 }
 
 __device__ __forceinline__ void pair_tile_coords(int t, const GemmArgs& a, int& mb, int& nb) {
@@ -121,7 +150,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   cluster_sync();  // barriers of both CTAs initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int num_tiles = args.num_tiles;
+  // work items: whole tiles, then the pieces of the split last-wave tiles
+  const int num_tiles = args.tail_first + (args.num_tiles - args.tail_first) * args.tail_split;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -153,9 +183,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         }
         if (t < 0) break;
         int mb, nb;
-        pair_tile_coords(t, args, mb, nb);
-        const int num_kb = gemm_num_kb(args, nb);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        pair_tile_coords(t < args.tail_first ? t : args.tail_first + (t - args.tail_first) % max(1, args.num_tiles - args.tail_first),
+                         args, mb, nb);
+        const PairWork wk = pair_work(args, t, gemm_num_kb(args, nb));
+        for (int kb = wk.k0; kb < wk.k1; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.err, ERR_WAIT_EMPTY)) {
             ok = false;
             break;
@@ -219,9 +250,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * PAIR_BN;
         int mb, nb;
-        pair_tile_coords(t, args, mb, nb);
-        const int num_kb = gemm_num_kb(args, nb);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        pair_tile_coords(t < args.tail_first ? t : args.tail_first + (t - args.tail_first) % max(1, args.num_tiles - args.tail_first),
+                         args, mb, nb);
+        const PairWork wk = pair_work(args, t, gemm_num_kb(args, nb));
+        for (int kb = wk.k0; kb < wk.k1; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, args.err, ERR_WAIT_FULL)) {
             ok = false;
             break;
@@ -236,7 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                                    : desc_kmajor_sw128(a_base + k * 32);
             const uint64_t bd = MN ? desc_mnmajor_sw128(b_base + k * 2048, GEMM_MN_CHUNK)
                                    : desc_kmajor_sw128(b_base + k * 32);
-            mma_bf16_pair(d_tmem, ad, bd, IDESC, (kb | k) != 0);
+            mma_bf16_pair(d_tmem, ad, bd, IDESC, (kb != wk.k0) || (k != 0));
           }
           mma_commit_pair(empty_bar(stage), 0x3);
           if (++stage == PAIR_STAGES) {
@@ -272,7 +304,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       }
       if (t < 0) break;
       int mb, nb;
-      pair_tile_coords(t, args, mb, nb);
+      pair_tile_coords(t < args.tail_first ? t : args.tail_first + (t - args.tail_first) % max(1, args.num_tiles - args.tail_first),
+                       args, mb, nb);
+      const int slab = t < args.tail_first ? -1 : t - args.tail_first;
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       const bool ready = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, args.err, ERR_WAIT_TFULL);
@@ -306,7 +340,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           // G' = 2 G on strictly lower blocks, G on diagonal blocks (TRI_LOWER_STORE)
           const int col = n0 + c * 32;
           const float scale = nb < mb ? 2.0f : 1.0f;
-          if (m < args.M) {
+          if (slab >= 0) {
+            // a K piece of a split tile: fp32 partial, row 128 rank + row_in_tile of its slab
+            float4* prow = reinterpret_cast<float4*>(
+                args.tail_part + ((long long)slab * PAIR_BM + (int)rank * 128 + row_in_tile) * PAIR_BN + c * 32);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              prow[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                    __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          } else if (m < args.M) {
             __nv_bfloat16* crow = args.C + (long long)m * args.ldC + col;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -354,6 +396,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, GEMM_TMEM_COLS);
+  }
+}
+
+// Block (r, y) finishes 1024 elements (4 per thread, 256 apart: coalesced)
+// of split tile tail_first + r: its tail_split K pieces added in K order,
+// times 2 off the diagonal blocks, rounded to bf16 into C.
+__global__ void __launch_bounds__(256) gram_tail_fixup(const GemmArgs a) {
+  const int R = a.num_tiles - a.tail_first, r = blockIdx.x;
+  if (r >= R) return;
+  int mb, nb;
+  pair_tri_coords(a.tail_first + r, mb, nb);
+  const float scale = nb < mb ? 2.0f : 1.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int e = blockIdx.y * 1024 + k * 256 + threadIdx.x;  // row-major in the 256 x 256 tile
+    if (e >= PAIR_BM * PAIR_BN) continue;
+    const int row = e / PAIR_BN, col = e - row * PAIR_BN;
+    const long long m = (long long)mb * PAIR_BM + row, cn = (long long)nb * PAIR_BN + col;
+    if (m >= a.M || cn >= a.N) continue;
+    float acc = 0.0f;
+    for (int q = 0; q < a.tail_split; ++q) {
+      const long long i = ((long long)(q * R + r) * PAIR_BM + row) * PAIR_BN + col;
+      if (AWQ_IDX_OK(i, (long long)R * a.tail_split * PAIR_BM * PAIR_BN, BS_GRAM_FIX)) acc += a.tail_part[i];
+    }
+    if (AWQ_IDX_OK(m * a.ldC + cn, (long long)a.M * a.ldC, BS_GRAM_FIX)) a.C[m * a.ldC + cn] = __float2bfloat16_rn(scale * acc);
   }
 }
 

@@ -83,6 +83,9 @@ struct GemmArgs {
   int* err;                    // device error word
   int* tile_counter;           // dynamic tile counter, zero at launch
   int group;                   // TRI_DIAG_STORE: quantisation group size (divides 256)
+  int tail_first;              // pair G' only: tiles from here on are split in K (num_tiles: no split)
+  int tail_split;              // K pieces per split tile (tail_first < num_tiles)
+  float* tail_part;            // fp32 partial tiles [(num_tiles - tail_first) * tail_split][256 x 256]
 };
 
 // Number of tiles of the lower block triangle with n_blocks_m row tiles of
