@@ -99,6 +99,22 @@ def test_sample_rows_bounded():
     assert bench.sample_rows(configs.WORKLOADS["C1"], 15.0) == 256  # the whole small layer
 
 
+def test_reference_step_sample_bounded():
+    """The oracle arm's step: rows as sample_rows gives them, and a token
+    slice (a multiple of 1024) only where 8 rows over every token would
+    overrun the step's budget; the estimated work then stays within it."""
+    from awq_inputs import configs
+    for key, wl in configs.WORKLOADS.items():
+        rows, tokens = bench.ref_sample(wl, bench.REF_STEP_S)
+        assert rows == bench.sample_rows(wl, bench.REF_STEP_S), key
+        assert tokens == wl.N or (tokens % 1024 == 0 and 1024 <= tokens < wl.N), key
+        if tokens < wl.N:
+            assert rows == 8, key
+        est = rows * wl.d_in * tokens * bench.ORACLE_ROW_COST_S
+        assert est <= bench.REF_STEP_S or tokens == 1024 or (rows == 8 and tokens == wl.N), key
+    assert bench.ref_sample(configs.WORKLOADS["C5"], bench.REF_STEP_S)[1] < 65536  # C5 runs on a token slice
+
+
 def test_pack_parity_against_stored_digests():
     """bench's code check: the oracle's own pack of C1 passes; a code changed
     away from the rounding-boundary band fails it; a code changed inside the
