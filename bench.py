@@ -234,9 +234,25 @@ def tri_macs_per_row(d_in, block=256):
     return float(sum(min(block, d_in - j0) * min(d_in, j0 + block) for j0 in range(0, d_in, block)))
 
 
-def launches_per_step(form, n_alpha):
-    # stats 2 + scales 1 + fake quant 1 + (Gram 1) + contraction 1 + reduce 2 + pack 1
-    return 8 + (1 if form == "gram" else 0)
+def gram_tail_split(d_in, N, pairs=74):
+    """Whether the Gram product's last wave runs as K pieces (and so ends with
+    the fix-up launch): the library's rule for a last wave of R <= pairs / 2
+    tiles of 256 x 256, S = pairs // R pieces of at least two 64-token steps."""
+    nbm = -(-d_in // 256)
+    tiles = nbm * (nbm + 1) // 2
+    pairs = min(tiles, pairs)
+    if tiles <= pairs:
+        return False
+    R = tiles % pairs
+    if R == 0:
+        return False
+    S = min(pairs // R, -(-N // 64) // 2)
+    return S >= 2 and R * S <= 74
+
+
+def launches_per_step(form, n_alpha, d_in=0, N=0):
+    # stats 2 + scales 1 + fake quant 1 + (Gram 1, + its last-wave fix-up) + contraction 1 + reduce 2 + pack 1
+    return 8 + ((2 if gram_tail_split(d_in, N) else 1) if form == "gram" else 0)
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -651,7 +667,7 @@ def run_ours(args, rank, world, local_rank):
                     "step k+1's inputs are copied on a second stream while step k computes; working set "
                     "(the candidate stack) larger than L2, no flush",
         "parity": parity,
-        "gpu_launches": launches_per_step(form, n_a) * K,
+        "gpu_launches": launches_per_step(form, n_a, d_in, N) * K,
         "clocks": clk,
         "wall_s_timed_region": round(t_wall, 3),
     }

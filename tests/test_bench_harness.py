@@ -54,6 +54,8 @@ def test_tri_macs_matches_block_count():
 def test_launch_count():
     assert bench.launches_per_step("direct", 20) == 8
     assert bench.launches_per_step("gram", 20) == 9
+    assert bench.launches_per_step("gram", 20, 4096, 4096) == 9      # C2: a last wave of 62 of 74 pairs
+    assert bench.launches_per_step("gram", 20, 8192, 65536) == 10    # C5: 528 = 7 x 74 + 10 tiles, split in K
 
 
 def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
