@@ -756,7 +756,7 @@ def run_only(args):
             fn = lambda: B._check(L.awq_step_gram(ctypes.c_void_p(X.data_ptr()), d_out, d_in, N, cptr, wsp, wsn, st),  # noqa: E731
                                   "gram")
             flops = 2.0 * N * tri
-            kernels = ["gemm_bf16_tcgen05 (EPI_STORE, MN-major, lower block triangle)"]
+            kernels = ["gemm_pair_bf16_tcgen05 (EPI_STORE, MN-major, lower block triangle)", "gram_tail_fixup"]
         else:
             fn = lambda: B._check(L.awq_step_contract(ctypes.c_void_p(X.data_ptr()), d_out, d_in, N, cptr, wsp,  # noqa: E731
                                                       wsn, st), "contract")
